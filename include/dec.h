@@ -1,0 +1,268 @@
+/*
+ * dec.h - C ABI of the batched single-token decoder step (B200, sm_100a).
+ *
+ * One call of dec_step advances B independent streams of a pre-norm
+ * transformer decoder by one token each: embedding (+ learned position),
+ * per layer pre-norm, fused Q/K/V projection, KV-cache append, causal
+ * self-attention over the stream's cache, output projection and residual,
+ * (Whisper) cross-attention over precomputed encoder K/V, the FFN, and the
+ * final norm with the tied LM head and the greedy argmax.
+ *
+ * Sources (docs.rs source pages), cited by crate, file and item:
+ *   [wa-dec]  whisper-apr 0.3.3 src/model/decoder_generated.rs
+ *   [wa-cuda] whisper-apr 0.3.0 src/cuda/impl_generated.rs
+ *   [focr]    franken_ocr 0.8.0 src/native_engine/decoder_qwen2.rs
+ *   [cera]    cera 0.5.4 src/model/whisper.rs
+ *   [q8]      lattice-inference 0.4.0 src/forward/cpu_q8.rs
+ *
+ * Conventions for every entry point:
+ *   - Pointers documented "host" are read during the call only; pointers
+ *     documented "device" must be CUDA device memory on the handle's device
+ *     and stay valid until the work queued on `stream` has run.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   - All argument checks run before any work is queued; a call that returns
+ *     an error other than DEC_ECUDA has changed no state.
+ *   - A handle is not thread-safe: serialise calls on one handle.
+ *   - dec_last_error(h) returns a message for the last failed call on h.
+ */
+#ifndef DEC_H
+#define DEC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dec_status {
+    DEC_OK = 0,
+    DEC_EINVAL = 1,     /* null pointer, bad shape, bad config, duplicate slot */
+    DEC_ERANGE = 2,     /* token >= vocab, position outside the position table */
+    DEC_EOVERFLOW = 3,  /* cache_lens[b] + 1 > max_cache_len (cache full) */
+    DEC_ESTATE = 4,     /* cache_lens[b] differs from the slot's length, slot not prefilled */
+    DEC_ENOMEM = 5,     /* device or pinned host allocation failed */
+    DEC_ECUDA = 6,      /* a CUDA call failed; the message names it */
+    DEC_ETIMEOUT = 7    /* a bounded device wait gave up (reported by dec_sync) */
+} dec_status;
+
+enum { DEC_FAMILY_WHISPER = 0, DEC_FAMILY_QWEN2 = 1 };
+enum { DEC_PROJ_F32 = 0, DEC_PROJ_W8A8 = 1, DEC_PROJ_W8A32 = 2 };
+
+#define DEC_MAX_BATCH 128
+
+/*
+ * Model and capacity description.
+ *   family      DEC_FAMILY_WHISPER: LayerNorm with bias, learned positions,
+ *               self- and cross-attention, GELU(tanh) FFN, all projections
+ *               biased ([cera] `decode_step_into`).
+ *               DEC_FAMILY_QWEN2: RMSNorm, NEOX RoPE, SwiGLU MLP, bias on
+ *               q/k/v only ([focr] `qwen2_decode_step`).
+ *   head_dim    must be 64; d_model = n_heads * 64.
+ *   d_ff        FFN width, a multiple of 16 (16-byte int8 weight loads).
+ *   max_pos     whisper: rows of the learned position table (positions must
+ *               be < max_pos); qwen2: exclusive bound on positions (RoPE table rows).
+ *   enc_len     whisper: encoder rows attended by cross-attention; 0 for qwen2.
+ *   proj_fmt    DEC_PROJ_F32 (f32 weights), DEC_PROJ_W8A8 (int8 weights and
+ *               int8 per-row activations, int32 accumulation; qwen2 only) or
+ *               DEC_PROJ_W8A32 (int8 weights, f32 activations; whisper only).
+ *   norm_eps    1e-5 (LayerNorm) / 1e-6 (RMSNorm) in the configs of the pages.
+ *   rope_theta  RoPE base (qwen2), e.g. 1e6.
+ *   max_slots   number of independent streams the handle holds caches for.
+ *   max_cache_len  rows per stream and layer in the self-attention cache.
+ */
+typedef struct dec_config {
+    int32_t family;
+    int32_t n_layers;
+    int32_t d_model;
+    int32_t n_heads;
+    int32_t head_dim;
+    int32_t d_ff;
+    int32_t vocab;
+    int32_t max_pos;
+    int32_t enc_len;
+    int32_t proj_fmt;
+    float norm_eps;
+    float rope_theta;
+    int32_t max_slots;
+    int32_t max_cache_len;
+} dec_config;
+
+/*
+ * One projection y = x W^T (+ b), W [out, in] row-major (PyTorch layout), host memory.
+ *   w      float when proj_fmt == DEC_PROJ_F32, int8_t (codes in [-127, 127]) otherwise
+ *   scale  per-output-row f32 scale s_n of the int8 formats (W_nk = s_n q_nk); NULL for f32
+ *   bias   f32 [out] or NULL (must be NULL exactly where the family has no bias)
+ */
+typedef struct dec_proj {
+    const void* w;
+    const float* scale;
+    const float* bias;
+} dec_proj;
+
+/*
+ * One layer's weights (host). Whisper uses norm1 (self-attn LN), q/k/v/o,
+ * norm2 (cross-attn LN), xq/xk/xv/xo, norm3 (FFN LN), fc1 [d_ff, d], fc2 [d, d_ff].
+ * Qwen2 uses norm1 (input RMSNorm weight), q/k/v/o, norm2 (post-attention RMSNorm
+ * weight), gate and up [d_ff, d], down [d, d_ff]. Unused members are ignored.
+ */
+typedef struct dec_layer_weights {
+    const float* norm1_w;
+    const float* norm1_b;
+    dec_proj q, k, v, o;
+    const float* norm2_w;
+    const float* norm2_b;
+    dec_proj xq, xk, xv, xo;
+    const float* norm3_w;
+    const float* norm3_b;
+    dec_proj fc1, fc2;
+    dec_proj gate, up, down;
+} dec_layer_weights;
+
+/*
+ * Model weights (host). tok_emb [vocab, d] f32 is both the embedding and the
+ * tied LM head ([focr] module doc: tied embeddings; [cera] proj_w). pos_emb
+ * [max_pos, d] f32 for whisper, NULL for qwen2. final_w / final_b: final norm
+ * (final_b NULL for RMSNorm). layers: [n_layers].
+ */
+typedef struct dec_weights {
+    const float* tok_emb;
+    const float* pos_emb;
+    const float* final_w;
+    const float* final_b;
+    const dec_layer_weights* layers;
+} dec_weights;
+
+typedef struct dec_handle dec_handle;
+
+/*
+ * Validate cfg, copy and pack all weights into device memory on the current
+ * CUDA device, and allocate every KV cache and workspace once ([wa-dec]
+ * `DecoderScratch`: per-token buffers allocated once). The caller may free
+ * its weight buffers after the call. On error *out is NULL and nothing leaks;
+ * the message is available from dec_last_error(NULL) on the same thread.
+ */
+dec_status dec_create(const dec_config* cfg, const dec_weights* w, dec_handle** out);
+
+/* Free everything the handle owns. Synchronises the device first. NULL is a no-op. */
+dec_status dec_destroy(dec_handle* h);
+
+/* Message of the last failed call on h (or of the last failed dec_create on
+ * this thread when h is NULL). Never NULL; "" when there was no error. */
+const char* dec_last_error(const dec_handle* h);
+
+/*
+ * Reset stream `slot` and run `n_tokens` tokens (host int32) at positions
+ * 0..n_tokens-1 through the decoder, filling its self-attention cache
+ * ([focr] `forward_prefill_seed` seeds the cache; here each row goes through
+ * the m = 1 step). Whisper: `enc_hidden` (device f32 [enc_len, d]) is
+ * required; cross-attention K and V are computed from it once per layer
+ * ([cera] `precompute_cross_attention`: K = enc Wk^T + bk, V = enc Wv^T + bv).
+ * Qwen2: enc_hidden must be NULL. n_tokens may be 0 (cross K/V only).
+ * last_logits (device f32 [vocab] or NULL) receives the last row's logits;
+ * the last row's argmax becomes the slot's greedy continuation token.
+ */
+dec_status dec_prefill(dec_handle* h, int32_t slot, const int32_t* tokens, int32_t n_tokens,
+                       const float* enc_hidden, float* last_logits, void* stream);
+
+/*
+ * Write rows [start_pos, start_pos + n_rows) of every layer's self-attention
+ * K and V for `slot` and set the slot length to start_pos + n_rows
+ * ([focr] `Qwen2KvCache::seed`). k and v are device f32 [n_layers, n_rows,
+ * n_heads * 64], token-major (already rotated K for qwen2). Requires
+ * start_pos <= the slot's current length (no holes). Rows are copied bit for bit.
+ * Whisper slots still need dec_prefill (n_tokens may be 0) for cross K/V.
+ */
+dec_status dec_kv_append(dec_handle* h, int32_t slot, int32_t start_pos, int32_t n_rows,
+                         const float* k, const float* v, void* stream);
+
+/*
+ * One decode step over `batch` streams.
+ *   slots       host int32 [batch], distinct slot ids, or NULL for 0..batch-1
+ *   tokens      host int32 [batch] input tokens, or NULL to feed each slot its
+ *               own previous greedy pick (set by the last dec_step/dec_prefill
+ *               on that slot; DEC_ESTATE if it has none)
+ *   positions   host int32 [batch]: learned-position row (whisper) or RoPE
+ *               position (qwen2) of the new token ([focr] batched step:
+ *               positions passed explicitly so the caller stays in charge)
+ *   cache_lens  host int32 [batch]: must equal each slot's current length
+ *               ([cera] `decode_step_into` checks seq_len == pos); the new
+ *               K/V row is written at that row and attention covers rows
+ *               0..cache_lens[b]; on success each slot's length grows by one
+ *   logits      device f32 [batch, vocab] or NULL (not written)
+ *   argmax      device int32 [batch] or NULL: greedy pick, lowest index on ties
+ *               ([focr] `argmax`)
+ * Queues the work on `stream` and returns without synchronising.
+ */
+dec_status dec_step(dec_handle* h, int32_t batch, const int32_t* slots, const int32_t* tokens,
+                    const int32_t* positions, const int32_t* cache_lens, float* logits,
+                    int32_t* argmax, void* stream);
+
+/*
+ * dec_step with host result buffers: queues the step, copies logits (host f32
+ * [batch, vocab] or NULL) and argmax (host int32 [batch] or NULL) back, and
+ * synchronises `stream` before returning. Host buffers may be pageable;
+ * pinned buffers copy faster.
+ */
+dec_status dec_step_host(dec_handle* h, int32_t batch, const int32_t* slots,
+                         const int32_t* tokens, const int32_t* positions,
+                         const int32_t* cache_lens, float* logits_host, int32_t* argmax_host,
+                         void* stream);
+
+/* Current length (cached rows) of `slot` as tracked by the handle. */
+dec_status dec_slot_len(const dec_handle* h, int32_t slot, int32_t* len);
+
+/*
+ * Copy rows [start, start + n) of layer `layer`'s self-attention K and V of
+ * `slot` into device buffers k_out, v_out (f32 [n, n_heads * 64], token-major).
+ * Rows at or beyond the slot length hold whatever was last written there.
+ */
+dec_status dec_kv_read(dec_handle* h, int32_t slot, int32_t layer, int32_t start, int32_t n,
+                       float* k_out, float* v_out, void* stream);
+
+/* Copy the residual stream after the last layer of the most recent dec_step
+ * (before the final norm), f32 [batch, d_model], into device `out`. */
+dec_status dec_hidden(dec_handle* h, float* out, int32_t batch, void* stream);
+
+/* Synchronise `stream` and report device-side failures (DEC_ETIMEOUT when a
+ * bounded wait inside a kernel gave up). Clears the device status word. */
+dec_status dec_sync(dec_handle* h, void* stream);
+
+/*
+ * Kernel-level entry points (no handle). They run one kernel of the step on
+ * caller-provided device buffers, for testing each kernel on its own.
+ */
+
+/*
+ * Split-K decode attention over head-first caches ([focr] `decode_attn_head`:
+ * s_j = q . k_j / 8, max-subtracted softmax, sum_j p_j v_j; a row whose
+ * softmax sum is not finite and positive gives zeros, [q8] full-attention step).
+ *   q        device f32 [batch, n_heads, 64]
+ *   k, v     device f32 [batch, n_heads, ld, 64] (head-first, ld rows per head)
+ *   lens     device int32 [batch]: keys attended per stream (rows 0..lens[b]-1),
+ *            0 <= lens[b] <= ld; lens[b] == 0 gives zeros
+ *   out      device f32 [batch, n_heads, 64]
+ *   workspace device scratch of at least dec_attention_workspace_size(batch,
+ *            n_heads, ld) bytes, 16-byte aligned; its first
+ *            batch * n_heads int32 must be zero before the first call (each call
+ *            leaves them zero again)
+ */
+size_t dec_attention_workspace_size(int32_t batch, int32_t n_heads, int32_t ld);
+dec_status dec_attention(const float* q, const float* k, const float* v, const int32_t* lens,
+                         int32_t batch, int32_t n_heads, int32_t ld, float* out,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * int8 x int8 -> int32 dot products acc[m, n] = sum_k xq[m, k] * wq[n, k]
+ * (the accumulator of [focr] `gemv_i8_bias_prequant`). xq device int8 [m, kdim],
+ * wq device int8 [n, kdim], acc device int32 [m, n]; kdim a multiple of 16,
+ * 1 <= m <= 64.
+ */
+dec_status dec_i8_dot(const int8_t* xq, const int8_t* wq, int32_t m, int32_t n, int32_t kdim,
+                      int32_t* acc, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DEC_H */

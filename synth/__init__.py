@@ -122,7 +122,7 @@ MODELS: Dict[str, ModelConfig] = {
                        head_dim=64, d_ff=2048, vocab=51865, max_pos=448, enc_len=1500,
                        proj_fmt=PROJ_F32, norm_eps=1e-5),
     "qwen2_0_5b_int8": _m(name="qwen2_0_5b_int8", family="qwen2", n_layers=24, d_model=1024,
-                          n_heads=16, head_dim=64, d_ff=2816, vocab=151936, max_pos=1 << 20,
+                          n_heads=16, head_dim=64, d_ff=2816, vocab=151936, max_pos=32768,
                           enc_len=0, proj_fmt=PROJ_W8A8, norm_eps=1e-6, rope_theta=1e6),
     "whisper_large_v3_w8a32": _m(name="whisper_large_v3_w8a32", family="whisper", n_layers=32,
                                  d_model=1280, n_heads=20, head_dim=64, d_ff=5120, vocab=51866,
@@ -136,10 +136,10 @@ MODELS: Dict[str, ModelConfig] = {
                              n_heads=3, head_dim=64, d_ff=320, vocab=997, max_pos=64, enc_len=37,
                              proj_fmt=PROJ_W8A32, norm_eps=1e-5),
     "tiny_qwen2": _m(name="tiny_qwen2", family="qwen2", n_layers=2, d_model=128, n_heads=2,
-                     head_dim=64, d_ff=352, vocab=1009, max_pos=1 << 20, enc_len=0,
+                     head_dim=64, d_ff=352, vocab=1009, max_pos=32768, enc_len=0,
                      proj_fmt=PROJ_W8A8, norm_eps=1e-6, rope_theta=1e6),
     "small_qwen2": _m(name="small_qwen2", family="qwen2", n_layers=3, d_model=256, n_heads=4,
-                      head_dim=64, d_ff=704, vocab=4099, max_pos=1 << 20, enc_len=0,
+                      head_dim=64, d_ff=704, vocab=4099, max_pos=32768, enc_len=0,
                       proj_fmt=PROJ_W8A8, norm_eps=1e-6, rope_theta=1e6),
 }
 

@@ -251,3 +251,15 @@ def test_identity_structured_qwen2_mlp_closed_form():
     mq, am = oracle.quantize_rows_i8_te(np.concatenate([m, np.zeros(f - d, F32)])[None, :])
     y = (mq[0, :d].astype(np.float64) * 127 * float(am[0]) * float(inv)).astype(F32)
     np.testing.assert_allclose(hidden[0], (x0 + y).astype(F32), rtol=1e-6, atol=1e-7)
+
+
+def test_quantisation_margin_diagnostic():
+    """The oracle's near-tie diagnostic reports 0 for an exact .5 tie and the true
+    distance otherwise, and changes no result."""
+    cfg, W = _model("tiny_qwen2")
+    dec = oracle.OracleDecoder(W, 8)
+    dec._margins = np.full(2, np.inf)
+    x = np.array([[127.0, 2.5, 1.0], [127.0, 2.25, 1.0]], F32)
+    q, a = dec._quant(x)
+    assert np.array_equal(q, oracle.quantize_rows_i8_te(x)[0])
+    assert dec._margins[0] == 0.0 and dec._margins[1] == 0.25

@@ -1,0 +1,235 @@
+"""ctypes binding of the C ABI in include/dec.h (argument marshalling only).
+
+Every step of the decoder runs in the CUDA library libdec.so built from csrc/.
+There is no CPU path: if the library is missing this module raises on import.
+Device buffers are passed as raw pointers (e.g. torch.Tensor.data_ptr()), streams
+as cudaStream_t handles (e.g. torch.cuda.current_stream().cuda_stream).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdec.so")
+
+DEC_OK, DEC_EINVAL, DEC_ERANGE, DEC_EOVERFLOW, DEC_ESTATE, DEC_ENOMEM, DEC_ECUDA, DEC_ETIMEOUT = range(8)
+STATUS_NAMES = ["DEC_OK", "DEC_EINVAL", "DEC_ERANGE", "DEC_EOVERFLOW", "DEC_ESTATE", "DEC_ENOMEM",
+                "DEC_ECUDA", "DEC_ETIMEOUT"]
+FAMILY = {"whisper": 0, "qwen2": 1}
+PROJ = {"f32": 0, "w8a8": 1, "w8a32": 2}
+
+# Every symbol include/dec.h declares.
+EXPORTS = ["dec_create", "dec_destroy", "dec_last_error", "dec_prefill", "dec_kv_append", "dec_step",
+           "dec_step_host", "dec_slot_len", "dec_kv_read", "dec_hidden", "dec_sync",
+           "dec_attention_workspace_size", "dec_attention", "dec_i8_dot"]
+
+
+class DecError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        self.status = status
+        name = STATUS_NAMES[status] if 0 <= status < len(STATUS_NAMES) else str(status)
+        super().__init__(f"{name}: {msg}")
+
+
+class DecConfig(C.Structure):
+    _fields_ = [("family", C.c_int32), ("n_layers", C.c_int32), ("d_model", C.c_int32),
+                ("n_heads", C.c_int32), ("head_dim", C.c_int32), ("d_ff", C.c_int32),
+                ("vocab", C.c_int32), ("max_pos", C.c_int32), ("enc_len", C.c_int32),
+                ("proj_fmt", C.c_int32), ("norm_eps", C.c_float), ("rope_theta", C.c_float),
+                ("max_slots", C.c_int32), ("max_cache_len", C.c_int32)]
+
+
+class DecProj(C.Structure):
+    _fields_ = [("w", C.c_void_p), ("scale", C.c_void_p), ("bias", C.c_void_p)]
+
+
+class DecLayerWeights(C.Structure):
+    _fields_ = [("norm1_w", C.c_void_p), ("norm1_b", C.c_void_p),
+                ("q", DecProj), ("k", DecProj), ("v", DecProj), ("o", DecProj),
+                ("norm2_w", C.c_void_p), ("norm2_b", C.c_void_p),
+                ("xq", DecProj), ("xk", DecProj), ("xv", DecProj), ("xo", DecProj),
+                ("norm3_w", C.c_void_p), ("norm3_b", C.c_void_p),
+                ("fc1", DecProj), ("fc2", DecProj),
+                ("gate", DecProj), ("up", DecProj), ("down", DecProj)]
+
+
+class DecWeights(C.Structure):
+    _fields_ = [("tok_emb", C.c_void_p), ("pos_emb", C.c_void_p), ("final_w", C.c_void_p),
+                ("final_b", C.c_void_p), ("layers", C.POINTER(DecLayerWeights))]
+
+
+def load_library(path: str = LIB_PATH) -> C.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"CUDA decoder library not built: {path} is missing "
+                          "(run transformer_decoder_kv_b200.build.build())")
+    lib = C.CDLL(path)
+    vp, i32, pi32 = C.c_void_p, C.c_int32, C.POINTER(C.c_int32)
+    sig = {
+        "dec_create": (C.c_int, [C.POINTER(DecConfig), C.POINTER(DecWeights), C.POINTER(vp)]),
+        "dec_destroy": (C.c_int, [vp]),
+        "dec_last_error": (C.c_char_p, [vp]),
+        "dec_prefill": (C.c_int, [vp, i32, pi32, i32, vp, vp, vp]),
+        "dec_kv_append": (C.c_int, [vp, i32, i32, i32, vp, vp, vp]),
+        "dec_step": (C.c_int, [vp, i32, pi32, pi32, pi32, pi32, vp, vp, vp]),
+        "dec_step_host": (C.c_int, [vp, i32, pi32, pi32, pi32, pi32, vp, vp, vp]),
+        "dec_slot_len": (C.c_int, [vp, i32, pi32]),
+        "dec_kv_read": (C.c_int, [vp, i32, i32, i32, i32, vp, vp, vp]),
+        "dec_hidden": (C.c_int, [vp, vp, i32, vp]),
+        "dec_sync": (C.c_int, [vp, vp]),
+        "dec_attention_workspace_size": (C.c_size_t, [i32, i32, i32]),
+        "dec_attention": (C.c_int, [vp, vp, vp, vp, i32, i32, i32, vp, vp, C.c_size_t, vp]),
+        "dec_i8_dot": (C.c_int, [vp, vp, i32, i32, i32, vp, vp]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib: Optional[C.CDLL] = None
+
+
+def lib() -> C.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = load_library()
+    return _lib
+
+
+def _i32arr(values) -> Optional[C.Array]:
+    if values is None:
+        return None
+    a = np.ascontiguousarray(np.asarray(values, dtype=np.int32))
+    return (C.c_int32 * len(a))(*a.tolist())
+
+
+def _ptr(a) -> Optional[int]:
+    """Pointer of a numpy array (host) or a tensor-like with data_ptr() (device); None stays None."""
+    if a is None:
+        return None
+    if hasattr(a, "data_ptr"):
+        return a.data_ptr()
+    return a.ctypes.data
+
+
+class Decoder:
+    """One handle of the CUDA decoder (dec_create ... dec_destroy)."""
+
+    def __init__(self, cfg, weights: dict, max_slots: int, max_cache_len: int):
+        self._lib = lib()
+        c = DecConfig(FAMILY[cfg.family], cfg.n_layers, cfg.d_model, cfg.n_heads, cfg.head_dim,
+                      cfg.d_ff, cfg.vocab, cfg.max_pos, cfg.enc_len, PROJ[cfg.proj_fmt],
+                      float(cfg.norm_eps), float(cfg.rope_theta), max_slots, max_cache_len)
+        self.cfg = cfg
+        self.max_slots = max_slots
+        self.max_cache_len = max_cache_len
+        keep = []
+
+        def arr(x, dtype):
+            if x is None:
+                return None
+            a = np.ascontiguousarray(x, dtype=dtype)
+            keep.append(a)
+            return a.ctypes.data
+
+        wdt = np.float32 if cfg.proj_fmt == "f32" else np.int8
+
+        def proj(p):
+            if p is None:
+                return DecProj(None, None, None)
+            return DecProj(arr(p["w"], wdt), arr(p["s"], np.float32), arr(p["b"], np.float32))
+
+        layers = (DecLayerWeights * cfg.n_layers)()
+        for i, L in enumerate(weights["layers"]):
+            lw = layers[i]
+            lw.norm1_w = arr(L.get("norm1_w"), np.float32)
+            lw.norm1_b = arr(L.get("norm1_b"), np.float32)
+            lw.norm2_w = arr(L.get("norm2_w"), np.float32)
+            lw.norm2_b = arr(L.get("norm2_b"), np.float32)
+            lw.norm3_w = arr(L.get("norm3_w"), np.float32)
+            lw.norm3_b = arr(L.get("norm3_b"), np.float32)
+            for name in ("q", "k", "v", "o", "xq", "xk", "xv", "xo", "fc1", "fc2", "gate", "up", "down"):
+                setattr(lw, name, proj(L.get(name)))
+        w = DecWeights(arr(weights["tok_emb"], np.float32), arr(weights.get("pos_emb"), np.float32),
+                       arr(weights["final_w"], np.float32), arr(weights.get("final_b"), np.float32),
+                       layers)
+        h = C.c_void_p()
+        st = self._lib.dec_create(C.byref(c), C.byref(w), C.byref(h))
+        del keep
+        if st != DEC_OK:
+            raise DecError(st, self._lib.dec_last_error(None).decode())
+        self._h = h
+
+    # -- helpers --
+    def _check(self, st: int):
+        if st != DEC_OK:
+            raise DecError(st, self._lib.dec_last_error(self._h).decode())
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.dec_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- the C ABI --
+    def prefill(self, slot: int, tokens: Sequence[int], enc_hidden=None, last_logits=None, stream: int = 0):
+        toks = _i32arr(tokens) if len(tokens) else None
+        self._check(self._lib.dec_prefill(self._h, slot, toks, len(tokens), _ptr(enc_hidden),
+                                          _ptr(last_logits), stream))
+
+    def kv_append(self, slot: int, start: int, n_rows: int, k, v, stream: int = 0):
+        self._check(self._lib.dec_kv_append(self._h, slot, start, n_rows, _ptr(k), _ptr(v), stream))
+
+    def step(self, batch: int, slots, tokens, positions, cache_lens, logits=None, argmax=None,
+             stream: int = 0):
+        self._check(self._lib.dec_step(self._h, batch, _i32arr(slots), _i32arr(tokens),
+                                       _i32arr(positions), _i32arr(cache_lens), _ptr(logits),
+                                       _ptr(argmax), stream))
+
+    def step_host(self, batch: int, slots, tokens, positions, cache_lens, logits_host=None,
+                  argmax_host=None, stream: int = 0):
+        self._check(self._lib.dec_step_host(self._h, batch, _i32arr(slots), _i32arr(tokens),
+                                            _i32arr(positions), _i32arr(cache_lens),
+                                            _ptr(logits_host), _ptr(argmax_host), stream))
+
+    def slot_len(self, slot: int) -> int:
+        n = C.c_int32()
+        self._check(self._lib.dec_slot_len(self._h, slot, C.byref(n)))
+        return n.value
+
+    def kv_read(self, slot: int, layer: int, start: int, n: int, k_out, v_out, stream: int = 0):
+        self._check(self._lib.dec_kv_read(self._h, slot, layer, start, n, _ptr(k_out), _ptr(v_out), stream))
+
+    def hidden(self, out, batch: int, stream: int = 0):
+        self._check(self._lib.dec_hidden(self._h, _ptr(out), batch, stream))
+
+    def sync(self, stream: int = 0):
+        self._check(self._lib.dec_sync(self._h, stream))
+
+
+def attention(q, k, v, lens, batch: int, n_heads: int, ld: int, out, workspace, workspace_bytes: int,
+              stream: int = 0):
+    st = lib().dec_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(lens), batch, n_heads, ld, _ptr(out),
+                             _ptr(workspace), workspace_bytes, stream)
+    if st != DEC_OK:
+        raise DecError(st, "dec_attention failed")
+
+
+def attention_workspace_size(batch: int, n_heads: int, ld: int) -> int:
+    return int(lib().dec_attention_workspace_size(batch, n_heads, ld))
+
+
+def i8_dot(xq, wq, m: int, n: int, kdim: int, acc, stream: int = 0):
+    st = lib().dec_i8_dot(_ptr(xq), _ptr(wq), m, n, kdim, _ptr(acc), stream)
+    if st != DEC_OK:
+        raise DecError(st, "dec_i8_dot failed")

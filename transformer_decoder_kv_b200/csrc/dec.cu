@@ -1,0 +1,885 @@
+// C ABI of the batched single-token decoder step (see include/dec.h).
+//
+// Host side: validation before any launch, weight packing at create time, one
+// launch sequence per step on the caller's stream (programmatic dependent launch
+// between kernels), and the handle's bookkeeping of slot lengths.
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <type_traits>
+#include <vector>
+
+#include "../../include/dec.h"
+#include "attention.cuh"
+#include "common.cuh"
+#include "gemv.cuh"
+#include "gemv_launch.cuh"
+#include "misc.cuh"
+
+using namespace dec;
+
+namespace {
+
+constexpr int kMetaRing = 8;
+constexpr int kMaxSplits = 32;
+
+thread_local std::string g_create_error;
+
+struct LayerDev {
+    float *n1w = nullptr, *n1b = nullptr, *n2w = nullptr, *n2b = nullptr, *n3w = nullptr, *n3b = nullptr;
+    void* wqkv = nullptr;
+    float *sqkv = nullptr, *bqkv = nullptr;
+    void* wo = nullptr;
+    float *so = nullptr, *bo = nullptr;
+    void *wxq = nullptr, *wxk = nullptr, *wxv = nullptr, *wxo = nullptr;
+    float *sxq = nullptr, *sxk = nullptr, *sxv = nullptr, *sxo = nullptr;
+    float *bxq = nullptr, *bxk = nullptr, *bxv = nullptr, *bxo = nullptr;
+    void *w1 = nullptr, *w2 = nullptr;
+    float *s1 = nullptr, *s2 = nullptr, *b1 = nullptr, *b2 = nullptr;
+    void *wg = nullptr, *wu = nullptr, *wd = nullptr;
+    float *sg = nullptr, *su = nullptr, *sd = nullptr;
+};
+
+}  // namespace
+
+struct dec_handle {
+    dec_config cfg{};
+    int device = 0;
+    int num_sms = 148;
+    std::vector<void*> dallocs;
+    std::vector<void*> hallocs;
+    float *tok_emb = nullptr, *pos_emb = nullptr, *final_w = nullptr, *final_b = nullptr;
+    float2* rope = nullptr;
+    std::vector<LayerDev> layers;
+    float *kc = nullptr, *vc = nullptr, *xkc = nullptr, *xvc = nullptr;
+    long long self_slot_stride = 0, self_layer_stride = 0, cross_slot_stride = 0, cross_layer_stride = 0;
+    int max_batch = 0;
+    // workspace
+    float *x = nullptr, *q = nullptr, *ctx = nullptr, *ffn = nullptr, *xq = nullptr;
+    float* part = nullptr;
+    int* counters = nullptr;
+    unsigned long long* keys = nullptr;
+    int* head_counter = nullptr;
+    int* last_tok = nullptr;
+    int* dev_err = nullptr;
+    StepMeta* dmeta = nullptr;
+    StepMeta* hmeta[kMetaRing] = {};
+    cudaEvent_t hev[kMetaRing] = {};
+    int ring = 0;
+    // host view of the slots
+    std::vector<int> slot_len;
+    std::vector<char> has_tok, has_cross;
+    int last_batch = 0;
+    float* stage_logits = nullptr;   // dec_step_host result staging
+    int* stage_argmax = nullptr;
+    std::string err;
+};
+
+namespace {
+
+dec_status fail(dec_handle* h, dec_status st, const std::string& msg) {
+    if (h)
+        h->err = msg;
+    else
+        g_create_error = msg;
+    return st;
+}
+
+dec_status cuda_fail(dec_handle* h, cudaError_t e, const char* what) {
+    return fail(h, DEC_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+#define DEC_CUDA(h, call)                                    \
+    do {                                                     \
+        cudaError_t e_ = (call);                             \
+        if (e_ != cudaSuccess) return cuda_fail((h), e_, #call); \
+    } while (0)
+
+template <typename T>
+dec_status dalloc(dec_handle* h, T** p, size_t bytes) {
+    void* q = nullptr;
+    if (bytes == 0) bytes = 16;
+    cudaError_t e = cudaMalloc(&q, bytes);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(h, DEC_ENOMEM, "cudaMalloc of " + std::to_string(bytes) + " bytes failed");
+    }
+    h->dallocs.push_back(q);
+    *p = static_cast<T*>(q);
+    return DEC_OK;
+}
+
+template <typename T>
+dec_status upload(dec_handle* h, T** dst, const void* src, size_t bytes) {
+    dec_status st = dalloc(h, dst, bytes);
+    if (st != DEC_OK) return st;
+    DEC_CUDA(h, cudaMemcpy(*dst, src, bytes, cudaMemcpyHostToDevice));
+    return DEC_OK;
+}
+
+#define DEC_TRY(x)                        \
+    do {                                  \
+        dec_status s_ = (x);              \
+        if (s_ != DEC_OK) return s_;      \
+    } while (0)
+
+size_t wbytes(const dec_config& c) { return c.proj_fmt == DEC_PROJ_F32 ? 4 : 1; }
+
+// Upload a projection: weights [out, in], optional scales [out] and bias [out].
+dec_status upload_proj(dec_handle* h, const dec_proj& p, int out, int in, bool want_bias, void** w, float** s,
+                       float** b, const char* name) {
+    const dec_config& c = h->cfg;
+    if (!p.w) return fail(h, DEC_EINVAL, std::string("missing weights for ") + name);
+    if (c.proj_fmt != DEC_PROJ_F32 && !p.scale) return fail(h, DEC_EINVAL, std::string("missing scales for ") + name);
+    if (want_bias != (p.bias != nullptr))
+        return fail(h, DEC_EINVAL, std::string(want_bias ? "missing bias for " : "unexpected bias for ") + name);
+    DEC_TRY(upload(h, w, p.w, size_t(out) * in * wbytes(c)));
+    if (c.proj_fmt != DEC_PROJ_F32) DEC_TRY(upload(h, s, p.scale, size_t(out) * 4));
+    if (p.bias) DEC_TRY(upload(h, b, p.bias, size_t(out) * 4));
+    return DEC_OK;
+}
+
+// Fused q|k|v panel [3d, d] with its scales and biases (franken_ocr decoder_qwen2.rs, `concat_qkv`).
+dec_status upload_qkv(dec_handle* h, const dec_layer_weights& L, LayerDev& D) {
+    const dec_config& c = h->cfg;
+    const int d = c.d_model;
+    const size_t wb = wbytes(c), mat = size_t(d) * d * wb;
+    const dec_proj* ps[3] = {&L.q, &L.k, &L.v};
+    for (int i = 0; i < 3; ++i) {
+        if (!ps[i]->w) return fail(h, DEC_EINVAL, "missing q/k/v weights");
+        if (c.proj_fmt != DEC_PROJ_F32 && !ps[i]->scale) return fail(h, DEC_EINVAL, "missing q/k/v scales");
+        if (!ps[i]->bias) return fail(h, DEC_EINVAL, "missing q/k/v bias");
+    }
+    DEC_TRY(dalloc(h, &D.wqkv, 3 * mat));
+    DEC_TRY(dalloc(h, &D.bqkv, size_t(3) * d * 4));
+    if (c.proj_fmt != DEC_PROJ_F32) DEC_TRY(dalloc(h, &D.sqkv, size_t(3) * d * 4));
+    for (int i = 0; i < 3; ++i) {
+        DEC_CUDA(h, cudaMemcpy(static_cast<char*>(D.wqkv) + i * mat, ps[i]->w, mat, cudaMemcpyHostToDevice));
+        DEC_CUDA(h, cudaMemcpy(D.bqkv + i * d, ps[i]->bias, size_t(d) * 4, cudaMemcpyHostToDevice));
+        if (D.sqkv) DEC_CUDA(h, cudaMemcpy(D.sqkv + i * d, ps[i]->scale, size_t(d) * 4, cudaMemcpyHostToDevice));
+    }
+    return DEC_OK;
+}
+
+dec_status validate_config(const dec_config& c) {
+    auto bad = [](const std::string& m) { return fail(nullptr, DEC_EINVAL, m); };
+    if (c.family != DEC_FAMILY_WHISPER && c.family != DEC_FAMILY_QWEN2) return bad("unknown family");
+    if (c.head_dim != 64) return bad("head_dim must be 64");
+    if (c.n_heads < 1 || c.d_model != c.n_heads * 64) return bad("d_model must equal n_heads * 64");
+    if (c.n_layers < 1) return bad("n_layers must be >= 1");
+    if (c.d_ff < 16 || c.d_ff % 16) return bad("d_ff must be a positive multiple of 16");
+    if (c.vocab < 1) return bad("vocab must be >= 1");
+    if (c.max_pos < 1) return bad("max_pos must be >= 1");
+    if (c.max_slots < 1) return bad("max_slots must be >= 1");
+    if (c.max_cache_len < 1) return bad("max_cache_len must be >= 1");
+    if (!(c.norm_eps > 0.0f)) return bad("norm_eps must be > 0");
+    if (c.family == DEC_FAMILY_WHISPER) {
+        if (c.enc_len < 1) return bad("whisper needs enc_len >= 1");
+        if (c.proj_fmt != DEC_PROJ_F32 && c.proj_fmt != DEC_PROJ_W8A32)
+            return bad("whisper supports f32 or w8a32 projections");
+    } else {
+        if (c.proj_fmt != DEC_PROJ_W8A8) return bad("qwen2 supports w8a8 projections");
+        if (!(c.rope_theta > 0.0f)) return bad("rope_theta must be > 0");
+        if (c.max_pos > (1 << 22)) return bad("max_pos too large for the RoPE table");
+    }
+    return DEC_OK;
+}
+
+// NEOX RoPE table: angle = pos * theta^(-2i/64) in double, cos and sin rounded to f32.
+dec_status build_rope(dec_handle* h) {
+    const dec_config& c = h->cfg;
+    std::vector<float2> t(size_t(c.max_pos) * 32);
+    for (int p = 0; p < c.max_pos; ++p)
+        for (int i = 0; i < 32; ++i) {
+            const double inv = std::pow(double(c.rope_theta), -2.0 * i / 64.0);
+            const double ang = double(p) * inv;
+            t[size_t(p) * 32 + i] = make_float2(float(std::cos(ang)), float(std::sin(ang)));
+        }
+    return upload(h, &h->rope, t.data(), t.size() * sizeof(float2));
+}
+
+// ------------------------------------------------------------------ launches
+
+template <typename K, typename... Args>
+cudaError_t launch(K kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+
+template <typename WT, bool I8, int PRO, int EPI, int MAP>
+dec_status gemv(dec_handle* h, const GemvArgs& a, cudaStream_t st) {
+    cudaError_t e = gemv_launch<WT, I8, PRO, EPI, MAP>(h->num_sms, a, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "projection kernel launch");
+    return DEC_OK;
+}
+
+// Whisper projections exist as f32 or W8A32.
+template <int PRO, int EPI, int MAP>
+dec_status gemv_whisper(dec_handle* h, const GemvArgs& a, cudaStream_t st) {
+    if (h->cfg.proj_fmt == DEC_PROJ_F32) return gemv<float, false, PRO, EPI, MAP>(h, a, st);
+    return gemv<int8_t, false, PRO, EPI, MAP>(h, a, st);
+}
+
+// Split count for one attention launch: minimise (waves x tiles per CTA).
+int choose_splits(const dec_handle* h, int rows, int max_tiles) {
+    if (max_tiles <= 1) return 1;
+    const int slots = h->num_sms * 2;
+    int best = 1;
+    double best_cost = 1e30;
+    for (int s = 1; s <= std::min(kMaxSplits, max_tiles); ++s) {
+        const int tps = (max_tiles + s - 1) / s;
+        const int eff = (max_tiles + tps - 1) / tps;
+        if (eff != s) continue;
+        const double waves = std::ceil(double(rows) * s / slots);
+        const double cost = waves * (tps + 1.5) + (s > 1 ? 0.5 : 0.0);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = s;
+        }
+    }
+    return best;
+}
+
+dec_status attention(dec_handle* h, AttnArgs a, int B, int max_keys, cudaStream_t st) {
+    static int configured = 0;
+    if (!configured) {
+        DEC_CUDA(h, cudaFuncSetAttribute(k_attention, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kAttnSmemBytes)));
+        configured = 1;
+    }
+    const int max_tiles = (max_keys + kAttnTile - 1) / kAttnTile;
+    a.S = choose_splits(h, B * a.H, max_tiles);
+    DEC_CUDA(h, launch(k_attention, dim3(a.S, a.H, B), dim3(kAttnThreads), kAttnSmemBytes, st, a));
+    return DEC_OK;
+}
+
+GemvArgs base_args(dec_handle* h, int B) {
+    GemvArgs g{};
+    g.B = B;
+    g.eps = h->cfg.norm_eps;
+    g.meta = h->dmeta;
+    return g;
+}
+
+// One step for the batch described in h->dmeta (already uploaded).
+dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int* argmax, cudaStream_t st) {
+    const dec_config& c = h->cfg;
+    const int d = c.d_model, F = c.d_ff, H = c.n_heads;
+    DEC_CUDA(h, launch(k_embed, dim3(B), dim3(128), 0, st, (const float*)h->tok_emb, (const float*)h->pos_emb,
+                       (const StepMeta*)h->dmeta, (const int*)h->last_tok, h->x, d));
+    for (int l = 0; l < c.n_layers; ++l) {
+        const LayerDev& L = h->layers[l];
+        float* kc = h->kc + l * h->self_layer_stride;
+        float* vc = h->vc + l * h->self_layer_stride;
+        // ---- q|k|v with the cache append ----
+        GemvArgs g = base_args(h, B);
+        g.x = h->x;
+        g.x_ld = d;
+        g.norm_w = L.n1w;
+        g.norm_b = L.n1b;
+        g.K = d;
+        g.N = 3 * d;
+        g.W = L.wqkv;
+        g.scale = L.sqkv;
+        g.bias = L.bqkv;
+        g.out = h->q;
+        g.out_ld = d;
+        g.kc = kc;
+        g.vc = vc;
+        g.slot_stride = h->self_slot_stride;
+        g.ld = c.max_cache_len;
+        g.d = d;
+        if (c.family == DEC_FAMILY_WHISPER) {
+            DEC_TRY((gemv_whisper<PRO_LN, EPI_QKV, MAP_ADJ>(h, g, st)));
+        } else {
+            g.rope = h->rope;
+            DEC_TRY((gemv<int8_t, true, PRO_RMS, EPI_QKV, MAP_ROPE>(h, g, st)));
+        }
+        // ---- self-attention over rows 0..len ----
+        AttnArgs at{};
+        at.q = h->q;
+        at.q_bstride = d;
+        at.k = kc;
+        at.v = vc;
+        at.slot_stride = h->self_slot_stride;
+        at.ld = c.max_cache_len;
+        at.H = H;
+        at.mode = ATTN_SELF;
+        at.meta = h->dmeta;
+        at.out = h->ctx;
+        at.out_bstride = d;
+        at.part = h->part;
+        at.counters = h->counters;
+        at.err = h->dev_err;
+        DEC_TRY(attention(h, at, B, max_len_plus1, st));
+        // ---- output projection + residual ----
+        g = base_args(h, B);
+        g.x = h->ctx;
+        g.x_ld = d;
+        g.K = d;
+        g.N = d;
+        g.W = L.wo;
+        g.scale = L.so;
+        g.bias = L.bo;
+        g.out = h->x;
+        g.out_ld = d;
+        if (c.family == DEC_FAMILY_WHISPER) {
+            DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st)));
+        } else {
+            DEC_TRY((gemv<int8_t, true, PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st)));
+        }
+        if (c.family == DEC_FAMILY_WHISPER) {
+            // ---- cross-attention block ----
+            g = base_args(h, B);
+            g.x = h->x;
+            g.x_ld = d;
+            g.norm_w = L.n2w;
+            g.norm_b = L.n2b;
+            g.K = d;
+            g.N = d;
+            g.W = L.wxq;
+            g.scale = L.sxq;
+            g.bias = L.bxq;
+            g.out = h->xq;
+            g.out_ld = d;
+            DEC_TRY((gemv_whisper<PRO_LN, EPI_STORE, MAP_ADJ>(h, g, st)));
+            at.q = h->xq;
+            at.k = h->xkc + l * h->cross_layer_stride;
+            at.v = h->xvc + l * h->cross_layer_stride;
+            at.slot_stride = h->cross_slot_stride;
+            at.ld = c.enc_len;
+            at.mode = ATTN_CROSS;
+            at.n_fixed = c.enc_len;
+            DEC_TRY(attention(h, at, B, c.enc_len, st));
+            g = base_args(h, B);
+            g.x = h->ctx;
+            g.x_ld = d;
+            g.K = d;
+            g.N = d;
+            g.W = L.wxo;
+            g.scale = L.sxo;
+            g.bias = L.bxo;
+            g.out = h->x;
+            g.out_ld = d;
+            DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st)));
+            // ---- GELU FFN ----
+            g = base_args(h, B);
+            g.x = h->x;
+            g.x_ld = d;
+            g.norm_w = L.n3w;
+            g.norm_b = L.n3b;
+            g.K = d;
+            g.N = F;
+            g.W = L.w1;
+            g.scale = L.s1;
+            g.bias = L.b1;
+            g.out = h->ffn;
+            g.out_ld = F;
+            DEC_TRY((gemv_whisper<PRO_LN, EPI_GELU, MAP_ADJ>(h, g, st)));
+            g = base_args(h, B);
+            g.x = h->ffn;
+            g.x_ld = F;
+            g.K = F;
+            g.N = d;
+            g.W = L.w2;
+            g.scale = L.s2;
+            g.bias = L.b2;
+            g.out = h->x;
+            g.out_ld = d;
+            DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st)));
+        } else {
+            // ---- SwiGLU MLP ----
+            g = base_args(h, B);
+            g.x = h->x;
+            g.x_ld = d;
+            g.norm_w = L.n2w;
+            g.K = d;
+            g.N = F;
+            g.W = L.wg;
+            g.W2 = L.wu;
+            g.scale = L.sg;
+            g.scale2 = L.su;
+            g.out = h->ffn;
+            g.out_ld = F;
+            DEC_TRY((gemv<int8_t, true, PRO_RMS, EPI_SWIGLU, MAP_DUAL>(h, g, st)));
+            g = base_args(h, B);
+            g.x = h->ffn;
+            g.x_ld = F;
+            g.K = F;
+            g.N = d;
+            g.W = L.wd;
+            g.scale = L.sd;
+            g.out = h->x;
+            g.out_ld = d;
+            DEC_TRY((gemv<int8_t, true, PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st)));
+        }
+    }
+    // ---- final norm + tied head + greedy argmax ----
+    GemvArgs g = base_args(h, B);
+    g.x = h->x;
+    g.x_ld = d;
+    g.norm_w = h->final_w;
+    g.norm_b = h->final_b;
+    g.K = d;
+    g.N = c.vocab;
+    g.W = h->tok_emb;
+    g.out = logits;
+    g.out_ld = c.vocab;
+    g.keys = h->keys;
+    g.counter = h->head_counter;
+    g.argmax_out = argmax;
+    g.last_tok = h->last_tok;
+    if (c.family == DEC_FAMILY_WHISPER) {
+        DEC_TRY((gemv<float, false, PRO_LN, EPI_HEAD, MAP_ADJ>(h, g, st)));
+    } else {
+        DEC_TRY((gemv<float, false, PRO_RMS, EPI_HEAD, MAP_ADJ>(h, g, st)));
+    }
+    return DEC_OK;
+}
+
+// Upload the step description through the pinned ring.
+dec_status upload_meta(dec_handle* h, const StepMeta& m, cudaStream_t st) {
+    const int i = h->ring;
+    h->ring = (h->ring + 1) % kMetaRing;
+    DEC_CUDA(h, cudaEventSynchronize(h->hev[i]));
+    std::memcpy(h->hmeta[i], &m, sizeof(StepMeta));
+    DEC_CUDA(h, cudaMemcpyAsync(h->dmeta, h->hmeta[i], sizeof(StepMeta), cudaMemcpyHostToDevice, st));
+    DEC_CUDA(h, cudaEventRecord(h->hev[i], st));
+    return DEC_OK;
+}
+
+dec_status check_device(dec_handle* h) {
+    int cur = -1;
+    DEC_CUDA(h, cudaGetDevice(&cur));
+    if (cur != h->device) return fail(h, DEC_EINVAL, "the current CUDA device is not the handle's device");
+    return DEC_OK;
+}
+
+dec_status validate_step(dec_handle* h, int B, const int32_t* slots, const int32_t* tokens,
+                         const int32_t* positions, const int32_t* cache_lens, StepMeta& m, int& max_len) {
+    const dec_config& c = h->cfg;
+    if (B < 1 || B > h->max_batch)
+        return fail(h, DEC_EINVAL, "batch must be in [1, " + std::to_string(h->max_batch) + "]");
+    if (!positions || !cache_lens) return fail(h, DEC_EINVAL, "positions and cache_lens are required");
+    std::vector<char> seen(c.max_slots, 0);
+    m.B = B;
+    max_len = 0;
+    for (int b = 0; b < B; ++b) {
+        const int s = slots ? slots[b] : b;
+        if (s < 0 || s >= c.max_slots) return fail(h, DEC_EINVAL, "slot out of range");
+        if (seen[s]) return fail(h, DEC_EINVAL, "duplicate slot in batch");
+        seen[s] = 1;
+        if (tokens) {
+            if (tokens[b] < 0 || tokens[b] >= c.vocab)
+                return fail(h, DEC_ERANGE, "token " + std::to_string(tokens[b]) + " outside [0, vocab)");
+        } else if (!h->has_tok[s]) {
+            return fail(h, DEC_ESTATE, "slot " + std::to_string(s) + " has no previous greedy pick");
+        }
+        if (positions[b] < 0 || positions[b] >= c.max_pos)
+            return fail(h, DEC_ERANGE, "position " + std::to_string(positions[b]) + " outside [0, max_pos)");
+        if (cache_lens[b] != h->slot_len[s])
+            return fail(h, DEC_ESTATE, "cache_lens[" + std::to_string(b) + "] = " + std::to_string(cache_lens[b]) +
+                                           " but slot " + std::to_string(s) + " holds " +
+                                           std::to_string(h->slot_len[s]) + " rows");
+        if (cache_lens[b] + 1 > c.max_cache_len)
+            return fail(h, DEC_EOVERFLOW, "cache overflow: " + std::to_string(cache_lens[b]) + " + 1 > " +
+                                              std::to_string(c.max_cache_len));
+        if (c.family == DEC_FAMILY_WHISPER && !h->has_cross[s])
+            return fail(h, DEC_ESTATE, "slot " + std::to_string(s) + " has no cross-attention K/V (prefill it)");
+        m.slot[b] = s;
+        m.tok[b] = tokens ? tokens[b] : -1;
+        m.pos[b] = positions[b];
+        m.len[b] = cache_lens[b];
+        max_len = std::max(max_len, cache_lens[b] + 1);
+    }
+    return DEC_OK;
+}
+
+dec_status step_validated(dec_handle* h, const StepMeta& m, int max_len, float* logits, int* argmax,
+                          cudaStream_t st) {
+    DEC_TRY(upload_meta(h, m, st));
+    DEC_TRY(run_step(h, m.B, max_len, logits, argmax, st));
+    for (int b = 0; b < m.B; ++b) {
+        h->slot_len[m.slot[b]] += 1;
+        h->has_tok[m.slot[b]] = 1;
+    }
+    h->last_batch = m.B;
+    return DEC_OK;
+}
+
+}  // namespace
+
+// ===================================================================== C ABI
+
+extern "C" {
+
+const char* dec_last_error(const dec_handle* h) { return h ? h->err.c_str() : g_create_error.c_str(); }
+
+dec_status dec_destroy(dec_handle* h) {
+    if (!h) return DEC_OK;
+    cudaDeviceSynchronize();
+    for (void* p : h->dallocs) cudaFree(p);
+    for (void* p : h->hallocs) cudaFreeHost(p);
+    for (int i = 0; i < kMetaRing; ++i)
+        if (h->hev[i]) cudaEventDestroy(h->hev[i]);
+    delete h;
+    return DEC_OK;
+}
+
+static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_weights* w) {
+    const dec_config& c = *cfg;
+    const int d = c.d_model, F = c.d_ff, H = c.n_heads, L = c.n_layers;
+    const bool wh = c.family == DEC_FAMILY_WHISPER;
+    DEC_CUDA(h, cudaGetDevice(&h->device));
+    DEC_CUDA(h, cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device));
+    if (!w->tok_emb || !w->final_w || !w->layers) return fail(h, DEC_EINVAL, "missing embedding, final norm or layers");
+    if (wh && (!w->pos_emb || !w->final_b)) return fail(h, DEC_EINVAL, "whisper needs pos_emb and final_b");
+    DEC_TRY(upload(h, &h->tok_emb, w->tok_emb, size_t(c.vocab) * d * 4));
+    if (wh) {
+        DEC_TRY(upload(h, &h->pos_emb, w->pos_emb, size_t(c.max_pos) * d * 4));
+        DEC_TRY(upload(h, &h->final_b, w->final_b, size_t(d) * 4));
+    } else {
+        DEC_TRY(build_rope(h));
+    }
+    DEC_TRY(upload(h, &h->final_w, w->final_w, size_t(d) * 4));
+    h->layers.resize(L);
+    for (int l = 0; l < L; ++l) {
+        const dec_layer_weights& W = w->layers[l];
+        LayerDev& D = h->layers[l];
+        if (!W.norm1_w || !W.norm2_w) return fail(h, DEC_EINVAL, "missing norm weights");
+        DEC_TRY(upload(h, &D.n1w, W.norm1_w, size_t(d) * 4));
+        DEC_TRY(upload(h, &D.n2w, W.norm2_w, size_t(d) * 4));
+        DEC_TRY(upload_qkv(h, W, D));
+        if (wh) {
+            if (!W.norm1_b || !W.norm2_b || !W.norm3_w || !W.norm3_b)
+                return fail(h, DEC_EINVAL, "missing layer norm parameters");
+            DEC_TRY(upload(h, &D.n1b, W.norm1_b, size_t(d) * 4));
+            DEC_TRY(upload(h, &D.n2b, W.norm2_b, size_t(d) * 4));
+            DEC_TRY(upload(h, &D.n3w, W.norm3_w, size_t(d) * 4));
+            DEC_TRY(upload(h, &D.n3b, W.norm3_b, size_t(d) * 4));
+            DEC_TRY(upload_proj(h, W.o, d, d, true, &D.wo, &D.so, &D.bo, "o"));
+            DEC_TRY(upload_proj(h, W.xq, d, d, true, &D.wxq, &D.sxq, &D.bxq, "xq"));
+            DEC_TRY(upload_proj(h, W.xk, d, d, true, &D.wxk, &D.sxk, &D.bxk, "xk"));
+            DEC_TRY(upload_proj(h, W.xv, d, d, true, &D.wxv, &D.sxv, &D.bxv, "xv"));
+            DEC_TRY(upload_proj(h, W.xo, d, d, true, &D.wxo, &D.sxo, &D.bxo, "xo"));
+            DEC_TRY(upload_proj(h, W.fc1, F, d, true, &D.w1, &D.s1, &D.b1, "fc1"));
+            DEC_TRY(upload_proj(h, W.fc2, d, F, true, &D.w2, &D.s2, &D.b2, "fc2"));
+        } else {
+            DEC_TRY(upload_proj(h, W.o, d, d, false, &D.wo, &D.so, &D.bo, "o"));
+            float* nobias = nullptr;
+            DEC_TRY(upload_proj(h, W.gate, F, d, false, &D.wg, &D.sg, &nobias, "gate"));
+            DEC_TRY(upload_proj(h, W.up, F, d, false, &D.wu, &D.su, &nobias, "up"));
+            DEC_TRY(upload_proj(h, W.down, d, F, false, &D.wd, &D.sd, &nobias, "down"));
+        }
+    }
+    // caches
+    h->self_slot_stride = (long long)H * c.max_cache_len * 64;
+    h->self_layer_stride = h->self_slot_stride * c.max_slots;
+    const size_t self_bytes = size_t(L) * h->self_layer_stride * 4;
+    DEC_TRY(dalloc(h, &h->kc, self_bytes));
+    DEC_TRY(dalloc(h, &h->vc, self_bytes));
+    DEC_CUDA(h, cudaMemset(h->kc, 0, self_bytes));
+    DEC_CUDA(h, cudaMemset(h->vc, 0, self_bytes));
+    if (wh) {
+        h->cross_slot_stride = (long long)H * c.enc_len * 64;
+        h->cross_layer_stride = h->cross_slot_stride * c.max_slots;
+        const size_t cross_bytes = size_t(L) * h->cross_layer_stride * 4;
+        DEC_TRY(dalloc(h, &h->xkc, cross_bytes));
+        DEC_TRY(dalloc(h, &h->xvc, cross_bytes));
+    }
+    // workspace
+    h->max_batch = std::min(c.max_slots, DEC_MAX_BATCH);
+    const int MB = h->max_batch;
+    DEC_TRY(dalloc(h, &h->x, size_t(MB) * d * 4));
+    DEC_TRY(dalloc(h, &h->q, size_t(MB) * d * 4));
+    DEC_TRY(dalloc(h, &h->ctx, size_t(MB) * d * 4));
+    DEC_TRY(dalloc(h, &h->xq, size_t(MB) * d * 4));
+    DEC_TRY(dalloc(h, &h->ffn, size_t(MB) * F * 4));
+    DEC_TRY(dalloc(h, &h->part, size_t(MB) * H * kMaxSplits * kAttnPartStride * 4));
+    DEC_TRY(dalloc(h, &h->counters, size_t(MB) * H * 4));
+    DEC_CUDA(h, cudaMemset(h->counters, 0, size_t(MB) * H * 4));
+    DEC_TRY(dalloc(h, &h->keys, size_t(MB) * 8));
+    DEC_CUDA(h, cudaMemset(h->keys, 0, size_t(MB) * 8));
+    DEC_TRY(dalloc(h, &h->head_counter, 16));
+    DEC_CUDA(h, cudaMemset(h->head_counter, 0, 16));
+    DEC_TRY(dalloc(h, &h->last_tok, size_t(c.max_slots) * 4));
+    DEC_CUDA(h, cudaMemset(h->last_tok, 0, size_t(c.max_slots) * 4));
+    DEC_TRY(dalloc(h, &h->dev_err, 16));
+    DEC_CUDA(h, cudaMemset(h->dev_err, 0, 16));
+    DEC_TRY(dalloc(h, &h->dmeta, sizeof(StepMeta)));
+    DEC_TRY(dalloc(h, &h->stage_logits, size_t(MB) * c.vocab * 4));
+    DEC_TRY(dalloc(h, &h->stage_argmax, size_t(MB) * 4));
+    for (int i = 0; i < kMetaRing; ++i) {
+        void* p = nullptr;
+        if (cudaMallocHost(&p, sizeof(StepMeta)) != cudaSuccess) {
+            cudaGetLastError();
+            return fail(h, DEC_ENOMEM, "cudaMallocHost failed");
+        }
+        h->hallocs.push_back(p);
+        h->hmeta[i] = static_cast<StepMeta*>(p);
+        DEC_CUDA(h, cudaEventCreateWithFlags(&h->hev[i], cudaEventDisableTiming));
+    }
+    h->slot_len.assign(c.max_slots, 0);
+    h->has_tok.assign(c.max_slots, 0);
+    h->has_cross.assign(c.max_slots, 0);
+    DEC_CUDA(h, cudaDeviceSynchronize());
+    return DEC_OK;
+}
+
+dec_status dec_create(const dec_config* cfg, const dec_weights* w, dec_handle** out) {
+    g_create_error.clear();
+    if (!out) return fail(nullptr, DEC_EINVAL, "out is NULL");
+    *out = nullptr;
+    if (!cfg || !w) return fail(nullptr, DEC_EINVAL, "cfg and weights are required");
+    dec_status st = validate_config(*cfg);
+    if (st != DEC_OK) return st;
+    dec_handle* h = new dec_handle();
+    h->cfg = *cfg;
+    st = create_impl(h, cfg, w);
+    if (st != DEC_OK) {
+        g_create_error = h->err;
+        dec_destroy(h);
+        return st;
+    }
+    *out = h;
+    return DEC_OK;
+}
+
+dec_status dec_prefill(dec_handle* h, int32_t slot, const int32_t* tokens, int32_t n_tokens,
+                       const float* enc_hidden, float* last_logits, void* stream) {
+    if (!h) return DEC_EINVAL;
+    const dec_config& c = h->cfg;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (slot < 0 || slot >= c.max_slots) return fail(h, DEC_EINVAL, "slot out of range");
+    if (n_tokens < 0 || (n_tokens > 0 && !tokens)) return fail(h, DEC_EINVAL, "bad tokens");
+    if (n_tokens > c.max_cache_len) return fail(h, DEC_EOVERFLOW, "prefill longer than max_cache_len");
+    if (c.family == DEC_FAMILY_WHISPER) {
+        if (!enc_hidden) return fail(h, DEC_EINVAL, "whisper prefill needs enc_hidden");
+        if (n_tokens > c.max_pos) return fail(h, DEC_ERANGE, "prefill longer than the position table");
+    } else if (enc_hidden) {
+        return fail(h, DEC_EINVAL, "qwen2 has no cross-attention; enc_hidden must be NULL");
+    }
+    for (int i = 0; i < n_tokens; ++i)
+        if (tokens[i] < 0 || tokens[i] >= c.vocab) return fail(h, DEC_ERANGE, "token outside [0, vocab)");
+    DEC_TRY(check_device(h));
+    if (c.family == DEC_FAMILY_WHISPER) {
+        const int d = c.d_model;
+        for (int l = 0; l < c.n_layers; ++l) {
+            const LayerDev& L = h->layers[l];
+            float* ko = h->xkc + l * h->cross_layer_stride + slot * h->cross_slot_stride;
+            float* vo = h->xvc + l * h->cross_layer_stride + slot * h->cross_slot_stride;
+            dim3 grid((d + 63) / 64, (c.enc_len + 63) / 64);
+            if (c.proj_fmt == DEC_PROJ_F32) {
+                k_cross_kv<float><<<grid, 256, 0, st>>>(enc_hidden, (const float*)L.wxk, nullptr, L.bxk, ko, c.enc_len, d, d);
+                k_cross_kv<float><<<grid, 256, 0, st>>>(enc_hidden, (const float*)L.wxv, nullptr, L.bxv, vo, c.enc_len, d, d);
+            } else {
+                k_cross_kv<int8_t><<<grid, 256, 0, st>>>(enc_hidden, (const int8_t*)L.wxk, L.sxk, L.bxk, ko, c.enc_len, d, d);
+                k_cross_kv<int8_t><<<grid, 256, 0, st>>>(enc_hidden, (const int8_t*)L.wxv, L.sxv, L.bxv, vo, c.enc_len, d, d);
+            }
+            DEC_CUDA(h, cudaGetLastError());
+        }
+        h->has_cross[slot] = 1;
+    }
+    h->slot_len[slot] = 0;
+    h->has_tok[slot] = 0;
+    for (int i = 0; i < n_tokens; ++i) {
+        StepMeta m{};
+        m.B = 1;
+        m.slot[0] = slot;
+        m.tok[0] = tokens[i];
+        m.pos[0] = i;
+        m.len[0] = i;
+        float* lg = (i == n_tokens - 1) ? last_logits : nullptr;
+        DEC_TRY(step_validated(h, m, i + 1, lg, nullptr, st));
+    }
+    return DEC_OK;
+}
+
+dec_status dec_kv_append(dec_handle* h, int32_t slot, int32_t start_pos, int32_t n_rows, const float* k,
+                         const float* v, void* stream) {
+    if (!h) return DEC_EINVAL;
+    const dec_config& c = h->cfg;
+    if (slot < 0 || slot >= c.max_slots) return fail(h, DEC_EINVAL, "slot out of range");
+    if (n_rows < 0 || (n_rows > 0 && (!k || !v))) return fail(h, DEC_EINVAL, "bad rows");
+    if (start_pos < 0 || start_pos > h->slot_len[slot])
+        return fail(h, DEC_ESTATE, "start_pos must be within [0, slot length]");
+    if (start_pos + n_rows > c.max_cache_len) return fail(h, DEC_EOVERFLOW, "cache overflow");
+    DEC_TRY(check_device(h));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (n_rows > 0) {
+        dim3 grid(n_rows, c.n_layers);
+        k_kv_copy<<<grid, 128, 0, st>>>(h->kc, const_cast<float*>(k), 0, h->self_layer_stride, h->self_slot_stride,
+                                        slot, c.max_cache_len, start_pos, n_rows, c.d_model, 0);
+        k_kv_copy<<<grid, 128, 0, st>>>(h->vc, const_cast<float*>(v), 0, h->self_layer_stride, h->self_slot_stride,
+                                        slot, c.max_cache_len, start_pos, n_rows, c.d_model, 0);
+        DEC_CUDA(h, cudaGetLastError());
+    }
+    h->slot_len[slot] = start_pos + n_rows;
+    return DEC_OK;
+}
+
+dec_status dec_kv_read(dec_handle* h, int32_t slot, int32_t layer, int32_t start, int32_t n, float* k_out,
+                       float* v_out, void* stream) {
+    if (!h) return DEC_EINVAL;
+    const dec_config& c = h->cfg;
+    if (slot < 0 || slot >= c.max_slots || layer < 0 || layer >= c.n_layers)
+        return fail(h, DEC_EINVAL, "slot or layer out of range");
+    if (start < 0 || n < 0 || start + n > c.max_cache_len) return fail(h, DEC_EINVAL, "rows out of range");
+    if (n > 0 && (!k_out || !v_out)) return fail(h, DEC_EINVAL, "null output");
+    DEC_TRY(check_device(h));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (n > 0) {
+        dim3 grid(n, 1);
+        k_kv_copy<<<grid, 128, 0, st>>>(h->kc, k_out, 1, h->self_layer_stride, h->self_slot_stride, slot,
+                                        c.max_cache_len, start, n, c.d_model, layer);
+        k_kv_copy<<<grid, 128, 0, st>>>(h->vc, v_out, 1, h->self_layer_stride, h->self_slot_stride, slot,
+                                        c.max_cache_len, start, n, c.d_model, layer);
+        DEC_CUDA(h, cudaGetLastError());
+    }
+    return DEC_OK;
+}
+
+dec_status dec_step(dec_handle* h, int32_t batch, const int32_t* slots, const int32_t* tokens,
+                    const int32_t* positions, const int32_t* cache_lens, float* logits, int32_t* argmax,
+                    void* stream) {
+    if (!h) return DEC_EINVAL;
+    StepMeta m{};
+    int max_len = 0;
+    DEC_TRY(validate_step(h, batch, slots, tokens, positions, cache_lens, m, max_len));
+    DEC_TRY(check_device(h));
+    return step_validated(h, m, max_len, logits, argmax, static_cast<cudaStream_t>(stream));
+}
+
+dec_status dec_step_host(dec_handle* h, int32_t batch, const int32_t* slots, const int32_t* tokens,
+                         const int32_t* positions, const int32_t* cache_lens, float* logits_host,
+                         int32_t* argmax_host, void* stream) {
+    if (!h) return DEC_EINVAL;
+    StepMeta m{};
+    int max_len = 0;
+    DEC_TRY(validate_step(h, batch, slots, tokens, positions, cache_lens, m, max_len));
+    DEC_TRY(check_device(h));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const dec_config& c = h->cfg;
+    DEC_TRY(step_validated(h, m, max_len, logits_host ? h->stage_logits : nullptr, h->stage_argmax, st));
+    if (logits_host)
+        DEC_CUDA(h, cudaMemcpyAsync(logits_host, h->stage_logits, size_t(batch) * c.vocab * 4,
+                                    cudaMemcpyDeviceToHost, st));
+    if (argmax_host)
+        DEC_CUDA(h, cudaMemcpyAsync(argmax_host, h->stage_argmax, size_t(batch) * 4, cudaMemcpyDeviceToHost, st));
+    DEC_CUDA(h, cudaStreamSynchronize(st));
+    return DEC_OK;
+}
+
+dec_status dec_slot_len(const dec_handle* h, int32_t slot, int32_t* len) {
+    if (!h || !len || slot < 0 || slot >= h->cfg.max_slots) return DEC_EINVAL;
+    *len = h->slot_len[slot];
+    return DEC_OK;
+}
+
+dec_status dec_hidden(dec_handle* h, float* out, int32_t batch, void* stream) {
+    if (!h) return DEC_EINVAL;
+    if (!out || batch < 1 || batch > h->last_batch) return fail(h, DEC_EINVAL, "bad output or batch");
+    DEC_CUDA(h, cudaMemcpyAsync(out, h->x, size_t(batch) * h->cfg.d_model * 4, cudaMemcpyDeviceToDevice,
+                                static_cast<cudaStream_t>(stream)));
+    return DEC_OK;
+}
+
+dec_status dec_sync(dec_handle* h, void* stream) {
+    if (!h) return DEC_EINVAL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    DEC_CUDA(h, cudaStreamSynchronize(st));
+    int e = 0;
+    DEC_CUDA(h, cudaMemcpy(&e, h->dev_err, 4, cudaMemcpyDeviceToHost));
+    if (e) {
+        DEC_CUDA(h, cudaMemset(h->dev_err, 0, 4));
+        return fail(h, DEC_ETIMEOUT, "a bounded device wait gave up");
+    }
+    return DEC_OK;
+}
+
+size_t dec_attention_workspace_size(int32_t batch, int32_t n_heads, int32_t ld) {
+    (void)ld;
+    if (batch < 1 || n_heads < 1) return 0;
+    const size_t counters = ((size_t(batch) * n_heads * 4) + 255) / 256 * 256;
+    return counters + size_t(batch) * n_heads * kMaxSplits * kAttnPartStride * 4;
+}
+
+dec_status dec_attention(const float* q, const float* k, const float* v, const int32_t* lens, int32_t batch,
+                         int32_t n_heads, int32_t ld, float* out, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+    if (!q || !k || !v || !lens || !out || !workspace) return DEC_EINVAL;
+    if (batch < 1 || n_heads < 1 || ld < 1) return DEC_EINVAL;
+    if (workspace_bytes < dec_attention_workspace_size(batch, n_heads, ld)) return DEC_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15) return DEC_EINVAL;
+    static int configured = 0;
+    if (!configured) {
+        if (cudaFuncSetAttribute(k_attention, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kAttnSmemBytes)) !=
+            cudaSuccess)
+            return DEC_ECUDA;
+        configured = 1;
+    }
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    AttnArgs a{};
+    a.q = q;
+    a.q_bstride = (long long)n_heads * 64;
+    a.k = k;
+    a.v = v;
+    a.slot_stride = (long long)n_heads * ld * 64;
+    a.ld = ld;
+    a.H = n_heads;
+    a.mode = ATTN_OP;
+    a.batch = batch;
+    a.lens = lens;
+    a.out = out;
+    a.out_bstride = (long long)n_heads * 64;
+    const size_t counters = ((size_t(batch) * n_heads * 4) + 255) / 256 * 256;
+    a.counters = static_cast<int*>(workspace);
+    a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + counters);
+    a.err = nullptr;
+    dec_handle tmp;
+    tmp.num_sms = sms;
+    const int max_tiles = (ld + kAttnTile - 1) / kAttnTile;
+    a.S = choose_splits(&tmp, batch * n_heads, max_tiles);
+    cudaError_t e = launch(k_attention, dim3(a.S, n_heads, batch), dim3(kAttnThreads), kAttnSmemBytes,
+                           static_cast<cudaStream_t>(stream), a);
+    return e == cudaSuccess ? DEC_OK : DEC_ECUDA;
+}
+
+dec_status dec_i8_dot(const int8_t* xq, const int8_t* wq, int32_t m, int32_t n, int32_t kdim, int32_t* acc,
+                      void* stream) {
+    if (!xq || !wq || !acc) return DEC_EINVAL;
+    if (m < 1 || m > 64 || n < 1 || kdim < 16 || kdim % 16) return DEC_EINVAL;
+    dec_handle tmp;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&tmp.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    GemvArgs g{};
+    g.xq = xq;
+    g.x_ld = kdim;
+    g.K = kdim;
+    g.N = n;
+    g.B = m;
+    g.W = wq;
+    g.out_i32 = acc;
+    g.out_ld = n;
+    dec_status st = gemv<int8_t, true, PRO_RAW_I8, EPI_I32, MAP_ADJ>(&tmp, g, static_cast<cudaStream_t>(stream));
+    return st;
+}
+
+}  // extern "C"
