@@ -147,8 +147,9 @@ dec_status dec_create(const dec_config* cfg, const dec_weights* w, dec_handle** 
 /* Free everything the handle owns. Synchronises the device first. NULL is a no-op. */
 dec_status dec_destroy(dec_handle* h);
 
-/* Message of the last failed call on h (or of the last failed dec_create on
- * this thread when h is NULL). Never NULL; "" when there was no error. */
+/* Message of the last failed call on h (or, when h is NULL, of the last failed
+ * dec_create or handle-less call on this thread). Never NULL; "" when there was
+ * no error. */
 const char* dec_last_error(const dec_handle* h);
 
 /*
@@ -251,6 +252,26 @@ size_t dec_attention_workspace_size(int32_t batch, int32_t n_heads, int32_t ld);
 dec_status dec_attention(const float* q, const float* k, const float* v, const int32_t* lens,
                          int32_t batch, int32_t n_heads, int32_t ld, float* out,
                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Allocation-free variant of dec_attention, for callers that cannot allocate
+ * device memory themselves: code that runs under a host framework whose allocator
+ * owns the whole device and hands plug-ins no workspace, or latency-critical
+ * paths where cudaMalloc's implicit device synchronisation is not acceptable.
+ * (It has no counterpart in the pages; it is an interface convenience only.)
+ * Same arguments, numerics and output as dec_attention, minus the workspace:
+ * the split-K scratch lives in one fixed array of about 2.2 MB inside this
+ * library, which every GPU that loads the library holds until the process exits.
+ * Limits: batch * n_heads <= 1024 (DEC_EINVAL otherwise, message from
+ * dec_last_error(NULL)). The first call on a device looks up that array's device
+ * address (cudaGetSymbolAddress) with the device current; make that first call
+ * before any stream capture. Every call clears the arrival counters it needs
+ * (cudaMemsetAsync on `stream`) and shares the one array, which keeps the last
+ * call's contents: calls that overlap on the GPU (different streams, no ordering)
+ * race on it. It allocates nothing.
+ */
+dec_status dec_attention_noalloc(const float* q, const float* k, const float* v, const int32_t* lens,
+                                 int32_t batch, int32_t n_heads, int32_t ld, float* out, void* stream);
 
 /*
  * int8 x int8 -> int32 dot products acc[m, n] = sum_k xq[m, k] * wq[n, k]

@@ -25,7 +25,7 @@ PROJ = {"f32": 0, "w8a8": 1, "w8a32": 2}
 # Every symbol include/dec.h declares.
 EXPORTS = ["dec_create", "dec_destroy", "dec_last_error", "dec_prefill", "dec_kv_append", "dec_step",
            "dec_step_host", "dec_slot_len", "dec_kv_read", "dec_hidden", "dec_sync",
-           "dec_attention_workspace_size", "dec_attention", "dec_i8_dot"]
+           "dec_attention_workspace_size", "dec_attention", "dec_attention_noalloc", "dec_i8_dot"]
 
 
 class DecError(RuntimeError):
@@ -82,6 +82,7 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
         "dec_sync": (C.c_int, [vp, vp]),
         "dec_attention_workspace_size": (C.c_size_t, [i32, i32, i32]),
         "dec_attention": (C.c_int, [vp, vp, vp, vp, i32, i32, i32, vp, vp, C.c_size_t, vp]),
+        "dec_attention_noalloc": (C.c_int, [vp, vp, vp, vp, i32, i32, i32, vp, vp]),
         "dec_i8_dot": (C.c_int, [vp, vp, i32, i32, i32, vp, vp]),
     }
     for name, (res, args) in sig.items():
@@ -223,6 +224,14 @@ def attention(q, k, v, lens, batch: int, n_heads: int, ld: int, out, workspace, 
                              _ptr(workspace), workspace_bytes, stream)
     if st != DEC_OK:
         raise DecError(st, "dec_attention failed")
+
+
+def attention_noalloc(q, k, v, lens, batch: int, n_heads: int, ld: int, out, stream: int = 0):
+    """dec_attention without a caller workspace: the library's fixed scratch array is used."""
+    st = lib().dec_attention_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(lens), batch, n_heads, ld,
+                                     _ptr(out), stream)
+    if st != DEC_OK:
+        raise DecError(st, lib().dec_last_error(None).decode())
 
 
 def attention_workspace_size(batch: int, n_heads: int, ld: int) -> int:

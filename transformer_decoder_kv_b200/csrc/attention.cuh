@@ -60,7 +60,8 @@ __device__ __forceinline__ void attn_issue(float* sK, float* sV, uint64_t* bar, 
     bulk_g2s(sV, Vb + static_cast<long long>(tile) * kAttnTile * kHeadDim, bytes, bar);
 }
 
-__global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArgs a) {
+// Internal linkage: each translation unit that launches it carries its own copy.
+static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArgs a) {
     extern __shared__ __align__(128) unsigned char attn_smem[];
     float* sK = reinterpret_cast<float*>(attn_smem);
     float* sV = sK + kAttnStages * kAttnTile * kHeadDim;

@@ -30,6 +30,13 @@ constexpr int kMaxSplits = 32;
 
 thread_local std::string g_create_error;
 
+}  // namespace
+
+// Message for dec_last_error(NULL) from handle-less entry points in other files.
+void dec_set_thread_error(const char* msg) { g_create_error = msg ? msg : ""; }
+
+namespace {
+
 struct LayerDev {
     float *n1w = nullptr, *n1b = nullptr, *n2w = nullptr, *n2b = nullptr, *n3w = nullptr, *n3b = nullptr;
     void* wqkv = nullptr;
