@@ -71,7 +71,10 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
     __shared__ __align__(16) float wo[4][kHeadDim];
     __shared__ int s_flag;
 
-    pdl_wait();
+    // The step description and cache rows older than this step were written before
+    // the previous kernel ran; only the new row (self-attention) and q come from it.
+    // Standalone calls wait first: their inputs may come from any kernel.
+    if (a.mode == ATTN_OP) pdl_wait();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
 
@@ -87,6 +90,7 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
     }
     float* outp = a.out + b * a.out_bstride + h * kHeadDim;
     if (n <= 0) {
+        if (a.mode != ATTN_OP) pdl_wait();
         if (s == 0 && tid < kHeadDim) outp[tid] = 0.0f;
         return;
     }
@@ -100,17 +104,26 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
     const float* Kb = a.k + slot * a.slot_stride + static_cast<long long>(h) * a.ld * kHeadDim;
     const float* Vb = a.v + slot * a.slot_stride + static_cast<long long>(h) * a.ld * kHeadDim;
 
-    if (tid < kHeadDim) sq[tid] = a.q[b * a.q_bstride + h * kHeadDim + tid];
+    // tiles before the first one holding the row this step appends can be fetched
+    // before the dependency wait
+    const int first_new_tile = (a.mode == ATTN_SELF) ? (n - 1) / kAttnTile : ntiles;
+    int pre = 0;
     if (tid == 0) {
         for (int i = 0; i < kAttnStages; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
+        for (; pre < kAttnStages && t0 + pre < t1 && t0 + pre < first_new_tile; ++pre)
+            attn_issue(sK + pre * kAttnTile * kHeadDim, sV + pre * kAttnTile * kHeadDim, &bars[pre], Kb,
+                       Vb, t0 + pre, n);
     }
-    __syncthreads();
+    pdl_launch_dependents();
+    if (a.mode != ATTN_OP) pdl_wait();
+    if (tid < kHeadDim) sq[tid] = a.q[b * a.q_bstride + h * kHeadDim + tid];
     if (tid == 0) {
-        for (int i = 0; i < kAttnStages && t0 + i < t1; ++i)
+        for (int i = pre; i < kAttnStages && t0 + i < t1; ++i)
             attn_issue(sK + i * kAttnTile * kHeadDim, sV + i * kAttnTile * kHeadDim, &bars[i], Kb,
                        Vb, t0 + i, n);
     }
+    __syncthreads();
 
     const int jj = lane & 15, half = lane >> 4;
     const int key_in_tile = warp * 16 + jj;
@@ -188,7 +201,6 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
             attn_issue(sK + stage * kAttnTile * kHeadDim, sV + stage * kAttnTile * kHeadDim,
                        &bars[stage], Kb, Vb, t + kAttnStages, n);
     }
-    pdl_launch_dependents();
 
     // merge the four warps
     if (lane == 0) {

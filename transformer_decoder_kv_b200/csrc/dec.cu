@@ -279,6 +279,7 @@ GemvArgs base_args(dec_handle* h, int B) {
     g.B = B;
     g.eps = h->cfg.norm_eps;
     g.meta = h->dmeta;
+    g.err = h->dev_err;
     return g;
 }
 

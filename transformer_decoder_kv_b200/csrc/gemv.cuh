@@ -1,19 +1,22 @@
 // Weight-streaming projection kernels for small batches: y[b, n] = sum_k x[b, k] W[n, k].
 //
-// Each warp owns two weight rows at a time (a "task") and streams them from HBM
-// with 16-byte non-allocating loads, lane l covering bytes [16 l, 16 l + 16) of
-// every 512-byte run of the row. The (normalised, optionally int8-quantised)
-// activation rows of the batch tile sit in shared memory and are reused by every
-// task of the CTA. Per-lane partial sums for the 2 x BT outputs of a task are
-// reduced with a halving transpose, which leaves each output in one lane for the
-// fused epilogue.
+// Work unit: a block of 4 tasks = 8 weight rows (each warp owns one task = two
+// rows). CTAs are persistent over blocks. The rows of a block are moved from HBM
+// into a shared-memory ring by one thread with 1-D bulk async copies (one per row
+// and K chunk) completing on an mbarrier per stage; weights do not depend on the
+// previous kernel, so the first stages are issued before the programmatic-
+// dependent-launch wait and overlap the previous kernel's tail. The
+// (normalised, optionally int8-quantised) activation rows of the batch tile are
+// staged once per CTA after the wait, with 16-byte loads, and reused by every
+// block. Per-lane partial sums for the 2 x BT outputs of a task are reduced with a
+// halving transpose, which leaves each output in one lane for the fused epilogue.
 //
 // Prologues (per activation row, computed by every CTA from the raw residual
 // stream so that no separate norm kernel runs):
 //   PRO_NONE  x as is
 //   PRO_LN    LayerNorm (x - mean) / sqrt(var + eps) * g + b  (cera whisper.rs, layer_norm_inplace)
 //   PRO_RMS   RMSNorm x / sqrt(mean(x^2) + eps) * w             (franken_ocr decoder_qwen2.rs, family_norm)
-//   ACT_I8    then per-row symmetric int8 quantisation with ties to even:
+//   I8        then per-row symmetric int8 quantisation with ties to even:
 //             inv = 127 / amax, q = rint(x * inv), a = amax / 127  (decoder_qwen2.rs, quantize_row_i8_te)
 // Weight formats: f32; int8 with per-row scale and f32 activations (W8A32,
 // lattice-inference cpu_q8.rs matmul_bt_q8); int8 with int8 activations and int32
@@ -35,6 +38,9 @@ enum RowMap { MAP_ADJ = 0, MAP_ROPE = 1, MAP_DUAL = 2 };
 
 constexpr int kGemvWarps = 4;
 constexpr int kGemvThreads = kGemvWarps * 32;
+constexpr int kGemvRowsPerBlock = 2 * kGemvWarps;
+constexpr int kGemvMaxStages = 8;
+constexpr int kGemvStageBytes = 16 * 1024;   // weight bytes per stage at most
 
 struct GemvArgs {
     const float* x;          // activation rows (f32), row b at x + b * x_ld
@@ -66,6 +72,7 @@ struct GemvArgs {
     int* argmax_out;           // [B] or null
     int* last_tok;             // [slots]
     const StepMeta* meta;
+    int* err;                  // device status word
 };
 
 template <typename WT>
@@ -79,21 +86,9 @@ struct WVec<int8_t> {
     static constexpr int kElems = 16;
 };
 
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
-__device__ __forceinline__ float norm_value(int pro, float x, float mu, float rstd, const float* g,
-                                            const float* beta, int k) {
-    if (pro == PRO_LN) {
-        return __fadd_rn(__fmul_rn(__fmul_rn(__fsub_rn(x, mu), rstd), g[k]), beta[k]);
-    } else if (pro == PRO_RMS) {
-        return __fmul_rn(__fmul_rn(x, rstd), g[k]);
-    }
+__device__ __forceinline__ float norm_value(int pro, float x, float mu, float rstd, float g, float beta) {
+    if (pro == PRO_LN) return __fadd_rn(__fmul_rn(__fmul_rn(__fsub_rn(x, mu), rstd), g), beta);
+    if (pro == PRO_RMS) return __fmul_rn(__fmul_rn(x, rstd), g);
     return x;
 }
 
@@ -146,64 +141,209 @@ struct Dot<int8_t, true> {
     }
 };
 
-// Shared-memory bytes of the activation tile for a K chunk.
-template <int BT, bool I8>
-__host__ __device__ constexpr size_t gemv_xtile_bytes(int kc) {
-    return static_cast<size_t>(BT) * kc * (I8 ? 1 : 4);
+// Warp roles: kGemvConsumerWarps warps compute, one more warp moves weights.
+constexpr int kGemvConsumerWarps = 8;
+constexpr int kGemvThreadsWS = (kGemvConsumerWarps + 1) * 32;
+
+// Rows per consumer-warp task: four for batch tiles up to 8 (more independent rows
+// per warp), two for 16 and 32 (the 2 x BT accumulators bound the registers).
+__host__ __device__ constexpr int gemv_rows_per_task(int bt) { return bt <= 8 ? 4 : 2; }
+// Weight bytes per pipeline stage.
+__host__ __device__ constexpr int gemv_stage_bytes(int bt) { return bt <= 8 ? 32 * 1024 : 16 * 1024; }
+
+// Pair p of a row map (MAP_ADJ: 2p, 2p+1; MAP_ROPE: the NEOX pair (i, i + 32) of one
+// head; MAP_DUAL: row p of W and of W2). A task of R rows holds pairs R/2 t .. R/2 t + R/2 - 1.
+template <int MAP>
+__device__ __forceinline__ void pair_rows(int p, int& r0, int& r1) {
+    if (MAP == MAP_ROPE) {
+        const int hb = p >> 5, i = p & 31;
+        r0 = hb * 64 + i;
+        r1 = r0 + 32;
+    } else if (MAP == MAP_DUAL) {
+        r0 = p;
+        r1 = p;
+    } else {
+        r0 = 2 * p;
+        r1 = 2 * p + 1;
+    }
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 template <int BT, typename WT, bool I8, int PRO, int EPI, int MAP>
-__global__ void __launch_bounds__(kGemvThreads) k_gemv(const GemvArgs a, int KC) {
+__global__ void __launch_bounds__(kGemvThreadsWS, 2) k_gemv(const GemvArgs a, int KC, int NS) {
     using AccT = typename std::conditional<I8, int, float>::type;
     using XT = typename std::conditional<I8, int8_t, float>::type;
+    constexpr int NWC = kGemvConsumerWarps;
+    constexpr int R = gemv_rows_per_task(BT);   // weight rows per warp task
+    constexpr int P = R / 2;                    // row pairs per task
+    constexpr int ROWS_PER_BLOCK = R * NWC;
     constexpr int VE = WVec<WT>::kElems;
-    constexpr int NV = 2 * BT;                 // outputs per task
-    constexpr int NC = NV > 32 ? NV / 32 : 1;  // 32-value chunks
+    constexpr int NV = R * BT;                  // outputs per task
+    constexpr int NC = NV > 32 ? NV / 32 : 1;   // 32-value chunks
     constexpr int NVC = NV > 32 ? 32 : NV;
     constexpr int SH = transpose_shift<NVC>();
+    constexpr bool RAW_STAGE = I8 && PRO != PRO_RAW_I8;   // f32 rows staged apart from the int8 tile
     static_assert(!(I8 && !std::is_same<WT, int8_t>::value), "int8 activations need int8 weights");
 
-    extern __shared__ __align__(16) unsigned char gemv_smem[];
-    XT* sX = reinterpret_cast<XT*>(gemv_smem);
+    extern __shared__ __align__(128) unsigned char gemv_smem[];
+    const int stage_bytes = ROWS_PER_BLOCK * KC * static_cast<int>(sizeof(WT));
+    unsigned char* ring = gemv_smem;
+    XT* sX = reinterpret_cast<XT*>(gemv_smem + static_cast<size_t>(NS) * stage_bytes);
+    float* sXraw = RAW_STAGE ? reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(sX) +
+                                                         static_cast<size_t>(BT) * a.K * sizeof(XT))
+                             : reinterpret_cast<float*>(sX);
+    __shared__ __align__(8) uint64_t full[kGemvMaxStages];
+    __shared__ __align__(8) uint64_t empty[kGemvMaxStages];
+    __shared__ __align__(8) uint64_t bar_x;
     __shared__ float s_mu[BT], s_rstd[BT], s_inv[BT], s_a[BT];
     __shared__ unsigned long long s_key[BT];
+    __shared__ int s_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool producer = warp == NWC;
     const int b0 = blockIdx.y * BT;        // first batch row of this CTA's batch tile
-    const int nb = min(BT, a.B - b0);  // live rows of this batch tile
-    const int n_tasks = (MAP == MAP_DUAL) ? a.N : (a.N + 1) / 2;
-    const int nchunks = (a.K + KC - 1) / KC;
+    const int nb = min(BT, a.B - b0);      // live rows of this batch tile
+    const int n_pairs = (MAP == MAP_DUAL) ? a.N : (a.N + 1) / 2;
+    const int n_tasks = (n_pairs + P - 1) / P;
+    const int n_blocks = (n_tasks + NWC - 1) / NWC;
+    const int nkc = (a.K + KC - 1) / KC;
+    const int my_blocks = blockIdx.x < n_blocks ? (n_blocks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int n_items = my_blocks * nkc;
 
+    // rows of task t, in pair order (-1 = no row)
+    auto task_rows = [&](int task, int (&rows)[R]) {
+#pragma unroll
+        for (int q = 0; q < P; ++q) {
+            const int p = task * P + q;
+            int r0 = -1, r1 = -1;
+            if (task < n_tasks && p < n_pairs) pair_rows<MAP>(p, r0, r1);
+            rows[2 * q] = (r0 >= 0 && r0 < a.N) ? r0 : -1;
+            rows[2 * q + 1] = (r1 >= 0 && r1 < a.N) ? r1 : -1;
+        }
+    };
+
+    // ---- weight pipeline: item `it` = (block, K chunk) -> stage it % NS ----
+    auto issue = [&](int it) {
+        const int jb = blockIdx.x + (it / nkc) * gridDim.x;
+        const int c = it % nkc;
+        const int k0 = c * KC, kc = min(KC, a.K - k0);
+        const uint32_t row_bytes = static_cast<uint32_t>(kc) * sizeof(WT);
+        const int stage = it % NS;
+        unsigned char* dst = ring + static_cast<size_t>(stage) * stage_bytes;
+        uint32_t total = 0;
+        for (int w = 0; w < NWC; ++w) {
+            int rows[R];
+            task_rows(jb * NWC + w, rows);
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                if (rows[r] >= 0) total += row_bytes;
+        }
+        mbar_arrive_expect_tx(&full[stage], total);
+        for (int w = 0; w < NWC; ++w) {
+            int rows[R];
+            task_rows(jb * NWC + w, rows);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                if (rows[r] < 0) continue;
+                const void* base = (MAP == MAP_DUAL && (r & 1)) ? a.W2 : a.W;
+                const WT* g = reinterpret_cast<const WT*>(base) + static_cast<long long>(rows[r]) * a.K + k0;
+                bulk_g2s(dst + static_cast<size_t>(w * R + r) * KC * sizeof(WT), g, row_bytes, &full[stage]);
+            }
+        }
+    };
+
+    // weights do not depend on the previous kernel: start streaming before the wait
+    int n_issued = 0;
+    if (producer && lane == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], NWC);
+        }
+        mbar_init(&bar_x, 1);
+        mbar_fence_init();
+        for (; n_issued < NS && n_issued < n_items; ++n_issued) issue(n_issued);
+    }
+    pdl_launch_dependents();
     pdl_wait();
 
-    // ---- per-row statistics over the full K ----
-    if (PRO != PRO_RAW_I8) {
-        for (int b = warp; b < BT; b += kGemvWarps) {
+    // ---- activation rows (they come from the previous kernel): one bulk copy per row ----
+    const int in_elt = (PRO == PRO_RAW_I8) ? 1 : 4;
+    if (producer && lane == 0) {
+        const uint32_t row_bytes = static_cast<uint32_t>(a.K) * in_elt;
+        mbar_arrive_expect_tx(&bar_x, row_bytes * nb);
+        for (int b = 0; b < nb; ++b) {
+            if (PRO == PRO_RAW_I8)
+                bulk_g2s(reinterpret_cast<int8_t*>(sX) + static_cast<size_t>(b) * a.K,
+                         a.xq + static_cast<long long>(b0 + b) * a.x_ld, row_bytes, &bar_x);
+            else
+                bulk_g2s(sXraw + static_cast<size_t>(b) * a.K, a.x + static_cast<long long>(b0 + b) * a.x_ld,
+                         row_bytes, &bar_x);
+        }
+        s_flag = mbar_wait_bounded(&bar_x, 0, a.err) ? 1 : 0;
+    }
+    __syncthreads();
+    if (!s_flag) {
+        if (producer && lane == 0)
+            for (int i2 = 0; i2 < n_issued; ++i2) mbar_wait_bounded(&full[i2], 0, nullptr);
+        __syncthreads();
+        return;
+    }
+    (void)mbar_try_wait(&bar_x, 0);
+
+    // ---- per-row statistics from shared memory ----
+    if (PRO != PRO_RAW_I8 && !producer) {
+        for (int b = warp; b < BT; b += NWC) {
             float mu = 0.0f, rstd = 1.0f, inv = 0.0f, ascale = 0.0f;
             if (b < nb) {
-                const float* xr = a.x + static_cast<long long>(b0 + b) * a.x_ld;
+                const float4* xr = reinterpret_cast<const float4*>(sXraw + static_cast<size_t>(b) * a.K);
+                const float4* g4 = reinterpret_cast<const float4*>(a.norm_w);
+                const float4* be4 = reinterpret_cast<const float4*>(a.norm_b);
+                const int K4 = a.K >> 2;
                 if (PRO == PRO_LN) {
                     float sum = 0.0f;
-                    for (int k = lane; k < a.K; k += 32) sum += xr[k];
-                    sum = warp_sum(sum);
-                    mu = sum / static_cast<float>(a.K);
+                    for (int k = lane; k < K4; k += 32) {
+                        const float4 v = xr[k];
+                        sum += (v.x + v.y) + (v.z + v.w);
+                    }
+                    mu = warp_sum(sum) / static_cast<float>(a.K);
                     float var = 0.0f;
-                    for (int k = lane; k < a.K; k += 32) {
-                        const float dv = xr[k] - mu;
-                        var = fmaf(dv, dv, var);
+                    for (int k = lane; k < K4; k += 32) {
+                        const float4 v = xr[k];
+                        const float d0 = v.x - mu, d1 = v.y - mu, d2 = v.z - mu, d3 = v.w - mu;
+                        var = fmaf(d0, d0, var);
+                        var = fmaf(d1, d1, var);
+                        var = fmaf(d2, d2, var);
+                        var = fmaf(d3, d3, var);
                     }
                     var = warp_sum(var) / static_cast<float>(a.K);
                     rstd = 1.0f / sqrtf(var + a.eps);
                 } else if (PRO == PRO_RMS) {
                     float ss = 0.0f;
-                    for (int k = lane; k < a.K; k += 32) ss = fmaf(xr[k], xr[k], ss);
+                    for (int k = lane; k < K4; k += 32) {
+                        const float4 v = xr[k];
+                        ss = fmaf(v.x, v.x, ss);
+                        ss = fmaf(v.y, v.y, ss);
+                        ss = fmaf(v.z, v.z, ss);
+                        ss = fmaf(v.w, v.w, ss);
+                    }
                     ss = warp_sum(ss) / static_cast<float>(a.K);
                     rstd = 1.0f / sqrtf(ss + a.eps);
                 }
                 if (I8) {
                     float amax = 0.0f;
-                    for (int k = lane; k < a.K; k += 32)
-                        amax = fmaxf(amax, fabsf(norm_value(PRO, xr[k], mu, rstd, a.norm_w, a.norm_b, k)));
+                    for (int k = lane; k < K4; k += 32) {
+                        const float4 v = xr[k];
+                        float4 g = make_float4(1.f, 1.f, 1.f, 1.f), be = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (PRO != PRO_NONE) g = __ldg(g4 + k);
+                        if (PRO == PRO_LN) be = __ldg(be4 + k);
+                        amax = fmaxf(amax, fabsf(norm_value(PRO, v.x, mu, rstd, g.x, be.x)));
+                        amax = fmaxf(amax, fabsf(norm_value(PRO, v.y, mu, rstd, g.y, be.y)));
+                        amax = fmaxf(amax, fabsf(norm_value(PRO, v.z, mu, rstd, g.z, be.z)));
+                        amax = fmaxf(amax, fabsf(norm_value(PRO, v.w, mu, rstd, g.w, be.w)));
+                    }
                     amax = warp_max(amax);
                     inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
                     ascale = __fdiv_rn(amax, 127.0f);
@@ -220,202 +360,195 @@ __global__ void __launch_bounds__(kGemvThreads) k_gemv(const GemvArgs a, int KC)
     if (EPI == EPI_HEAD && tid < BT) s_key[tid] = 0ull;
     __syncthreads();
 
-    auto stage_chunk = [&](int k0, int kc) {
-        // activation tile [BT][kc] for columns [k0, k0 + kc); rows >= nb are zero
-        const int total = BT * kc;
-        for (int e = tid; e < total; e += kGemvThreads) {
-            const int b = e / kc, kk = e - b * kc, k = k0 + kk;
-            if (PRO == PRO_RAW_I8) {
-                sX[e] = (b < nb) ? static_cast<XT>(a.xq[static_cast<long long>(b0 + b) * a.x_ld + k]) : XT(0);
+    // ---- normalise (and quantise) in shared memory; padding rows become zero ----
+    if (PRO != PRO_RAW_I8 && (PRO != PRO_NONE || I8 || nb < BT)) {
+        const int K4 = a.K >> 2;
+        const int total = BT * K4;
+        for (int e = tid; e < total; e += kGemvThreadsWS) {
+            const int b = e / K4, k4 = e - b * K4;
+            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (b < nb) {
+                const float4 v = reinterpret_cast<const float4*>(sXraw)[e];
+                float4 g = make_float4(1.f, 1.f, 1.f, 1.f), be = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (PRO != PRO_NONE) g = __ldg(reinterpret_cast<const float4*>(a.norm_w) + k4);
+                if (PRO == PRO_LN) be = __ldg(reinterpret_cast<const float4*>(a.norm_b) + k4);
+                y.x = norm_value(PRO, v.x, s_mu[b], s_rstd[b], g.x, be.x);
+                y.y = norm_value(PRO, v.y, s_mu[b], s_rstd[b], g.y, be.y);
+                y.z = norm_value(PRO, v.z, s_mu[b], s_rstd[b], g.z, be.z);
+                y.w = norm_value(PRO, v.w, s_mu[b], s_rstd[b], g.w, be.w);
+            }
+            if (I8) {
+                uint32_t pk = 0;
+                if (b < nb) {
+                    const float inv = s_inv[b];
+                    pk = (static_cast<uint32_t>(quant_i8(y.x, inv)) & 0xffu) |
+                         ((static_cast<uint32_t>(quant_i8(y.y, inv)) & 0xffu) << 8) |
+                         ((static_cast<uint32_t>(quant_i8(y.z, inv)) & 0xffu) << 16) |
+                         ((static_cast<uint32_t>(quant_i8(y.w, inv)) & 0xffu) << 24);
+                }
+                reinterpret_cast<uint32_t*>(sX)[e] = pk;
             } else {
-                float y = 0.0f;
-                if (b < nb)
-                    y = norm_value(PRO, a.x[static_cast<long long>(b0 + b) * a.x_ld + k], s_mu[b], s_rstd[b],
-                                   a.norm_w, a.norm_b, k);
-                if (I8)
-                    sX[e] = static_cast<XT>(b < nb ? quant_i8(y, s_inv[b]) : 0);
-                else
-                    sX[e] = static_cast<XT>(y);
+                reinterpret_cast<float4*>(sX)[e] = y;
             }
         }
-    };
+    } else if (PRO == PRO_RAW_I8 && nb < BT) {
+        for (int e = nb * (a.K >> 2) + tid; e < BT * (a.K >> 2); e += kGemvThreadsWS)
+            reinterpret_cast<uint32_t*>(sX)[e] = 0u;
+    }
+    __syncthreads();
 
     // per-lane running argmax keys for the head epilogue
     unsigned long long best[NC];
 #pragma unroll
     for (int c = 0; c < NC; ++c) best[c] = 0ull;
 
-    auto rows_of = [&](int task, int& r0, int& r1) {
-        if (MAP == MAP_ROPE) {
-            const int hb = task >> 5, i = task & 31;
-            r0 = hb * 64 + i;
-            r1 = r0 + 32;
-        } else if (MAP == MAP_DUAL) {
-            r0 = task;
-            r1 = task;
-        } else {
-            r0 = 2 * task;
-            r1 = 2 * task + 1;
-        }
-    };
-
-    auto accumulate = [&](int r0, int r1, int k0, int kc, AccT (&acc)[2][BT]) {
-        const WT* W0 = reinterpret_cast<const WT*>(a.W) + static_cast<long long>(r0) * a.K + k0;
-        const WT* W1 = reinterpret_cast<const WT*>(MAP == MAP_DUAL ? a.W2 : a.W) +
-                       static_cast<long long>(r1) * a.K + k0;
-        const bool has1 = r1 < a.N;
-        constexpr int U = 4;
-        for (int kk = lane * VE; kk < kc; kk += 32 * VE * U) {
-            uint4 w0[U], w1[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int k = kk + u * 32 * VE;
-                if (k < kc) {
-                    w0[u] = ldg_stream(W0 + k);
-                    w1[u] = has1 ? ldg_stream(W1 + k) : make_uint4(0, 0, 0, 0);
-                }
+    if (producer) {
+        // refill each stage once all consumer warps have released it
+        if (lane == 0) {
+            for (int it = n_issued; it < n_items; ++it) {
+                const int stage = it % NS;
+                if (!mbar_wait_bounded(&empty[stage], static_cast<uint32_t>(it / NS - 1) & 1u, a.err)) break;
+                issue(it);
+                n_issued = it + 1;
             }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int k = kk + u * 32 * VE;
-                if (k < kc) {
-#pragma unroll
-                    for (int b = 0; b < BT; ++b) {
-                        const XT* xs = sX + b * kc + k;
-                        Dot<WT, I8>::run(w0[u], xs, acc[0][b]);
-                        Dot<WT, I8>::run(w1[u], xs, acc[1][b]);
-                    }
-                }
-            }
-        }
-    };
-
-    auto epilogue = [&](int task, int r0, int r1, AccT (&acc)[2][BT]) {
-        // flatten value index v = r + 2 b and reduce across the warp
-#pragma unroll
-        for (int c = 0; c < NC; ++c) {
-            AccT vals[NVC];
-#pragma unroll
-            for (int j = 0; j < NVC; ++j) {
-                const int v = c * 32 + j;
-                vals[j] = acc[v & 1][v >> 1];
-            }
-            const AccT red = warp_reduce_transpose<NVC>(vals);
-            const int v = c * 32 + (lane >> SH);
-            const int r = v & 1, b = v >> 1;
-            const bool primary = (lane & ((1 << SH) - 1)) == 0;
-            const int n = r ? r1 : r0;
-            const bool live = (b < nb) && (n < a.N);
-            // dequantise
-            float y;
-            if (EPI == EPI_I32) {
-                y = 0.0f;  // raw accumulators only: no scales exist for this epilogue
-            } else if (I8) {
-                const float* sc = (MAP == MAP_DUAL && r) ? a.scale2 : a.scale;
-                y = __fmul_rn(static_cast<float>(red), __fmul_rn(s_a[b], sc[live ? n : 0]));
-            } else {
-                y = static_cast<float>(red);
-                if (std::is_same<WT, int8_t>::value) y = __fmul_rn(y, a.scale[live ? n : 0]);
-            }
-            if (EPI != EPI_HEAD && EPI != EPI_SWIGLU && EPI != EPI_I32 && a.bias != nullptr && live)
-                y = __fadd_rn(y, a.bias[n]);
-            // partner value (other row of the pair, same batch row)
-            const float yp = __shfl_xor_sync(0xffffffffu, y, 1 << SH);
-            const int gb = b0 + b;
-            if (EPI == EPI_I32) {
-                if (primary && live) a.out_i32[static_cast<long long>(gb) * a.out_ld + n] = static_cast<int>(red);
-            } else if (EPI == EPI_STORE) {
-                if (primary && live) a.out[static_cast<long long>(gb) * a.out_ld + n] = y;
-            } else if (EPI == EPI_RESID) {
-                if (primary && live) {
-                    float* p = a.out + static_cast<long long>(gb) * a.out_ld + n;
-                    *p = __fadd_rn(*p, y);
-                }
-            } else if (EPI == EPI_GELU) {
-                if (primary && live) a.out[static_cast<long long>(gb) * a.out_ld + n] = gelu_tanh_f(y);
-            } else if (EPI == EPI_SWIGLU) {
-                // r = 0 holds gate row n, its partner holds up row n
-                if (primary && live && r == 0)
-                    a.out[static_cast<long long>(gb) * a.out_ld + n] = __fmul_rn(silu_f(y), yp);
-            } else if (EPI == EPI_QKV) {
-                const int sec = n / a.d, within = n - sec * a.d;
-                const int hh = within >> 6, i = within & 63;
-                float val = y;
-                if (a.rope != nullptr && sec < 2) {
-                    const float2 cs = a.rope[static_cast<long long>(a.meta->pos[gb < a.B ? gb : 0]) * 32 + (i & 31)];
-                    // pair (i, i + 32): x_i' = x_i c - x_{i+32} s ; x_{i+32}' = x_i s + x_{i+32} c
-                    if (i < 32)
-                        val = __fsub_rn(__fmul_rn(y, cs.x), __fmul_rn(yp, cs.y));
-                    else
-                        val = __fadd_rn(__fmul_rn(yp, cs.y), __fmul_rn(y, cs.x));
-                }
-                if (primary && live) {
-                    if (sec == 0) {
-                        a.out[static_cast<long long>(gb) * a.out_ld + within] = val;
-                    } else {
-                        const int slot = a.meta->slot[gb], row = a.meta->len[gb];
-                        float* cache = (sec == 1) ? a.kc : a.vc;
-                        cache[slot * a.slot_stride + (static_cast<long long>(hh) * a.ld + row) * kHeadDim + i] = val;
-                    }
-                }
-            } else if (EPI == EPI_HEAD) {
-                if (primary && live && a.out != nullptr) a.out[static_cast<long long>(gb) * a.out_ld + n] = y;
-                if (live) {
-                    const unsigned long long key = argmax_key(y, n);
-                    best[c] = key > best[c] ? key : best[c];
-                }
-            }
-        }
-    };
-
-    if (nchunks == 1) {
-        stage_chunk(0, a.K);
-        __syncthreads();
-        for (int task = blockIdx.x * kGemvWarps + warp; task < n_tasks; task += gridDim.x * kGemvWarps) {
-            int r0, r1;
-            rows_of(task, r0, r1);
-            AccT acc[2][BT];
-#pragma unroll
-            for (int r = 0; r < 2; ++r)
-#pragma unroll
-                for (int b = 0; b < BT; ++b) acc[r][b] = AccT(0);
-            accumulate(r0, r1, 0, a.K, acc);
-            epilogue(task, r0, r1, acc);
+            // every copy issued has landed before the CTA may leave (bounded)
+            for (int i2 = max(0, n_issued - NS); i2 < n_issued; ++i2)
+                mbar_wait_bounded(&full[i2 % NS], static_cast<uint32_t>(i2 / NS) & 1u, nullptr);
         }
     } else {
-        // one task per warp; the activation tile is staged chunk by chunk
-        const int task = blockIdx.x * kGemvWarps + warp;
-        int r0 = 0, r1 = 0;
-        const bool has_task = task < n_tasks;
-        if (has_task) rows_of(task, r0, r1);
-        AccT acc[2][BT];
-#pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-            for (int b = 0; b < BT; ++b) acc[r][b] = AccT(0);
-        for (int c = 0; c < nchunks; ++c) {
+        AccT acc[R][BT];
+        for (int it = 0; it < n_items; ++it) {
+            const int stage = it % NS;
+            const uint32_t phase = static_cast<uint32_t>(it / NS) & 1u;
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait_bounded(&full[stage], phase, a.err) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (lane != 0) (void)mbar_try_wait(&full[stage], phase);
+            const int jb = blockIdx.x + (it / nkc) * gridDim.x;
+            const int c = it % nkc;
             const int k0 = c * KC, kc = min(KC, a.K - k0);
-            __syncthreads();
-            stage_chunk(k0, kc);
-            __syncthreads();
-            if (has_task) {
-                accumulate(r0, r1, k0, kc, acc);
+            const int task = jb * NWC + warp;
+            if (c == 0) {
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+#pragma unroll
+                    for (int b = 0; b < BT; ++b) acc[r][b] = AccT(0);
+            }
+            if (task < n_tasks) {
+                const WT* wbase = reinterpret_cast<const WT*>(ring + static_cast<size_t>(stage) * stage_bytes) +
+                                  static_cast<size_t>(R * warp) * KC;
+                const XT* xbase = sX + k0;
+#pragma unroll 2
+                for (int kk = lane * VE; kk < kc; kk += 32 * VE) {
+                    uint4 wv[R];
+#pragma unroll
+                    for (int r = 0; r < R; ++r)
+                        wv[r] = *reinterpret_cast<const uint4*>(wbase + static_cast<size_t>(r) * KC + kk);
+#pragma unroll
+                    for (int b = 0; b < BT; ++b) {
+                        const XT* xs = xbase + static_cast<size_t>(b) * a.K + kk;
+#pragma unroll
+                        for (int r = 0; r < R; ++r) Dot<WT, I8>::run(wv[r], xs, acc[r][b]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (task < n_tasks && c == nkc - 1) {
+                int rows[R];
+                task_rows(task, rows);
+#pragma unroll
+                for (int cc = 0; cc < NC; ++cc) {
+                    AccT vals[NVC];
+#pragma unroll
+                    for (int j = 0; j < NVC; ++j) {
+                        const int v = cc * 32 + j;
+                        vals[j] = acc[v % R][v / R];
+                    }
+                    const AccT red = warp_reduce_transpose<NVC>(vals);
+                    const int v = cc * 32 + (lane >> SH);
+                    const int r = v % R, b = v / R;
+                    const bool primary = (lane & ((1 << SH) - 1)) == 0;
+                    const int n = rows[r];
+                    const bool live = (b < nb) && (n >= 0);
+                    float y;
+                    if (EPI == EPI_I32) {
+                        y = 0.0f;  // raw accumulators only: no scales exist for this epilogue
+                    } else if (I8) {
+                        const float* sc = (MAP == MAP_DUAL && (r & 1)) ? a.scale2 : a.scale;
+                        y = __fmul_rn(static_cast<float>(red), __fmul_rn(s_a[b], sc[live ? n : 0]));
+                    } else {
+                        y = static_cast<float>(red);
+                        if (std::is_same<WT, int8_t>::value) y = __fmul_rn(y, a.scale[live ? n : 0]);
+                    }
+                    if (EPI != EPI_HEAD && EPI != EPI_SWIGLU && EPI != EPI_I32 && a.bias != nullptr && live)
+                        y = __fadd_rn(y, a.bias[n]);
+                    // partner value (other row of the pair, same batch row): value index v ^ 1
+                    const float yp = __shfl_xor_sync(0xffffffffu, y, 1 << SH);
+                    const int gb = b0 + b;
+                    if (EPI == EPI_I32) {
+                        if (primary && live)
+                            a.out_i32[static_cast<long long>(gb) * a.out_ld + n] = static_cast<int>(red);
+                    } else if (EPI == EPI_STORE) {
+                        if (primary && live) a.out[static_cast<long long>(gb) * a.out_ld + n] = y;
+                    } else if (EPI == EPI_RESID) {
+                        if (primary && live) {
+                            float* p = a.out + static_cast<long long>(gb) * a.out_ld + n;
+                            *p = __fadd_rn(*p, y);
+                        }
+                    } else if (EPI == EPI_GELU) {
+                        if (primary && live) a.out[static_cast<long long>(gb) * a.out_ld + n] = gelu_tanh_f(y);
+                    } else if (EPI == EPI_SWIGLU) {
+                        // even r holds gate row n, its partner holds up row n
+                        if (primary && live && (r & 1) == 0)
+                            a.out[static_cast<long long>(gb) * a.out_ld + n] = __fmul_rn(silu_f(y), yp);
+                    } else if (EPI == EPI_QKV) {
+                        const int sec = n / a.d, within = n - sec * a.d;
+                        const int hh = within >> 6, i = within & 63;
+                        float val = y;
+                        if (a.rope != nullptr && sec < 2) {
+                            const float2 cs =
+                                a.rope[static_cast<long long>(a.meta->pos[gb < a.B ? gb : 0]) * 32 + (i & 31)];
+                            // pair (i, i + 32): x_i' = x_i c - x_{i+32} s ; x_{i+32}' = x_i s + x_{i+32} c
+                            if (i < 32)
+                                val = __fsub_rn(__fmul_rn(y, cs.x), __fmul_rn(yp, cs.y));
+                            else
+                                val = __fadd_rn(__fmul_rn(yp, cs.y), __fmul_rn(y, cs.x));
+                        }
+                        if (primary && live) {
+                            if (sec == 0) {
+                                a.out[static_cast<long long>(gb) * a.out_ld + within] = val;
+                            } else {
+                                const int slot = a.meta->slot[gb], row = a.meta->len[gb];
+                                float* cache = (sec == 1) ? a.kc : a.vc;
+                                cache[slot * a.slot_stride + (static_cast<long long>(hh) * a.ld + row) * kHeadDim + i] =
+                                    val;
+                            }
+                        }
+                    } else if (EPI == EPI_HEAD) {
+                        if (primary && live && a.out != nullptr)
+                            a.out[static_cast<long long>(gb) * a.out_ld + n] = y;
+                        if (live) {
+                            const unsigned long long key = argmax_key(y, n);
+                            best[cc] = key > best[cc] ? key : best[cc];
+                        }
+                    }
+                }
             }
         }
-        if (has_task) epilogue(task, r0, r1, acc);
     }
-    pdl_launch_dependents();
 
     if (EPI == EPI_HEAD) {
-        // fold the two rows of each batch row, then the CTA, then the grid
+        // fold the rows of each batch row, then the CTA, then the grid
+        __syncthreads();
+        if (!producer) {
 #pragma unroll
-        for (int c = 0; c < NC; ++c) {
-            unsigned long long o = __shfl_xor_sync(0xffffffffu, best[c], 1 << SH);
-            best[c] = o > best[c] ? o : best[c];
-            const int v = c * 32 + (lane >> SH);
-            const int b = v >> 1;
-            if ((lane & ((1 << SH) - 1)) == 0 && (v & 1) == 0 && b < nb && best[c] != 0ull)
-                atomicMax(&s_key[b], best[c]);
+            for (int c = 0; c < NC; ++c) {
+                const int v = c * 32 + (lane >> SH);
+                const int b = v / R;
+                if ((lane & ((1 << SH) - 1)) == 0 && b < nb && best[c] != 0ull) atomicMax(&s_key[b], best[c]);
+            }
         }
         __syncthreads();
         if (tid < nb && s_key[tid] != 0ull) atomicMax(&a.keys[b0 + tid], s_key[tid]);
@@ -429,7 +562,7 @@ __global__ void __launch_bounds__(kGemvThreads) k_gemv(const GemvArgs a, int KC)
         __syncthreads();
         if (s_last) {
             __threadfence();
-            for (int b = tid; b < a.B; b += kGemvThreads) {
+            for (int b = tid; b < a.B; b += kGemvThreadsWS) {
                 const unsigned long long k = atomicExch(&a.keys[b], 0ull);
                 const int idx = (k == 0ull) ? 0 : argmax_key_index(k);
                 if (a.argmax_out) a.argmax_out[b] = idx;

@@ -1,6 +1,6 @@
-// Launch planning for the projection kernels (batch tile, K chunking, grid size).
-// The template is instantiated explicitly in gemv_inst_*.cu so the many variants
-// compile in parallel; other translation units only see the declaration.
+// Launch planning for the projection kernels (batch tile, K chunk, pipeline depth,
+// grid size). The template is instantiated explicitly in gemv_inst_*.cu so the many
+// variants compile in parallel; other translation units only see the declaration.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -11,73 +11,104 @@
 
 namespace dec {
 
-constexpr size_t kGemvSmemBudget = 96 * 1024;
+constexpr size_t kGemvXBudget = 128 * 1024;      // activation tile bytes at most
+constexpr size_t kGemvRingBudget = 48 * 1024;    // weight ring bytes
+constexpr size_t kGemvSmemMax = 227 * 1024;
 
 template <typename WT, bool I8, int PRO, int EPI, int MAP>
 cudaError_t gemv_launch(int num_sms, const GemvArgs& a, cudaStream_t st);
 
 #ifdef DEC_GEMV_DEFINE
 
-inline int gemv_pow2ceil(int v) {
-    int p = 1;
-    while (p < v) p <<= 1;
+struct GemvPlan {
+    int KC, NS;
+    size_t smem;
+};
+
+// Activation bytes in shared memory: the tile, plus the raw f32 rows for the int8 path.
+template <bool I8, int PRO>
+size_t gemv_xbytes(int BT, int K) {
+    size_t x = size_t(BT) * K * (I8 ? 1 : 4);
+    if (I8 && PRO != PRO_RAW_I8) x += size_t(BT) * K * 4;
+    return x;
+}
+
+template <typename WT, bool I8, int PRO>
+GemvPlan gemv_plan(int BT, int K) {
+    GemvPlan p;
+    const int elt_w = sizeof(WT);
+    const int rows_per_block = gemv_rows_per_task(BT) * kGemvConsumerWarps;
+    // one stage = rows_per_block rows x KC columns
+    int kc = gemv_stage_bytes(BT) / (rows_per_block * elt_w);
+    kc = std::min(kc, K);
+    kc = std::max(16, kc / 16 * 16);
+    p.KC = kc;
+    const size_t stage = size_t(rows_per_block) * kc * elt_w;
+    const size_t xbytes = gemv_xbytes<I8, PRO>(BT, K);
+    // two CTAs per SM when the activation tile leaves room for two stages each,
+    // otherwise one CTA with a deeper ring
+    const size_t two_cta = 110 * 1024;
+    size_t ring;
+    if (xbytes + 2 * stage <= two_cta)
+        ring = two_cta - xbytes;
+    else
+        ring = 220 * 1024 - xbytes;
+    p.NS = int(std::min<size_t>(kGemvMaxStages, std::max<size_t>(2, ring / stage)));
+    p.smem = size_t(p.NS) * stage + xbytes;
     return p;
 }
 
 template <int BT, typename WT, bool I8, int PRO, int EPI, int MAP>
 cudaError_t gemv_launch_bt(int num_sms, const GemvArgs& a, cudaStream_t st) {
     auto kern = k_gemv<BT, WT, I8, PRO, EPI, MAP>;
-    const size_t elt = I8 ? 1 : 4;
-    int KC = a.K;
-    if (size_t(BT) * a.K * elt > kGemvSmemBudget) {
-        KC = int(kGemvSmemBudget / (size_t(BT) * elt));
-        KC = std::max(64, KC / 64 * 64);
-    }
-    const size_t smem = size_t(BT) * KC * elt;
-    static int per_sm = 0;  // per instantiation: occupancy at the full budget
+    const GemvPlan p = gemv_plan<WT, I8, PRO>(BT, a.K);
+    static bool attr_set = false;  // per instantiation
     cudaError_t e;
-    if (per_sm == 0) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemvSmemBudget));
+    if (!attr_set) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemvSmemMax - 2048));
         if (e != cudaSuccess) return e;
-        per_sm = -1;
+        attr_set = true;
     }
-    const int n_tasks = (MAP == MAP_DUAL) ? a.N : (a.N + 1) / 2;
-    const int need = (n_tasks + kGemvWarps - 1) / kGemvWarps;
-    int gx = need;
-    if (KC == a.K) {
-        // occupancy for this instantiation, cached per activation-tile size
-        static size_t occ_smem[4] = {~size_t(0), ~size_t(0), ~size_t(0), ~size_t(0)};
-        static int occ_val[4] = {0, 0, 0, 0};
-        int occ = -1;
-        for (int i = 0; i < 4; ++i)
-            if (occ_smem[i] == smem) occ = occ_val[i];
-        if (occ < 0) {
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGemvThreads, smem);
-            if (e != cudaSuccess) return e;
-            static int next = 0;
-            occ_smem[next] = smem;
-            occ_val[next] = occ;
-            next = (next + 1) & 3;
-        }
-        gx = std::min(need, num_sms * std::max(1, occ));
+    const int n_pairs = (MAP == MAP_DUAL) ? a.N : (a.N + 1) / 2;
+    const int pairs_per_task = gemv_rows_per_task(BT) / 2;
+    const int n_tasks = (n_pairs + pairs_per_task - 1) / pairs_per_task;
+    const int n_blocks = (n_tasks + kGemvConsumerWarps - 1) / kGemvConsumerWarps;
+    // occupancy for this instantiation, cached per shared-memory size
+    static size_t occ_smem[4] = {~size_t(0), ~size_t(0), ~size_t(0), ~size_t(0)};
+    static int occ_val[4] = {0, 0, 0, 0};
+    static int occ_next = 0;
+    int occ = -1;
+    for (int i = 0; i < 4; ++i)
+        if (occ_smem[i] == p.smem) occ = occ_val[i];
+    if (occ < 0) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGemvThreadsWS, p.smem);
+        if (e != cudaSuccess) return e;
+        occ_smem[occ_next] = p.smem;
+        occ_val[occ_next] = occ;
+        occ_next = (occ_next + 1) & 3;
     }
     const int gy = (a.B + BT - 1) / BT;
+    const int gx = std::max(1, std::min(n_blocks, (num_sms * std::max(1, occ)) / gy));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(gx, gy);
-    cfg.blockDim = dim3(kGemvThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.blockDim = dim3(kGemvThreadsWS);
+    cfg.dynamicSmemBytes = p.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a, KC);
+    return cudaLaunchKernelEx(&cfg, kern, a, p.KC, p.NS);
 }
 
 template <typename WT, bool I8, int PRO, int EPI, int MAP>
 cudaError_t gemv_launch(int num_sms, const GemvArgs& a, cudaStream_t st) {
-    const int bt = std::min(32, gemv_pow2ceil(a.B));
+    // batch tile: the largest power of two <= 32 covering the batch whose activation
+    // tile fits the budget
+    int bt = 1;
+    while (bt < a.B && bt < 32) bt <<= 1;
+    while (bt > 1 && gemv_xbytes<I8, PRO>(bt, a.K) > kGemvXBudget) bt >>= 1;
     switch (bt) {
         case 1: return gemv_launch_bt<1, WT, I8, PRO, EPI, MAP>(num_sms, a, st);
         case 2: return gemv_launch_bt<2, WT, I8, PRO, EPI, MAP>(num_sms, a, st);
