@@ -296,11 +296,20 @@ class OracleDecoder:
     parameters, and per-layer projections {"w", "s", "b"} in the model's format.
     """
 
-    def __init__(self, weights: dict, max_cache_len: int):
+    def __init__(self, weights: dict, max_cache_len: int, quant_jitter: Optional[int] = None,
+                 share_weights_with: Optional["OracleDecoder"] = None):
+        """quant_jitter: None (the oracle proper) or a seed. With a seed, every value
+        entering the int8 activation quantiser is first multiplied by (1 + u 2^-22),
+        u uniform in [-1, 1] -- at most 2 ulp. That models another correct f32
+        implementation of the norm / attention / SwiGLU feeding the quantiser, whose
+        value may differ in the last bits and so round the other way at a tie. Tests
+        use a few such runs to measure how far correct implementations drift apart;
+        it changes nothing when None."""
         self.W = weights
         self.cfg = weights["config"]
         self.max_len = max_cache_len
-        self._c64: dict = {}
+        self._c64: dict = share_weights_with._c64 if share_weights_with is not None else {}
+        self._jitter = np.random.default_rng(quant_jitter) if quant_jitter is not None else None
         # Diagnostics only (no effect on results): per-row smallest distance, in code
         # units, between an activation's x * inv and a rounding boundary k + 1/2, over all
         # int8 quantisations of the last forward_rows call.
@@ -337,6 +346,9 @@ class OracleDecoder:
         return y.astype(F32)
 
     def _quant(self, x):
+        if self._jitter is not None:
+            x64 = np.atleast_2d(np.asarray(x, F32)).astype(F64)
+            x = (x64 * (1.0 + self._jitter.uniform(-1.0, 1.0, x64.shape) * 2.0 ** -22)).astype(F32)
         q, a = quantize_rows_i8_te(x)
         if self._margins is not None:
             x32 = np.atleast_2d(np.asarray(x, F32))

@@ -8,61 +8,45 @@ import numpy as np
 import pytest
 
 import synth
-from tests._harness import ATOL, NEAR_TIE, RTOL, build_pair, close, step_both, top2_margin, within
+from tests._harness import ATOL, build_pair, check_row, close, step_both
 
 pytestmark = pytest.mark.gpu
 
 
 def _run(wl_name, steps=None, seed=0):
-    """Teacher-forced steps; returns the near-tie events.
-
-    A W8A8 stream whose GPU result leaves the tolerance is accepted only if the oracle
-    saw an int8 activation within NEAR_TIE of a rounding boundary in that same step
-    (both roundings are correct f32 outcomes); that stream's caches then legitimately
-    differ, so it leaves the comparison and the event is reported.
-    """
+    """Teacher-forced steps against the oracle (ensemble for W8A8); returns the
+    argmax near-tie events."""
     import torch
     wl = synth.workload(wl_name)
     p = build_pair(wl, seed)
     cfg = wl.model
     B = wl.batch
     toks = [int(t) for t in synth.token_ids(cfg, 999, B, seed)]
-    near_ties = []
-    live = set(range(B))
+    events = []
     for t in range(steps or wl.steps):
-        lg, am, hid, rl, rh = step_both(p, toks)
-        for b in sorted(live):
-            ok = within(hid[b], rh[b]) and within(lg[b], rl[b])
-            if not ok and cfg.proj_fmt == "w8a8" and p.margins[b] < NEAR_TIE:
-                near_ties.append((t, b, float(p.margins[b])))
-                live.discard(b)
-                continue
-            close(hid[b], rh[b], what=f"{wl_name} step {t} stream {b} hidden")
-            close(lg[b], rl[b], what=f"{wl_name} step {t} stream {b} logits")
-            # the device argmax is the argmax of the device logits, lowest index on ties
-            assert int(am[b]) == int(np.argmax(lg[b])), (t, b)
-            ref_pick = int(np.argmax(rl[b]))
-            if int(am[b]) != ref_pick:
-                m = top2_margin(rl[b])
-                assert m <= 2 * (ATOL + RTOL * abs(float(rl[b, ref_pick]))), (t, b, m)
-                near_ties.append((t, b, m))
+        lg, am, hid, rl, rh, env_h, env_l = step_both(p, toks)
+        for b in range(B):
+            ev = check_row(hid[b], lg[b], am[b], rh[b], rl[b], env_h[b], env_l[b],
+                           f"{wl_name} step {t} stream {b}")
+            if ev:
+                events.append(ev)
         toks = [int(np.argmax(rl[b])) for b in range(B)]
-    assert len(live) >= max(1, (2 * B) // 3), f"too many near-tie divergences: {near_ties}"
-    # K/V rows written by the steps agree with the oracle's cache rows
-    for slot in sorted(live):
-        st = p.states[slot]
+    # K/V rows written by prefill and steps agree with the oracle's cache rows
+    for slot, st in enumerate(p.states):
         for l in range(cfg.n_layers):
             n = st.n
             ko = torch.empty((n, cfg.d_model), device="cuda")
             vo = torch.empty((n, cfg.d_model), device="cuda")
             p.gpu.kv_read(slot, l, 0, n, ko, vo)
             torch.cuda.synchronize()
-            close(ko.cpu().numpy(), st.k[l][:n], what=f"K cache slot {slot} layer {l}")
-            close(vo.cpu().numpy(), st.v[l][:n], what=f"V cache slot {slot} layer {l}")
+            env_k = max([0.0] + [float(np.abs(sts[slot].k[l][:n] - st.k[l][:n]).max()) for _, sts in p.jrefs])
+            env_v = max([0.0] + [float(np.abs(sts[slot].v[l][:n] - st.v[l][:n]).max()) for _, sts in p.jrefs])
+            close(ko.cpu().numpy(), st.k[l][:n], atol=ATOL + 2 * env_k, what=f"K cache slot {slot} layer {l}")
+            close(vo.cpu().numpy(), st.v[l][:n], atol=ATOL + 2 * env_v, what=f"V cache slot {slot} layer {l}")
     p.gpu.close()
-    if near_ties:
-        print(f"{wl_name}: near-tie events (step, stream, margin): {near_ties}")
-    return near_ties
+    if events:
+        print(f"{wl_name}: near-tie events: {events}")
+    return events
 
 
 @pytest.mark.parametrize("wl_name", ["tiny_whisper_b3", "tiny_qwen2_b3", "tiny_whisper_w8a32_b3",
@@ -101,9 +85,9 @@ def test_batched_step_equals_solo_bitwise():
         pa = build_pair(wl)
         solo = [build_pair(wl, streams=[s], max_slots=1) for s in range(wl.batch)]
         toks = [11, 22, 33]
-        lg, _, _, _, _ = step_both(pa, toks)
+        lg = step_both(pa, toks)[0]
         for s in range(wl.batch):
-            l1, _, _, _, _ = step_both(solo[s], [toks[s]])
+            l1 = step_both(solo[s], [toks[s]])[0]
             assert np.array_equal(lg[s].view(np.uint32), l1[0].view(np.uint32)), (wl_name, s)
             solo[s].gpu.close()
         pa.gpu.close()
@@ -116,7 +100,7 @@ def test_host_step_matches_device_step():
     a = build_pair(wl)
     b = build_pair(wl)
     toks = [1, 2, 3]
-    lg, am, _, _, _ = step_both(a, toks)
+    lg, am = step_both(a, toks)[:2]
     pos = [st.n for st in b.states]
     lh = np.empty((wl.batch, cfg.vocab), np.float32)
     ah = np.empty(wl.batch, np.int32)

@@ -263,3 +263,26 @@ def test_quantisation_margin_diagnostic():
     q, a = dec._quant(x)
     assert np.array_equal(q, oracle.quantize_rows_i8_te(x)[0])
     assert dec._margins[0] == 0.0 and dec._margins[1] == 0.25
+
+
+def test_quant_jitter_is_small_and_off_by_default():
+    """The jittered oracle used by the W8A8 parity ensemble moves quantiser inputs by at
+    most 2^-22 relative, and only when asked."""
+    cfg, W = _model("tiny_qwen2")
+    a = oracle.OracleDecoder(W, 32)
+    b = oracle.OracleDecoder(W, 32, quant_jitter=None, share_weights_with=a)
+    c = oracle.OracleDecoder(W, 32, quant_jitter=7, share_weights_with=a)
+    x = (np.random.default_rng(0).standard_normal((3, 128)) * 2).astype(F32)
+    qa, aa = a._quant(x)
+    qb, ab = b._quant(x)
+    assert np.array_equal(qa, qb) and np.array_equal(aa, ab)
+    c._jitter = np.random.default_rng(7)
+    x64 = x.astype(np.float64)
+    xj = (x64 * (1.0 + np.random.default_rng(7).uniform(-1.0, 1.0, x64.shape) * 2.0 ** -22)).astype(F32)
+    assert np.all(np.abs(xj.astype(np.float64) - x64) <= np.abs(x64) * 2.0 ** -21)
+    qc, ac = c._quant(x)
+    assert np.abs(qc.astype(int) - qa.astype(int)).max() <= 1
+    toks = [3, 1, 4, 1, 5]
+    sa, sc = a.new_state(None), c.new_state(None)
+    la, lc = a.prefill(sa, toks), c.prefill(sc, toks)
+    assert np.abs(la - lc).max() < 0.05

@@ -12,6 +12,8 @@
 #include <cstring>
 #include <string>
 #include <type_traits>
+#include <array>
+#include <map>
 #include <vector>
 
 #include "../../include/dec.h"
@@ -82,6 +84,11 @@ struct dec_handle {
     std::vector<int> slot_len;
     std::vector<char> has_tok, has_cross;
     int last_batch = 0;
+    // CUDA graphs of the step's launch sequence, keyed by what changes its launches:
+    // batch size, self-attention tile count, output pointers. A null entry means
+    // capture failed for that key and the step runs eagerly.
+    std::map<std::array<long long, 4>, cudaGraphExec_t> graphs;
+    cudaStream_t cap_stream = nullptr;
     float* stage_logits = nullptr;   // dec_step_host result staging
     int* stage_argmax = nullptr;
     std::string err;
@@ -266,6 +273,8 @@ dec_status attention(dec_handle* h, AttnArgs a, int B, int max_keys, cudaStream_
     static int configured = 0;
     if (!configured) {
         DEC_CUDA(h, cudaFuncSetAttribute(k_attention, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kAttnSmemBytes)));
+        DEC_CUDA(h, cudaFuncSetAttribute(k_attention, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         cudaSharedmemCarveoutMaxShared));
         configured = 1;
     }
     const int max_tiles = (max_keys + kAttnTile - 1) / kAttnTile;
@@ -517,10 +526,43 @@ dec_status validate_step(dec_handle* h, int B, const int32_t* slots, const int32
     return DEC_OK;
 }
 
+// Record the step's launch sequence into a graph for later identical steps. Capture
+// problems are not errors: the key is marked and such steps keep running eagerly.
+void capture_step(dec_handle* h, const std::array<long long, 4>& key, int B, int max_len, float* logits,
+                  int* argmax) {
+    if (h->graphs.size() >= 256) {
+        for (auto& kv : h->graphs)
+            if (kv.second) cudaGraphExecDestroy(kv.second);
+        h->graphs.clear();
+    }
+    cudaGraphExec_t exec = nullptr;
+    if (cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal) == cudaSuccess) {
+        const std::string saved = h->err;
+        const dec_status s = run_step(h, B, max_len, logits, argmax, h->cap_stream);
+        cudaGraph_t g = nullptr;
+        const cudaError_t e = cudaStreamEndCapture(h->cap_stream, &g);
+        if (s == DEC_OK && e == cudaSuccess && g != nullptr) {
+            if (cudaGraphInstantiate(&exec, g, 0) != cudaSuccess) exec = nullptr;
+        }
+        if (g) cudaGraphDestroy(g);
+        h->err = saved;
+    }
+    cudaGetLastError();
+    h->graphs[key] = exec;
+}
+
 dec_status step_validated(dec_handle* h, const StepMeta& m, int max_len, float* logits, int* argmax,
                           cudaStream_t st) {
     DEC_TRY(upload_meta(h, m, st));
-    DEC_TRY(run_step(h, m.B, max_len, logits, argmax, st));
+    const std::array<long long, 4> key = {m.B, (max_len + kAttnTile - 1) / kAttnTile,
+                                          reinterpret_cast<long long>(logits), reinterpret_cast<long long>(argmax)};
+    auto it = h->graphs.find(key);
+    if (it != h->graphs.end() && it->second != nullptr) {
+        DEC_CUDA(h, cudaGraphLaunch(it->second, st));
+    } else {
+        DEC_TRY(run_step(h, m.B, max_len, logits, argmax, st));
+        if (it == h->graphs.end()) capture_step(h, key, m.B, max_len, logits, argmax);
+    }
     for (int b = 0; b < m.B; ++b) {
         h->slot_len[m.slot[b]] += 1;
         h->has_tok[m.slot[b]] = 1;
@@ -540,6 +582,9 @@ const char* dec_last_error(const dec_handle* h) { return h ? h->err.c_str() : g_
 dec_status dec_destroy(dec_handle* h) {
     if (!h) return DEC_OK;
     cudaDeviceSynchronize();
+    for (auto& kv : h->graphs)
+        if (kv.second) cudaGraphExecDestroy(kv.second);
+    if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
     for (void* p : h->dallocs) cudaFree(p);
     for (void* p : h->hallocs) cudaFreeHost(p);
     for (int i = 0; i < kMetaRing; ++i)
@@ -641,6 +686,7 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
         h->hmeta[i] = static_cast<StepMeta*>(p);
         DEC_CUDA(h, cudaEventCreateWithFlags(&h->hev[i], cudaEventDisableTiming));
     }
+    DEC_CUDA(h, cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking));
     h->slot_len.assign(c.max_slots, 0);
     h->has_tok.assign(c.max_slots, 0);
     h->has_cross.assign(c.max_slots, 0);

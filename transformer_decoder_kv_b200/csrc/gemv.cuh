@@ -141,14 +141,15 @@ struct Dot<int8_t, true> {
     }
 };
 
-// Warp roles: kGemvConsumerWarps warps compute, one more warp moves weights.
-constexpr int kGemvConsumerWarps = 8;
-constexpr int kGemvThreadsWS = (kGemvConsumerWarps + 1) * 32;
-
-// Rows per consumer-warp task: four for batch tiles up to 8 (more independent rows
-// per warp), two for 16 and 32 (the 2 x BT accumulators bound the registers).
-__host__ __device__ constexpr int gemv_rows_per_task(int bt) { return bt <= 8 ? 4 : 2; }
-// Weight bytes per pipeline stage.
+// Warp roles: gemv_consumer_warps(BT) warps compute, one more warp moves weights.
+// Batch tiles of 1-2 use 4 consumer warps and 8-row blocks, so that even a 1 MB
+// matrix spreads over every SM; larger tiles use 8 consumer warps.
+__host__ __device__ constexpr int gemv_consumer_warps(int bt) { return bt <= 2 ? 4 : 8; }
+__host__ __device__ constexpr int gemv_threads(int bt) { return (gemv_consumer_warps(bt) + 1) * 32; }
+// Rows per consumer-warp task: four for batch tiles 4 and 8 (more independent rows
+// per warp), two otherwise (for 16 and 32 the R x BT accumulators bound the registers).
+__host__ __device__ constexpr int gemv_rows_per_task(int bt) { return (bt == 4 || bt == 8) ? 4 : 2; }
+// Weight bytes per pipeline stage at most.
 __host__ __device__ constexpr int gemv_stage_bytes(int bt) { return bt <= 8 ? 32 * 1024 : 16 * 1024; }
 
 // Pair p of a row map (MAP_ADJ: 2p, 2p+1; MAP_ROPE: the NEOX pair (i, i + 32) of one
@@ -173,10 +174,11 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 }
 
 template <int BT, typename WT, bool I8, int PRO, int EPI, int MAP>
-__global__ void __launch_bounds__(kGemvThreadsWS, 2) k_gemv(const GemvArgs a, int KC, int NS) {
+__global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, int KC, int NS) {
     using AccT = typename std::conditional<I8, int, float>::type;
     using XT = typename std::conditional<I8, int8_t, float>::type;
-    constexpr int NWC = kGemvConsumerWarps;
+    constexpr int NWC = gemv_consumer_warps(BT);
+    constexpr int NT = gemv_threads(BT);
     constexpr int R = gemv_rows_per_task(BT);   // weight rows per warp task
     constexpr int P = R / 2;                    // row pairs per task
     constexpr int ROWS_PER_BLOCK = R * NWC;
@@ -242,17 +244,40 @@ __global__ void __launch_bounds__(kGemvThreadsWS, 2) k_gemv(const GemvArgs a, in
                 if (rows[r] >= 0) total += row_bytes;
         }
         mbar_arrive_expect_tx(&full[stage], total);
+        // slots in order; runs of consecutive full rows of one matrix move as one copy
+        int run_row = -1, run_len = 0, run_slot = 0;
+        const void* run_base = nullptr;
+        auto flush = [&]() {
+            if (run_len > 0) {
+                const WT* g = reinterpret_cast<const WT*>(run_base) + static_cast<long long>(run_row) * a.K + k0;
+                bulk_g2s(dst + static_cast<size_t>(run_slot) * KC * sizeof(WT), g, row_bytes * run_len, &full[stage]);
+            }
+            run_len = 0;
+        };
         for (int w = 0; w < NWC; ++w) {
             int rows[R];
             task_rows(jb * NWC + w, rows);
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                if (rows[r] < 0) continue;
+                const int slot = w * R + r;
                 const void* base = (MAP == MAP_DUAL && (r & 1)) ? a.W2 : a.W;
-                const WT* g = reinterpret_cast<const WT*>(base) + static_cast<long long>(rows[r]) * a.K + k0;
-                bulk_g2s(dst + static_cast<size_t>(w * R + r) * KC * sizeof(WT), g, row_bytes, &full[stage]);
+                if (rows[r] < 0) {
+                    flush();
+                    continue;
+                }
+                if (run_len > 0 && nkc == 1 && base == run_base && rows[r] == run_row + run_len &&
+                    slot == run_slot + run_len) {
+                    ++run_len;
+                } else {
+                    flush();
+                    run_row = rows[r];
+                    run_base = base;
+                    run_slot = slot;
+                    run_len = 1;
+                }
             }
         }
+        flush();
     };
 
     // weights do not depend on the previous kernel: start streaming before the wait
@@ -364,7 +389,7 @@ __global__ void __launch_bounds__(kGemvThreadsWS, 2) k_gemv(const GemvArgs a, in
     if (PRO != PRO_RAW_I8 && (PRO != PRO_NONE || I8 || nb < BT)) {
         const int K4 = a.K >> 2;
         const int total = BT * K4;
-        for (int e = tid; e < total; e += kGemvThreadsWS) {
+        for (int e = tid; e < total; e += NT) {
             const int b = e / K4, k4 = e - b * K4;
             float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
             if (b < nb) {
@@ -392,7 +417,7 @@ __global__ void __launch_bounds__(kGemvThreadsWS, 2) k_gemv(const GemvArgs a, in
             }
         }
     } else if (PRO == PRO_RAW_I8 && nb < BT) {
-        for (int e = nb * (a.K >> 2) + tid; e < BT * (a.K >> 2); e += kGemvThreadsWS)
+        for (int e = nb * (a.K >> 2) + tid; e < BT * (a.K >> 2); e += NT)
             reinterpret_cast<uint32_t*>(sX)[e] = 0u;
     }
     __syncthreads();
@@ -562,7 +587,7 @@ __global__ void __launch_bounds__(kGemvThreadsWS, 2) k_gemv(const GemvArgs a, in
         __syncthreads();
         if (s_last) {
             __threadfence();
-            for (int b = tid; b < a.B; b += kGemvThreadsWS) {
+            for (int b = tid; b < a.B; b += NT) {
                 const unsigned long long k = atomicExch(&a.keys[b], 0ull);
                 const int idx = (k == 0ull) ? 0 : argmax_key_index(k);
                 if (a.argmax_out) a.argmax_out[b] = idx;

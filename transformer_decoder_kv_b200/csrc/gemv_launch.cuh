@@ -37,8 +37,8 @@ template <typename WT, bool I8, int PRO>
 GemvPlan gemv_plan(int BT, int K) {
     GemvPlan p;
     const int elt_w = sizeof(WT);
-    const int rows_per_block = gemv_rows_per_task(BT) * kGemvConsumerWarps;
-    // one stage = rows_per_block rows x KC columns
+    const int rows_per_block = gemv_rows_per_task(BT) * gemv_consumer_warps(BT);
+    // one stage = rows_per_block rows x KC columns (whole rows when they fit)
     int kc = gemv_stage_bytes(BT) / (rows_per_block * elt_w);
     kc = std::min(kc, K);
     kc = std::max(16, kc / 16 * 16);
@@ -67,12 +67,16 @@ cudaError_t gemv_launch_bt(int num_sms, const GemvArgs& a, cudaStream_t st) {
     if (!attr_set) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemvSmemMax - 2048));
         if (e != cudaSuccess) return e;
+        // one shared-memory carveout for every kernel of the step, so that consecutive
+        // kernels can share an SM without reconfiguring it
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
         attr_set = true;
     }
     const int n_pairs = (MAP == MAP_DUAL) ? a.N : (a.N + 1) / 2;
     const int pairs_per_task = gemv_rows_per_task(BT) / 2;
     const int n_tasks = (n_pairs + pairs_per_task - 1) / pairs_per_task;
-    const int n_blocks = (n_tasks + kGemvConsumerWarps - 1) / kGemvConsumerWarps;
+    const int n_blocks = (n_tasks + gemv_consumer_warps(BT) - 1) / gemv_consumer_warps(BT);
     // occupancy for this instantiation, cached per shared-memory size
     static size_t occ_smem[4] = {~size_t(0), ~size_t(0), ~size_t(0), ~size_t(0)};
     static int occ_val[4] = {0, 0, 0, 0};
@@ -81,7 +85,7 @@ cudaError_t gemv_launch_bt(int num_sms, const GemvArgs& a, cudaStream_t st) {
     for (int i = 0; i < 4; ++i)
         if (occ_smem[i] == p.smem) occ = occ_val[i];
     if (occ < 0) {
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGemvThreadsWS, p.smem);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, gemv_threads(BT), p.smem);
         if (e != cudaSuccess) return e;
         occ_smem[occ_next] = p.smem;
         occ_val[occ_next] = occ;
@@ -91,7 +95,7 @@ cudaError_t gemv_launch_bt(int num_sms, const GemvArgs& a, cudaStream_t st) {
     const int gx = std::max(1, std::min(n_blocks, (num_sms * std::max(1, occ)) / gy));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(gx, gy);
-    cfg.blockDim = dim3(kGemvThreadsWS);
+    cfg.blockDim = dim3(gemv_threads(BT));
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
