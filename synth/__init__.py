@@ -174,8 +174,17 @@ WORKLOADS: Dict[str, Workload] = {
     "tiny_whisper_w8a32_b3": Workload("tiny_whisper_w8a32_b3", MODELS["tiny_whisper_w8a32"],
                                       batch=3, max_cache_len=64, cache_init="prefill", lens_lo=1,
                                       lens_hi=20, steps=6),
+    # batch 9: the tensor-core projection path (batch tiles of 16)
+    "tiny_whisper_b9": Workload("tiny_whisper_b9", MODELS["tiny_whisper"], batch=9,
+                                max_cache_len=64, cache_init="prefill", lens_lo=1, lens_hi=20,
+                                steps=4),
+    "tiny_whisper_w8a32_b9": Workload("tiny_whisper_w8a32_b9", MODELS["tiny_whisper_w8a32"],
+                                      batch=9, max_cache_len=64, cache_init="prefill", lens_lo=1,
+                                      lens_hi=20, steps=4),
     "tiny_qwen2_b3": Workload("tiny_qwen2_b3", MODELS["tiny_qwen2"], batch=3, max_cache_len=96,
                               cache_init="prefill", lens_lo=1, lens_hi=40, steps=6),
+    "tiny_qwen2_b9": Workload("tiny_qwen2_b9", MODELS["tiny_qwen2"], batch=9, max_cache_len=96,
+                              cache_init="prefill", lens_lo=1, lens_hi=40, steps=4),
     "small_qwen2_kv_b5": Workload("small_qwen2_kv_b5", MODELS["small_qwen2"], batch=5,
                                   max_cache_len=700, cache_init="kv_seed", lens_lo=1,
                                   lens_hi=600, steps=4),

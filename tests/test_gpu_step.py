@@ -50,7 +50,8 @@ def _run(wl_name, steps=None, seed=0):
 
 
 @pytest.mark.parametrize("wl_name", ["tiny_whisper_b3", "tiny_qwen2_b3", "tiny_whisper_w8a32_b3",
-                                     "small_qwen2_kv_b5"])
+                                     "small_qwen2_kv_b5", "tiny_whisper_b9", "tiny_whisper_w8a32_b9",
+                                     "tiny_qwen2_b9"])
 def test_step_matches_oracle(wl_name):
     _run(wl_name)
 
@@ -142,3 +143,35 @@ def test_errors_are_rejected_before_any_work():
     assert status(lambda: q.gpu.step(1, None, [0], [8], [8])) == binding.DEC_EOVERFLOW
     for x in (p, fresh, q):
         x.gpu.close()
+
+
+def test_tensor_core_path_is_batch_invariant_bitwise():
+    """Batch 9 (two 8-column tiles) and batch 8 (one tile) give the same bits for the
+    same stream: each output column of the tensor-core projections depends only on its
+    own activation row."""
+    for wl_name in ("tiny_whisper_b9", "tiny_whisper_w8a32_b9"):
+        wl = synth.workload(wl_name)
+        p9 = build_pair(wl)
+        p8 = build_pair(wl, streams=list(range(8)), max_slots=8)
+        toks = list(range(100, 109))
+        l9 = step_both(p9, toks)[0]
+        l8 = step_both(p8, toks[:8])[0]
+        assert np.array_equal(l9[:8].view(np.uint32), l8.view(np.uint32)), wl_name
+        p9.gpu.close()
+        p8.gpu.close()
+
+
+def test_w8a8_tensor_core_path_equals_dp4a_path_bitwise():
+    """W8A8 products are exact integer sums on both paths (int8 tensor cores from batch 8
+    on, dp4a below) and the quantiser is shared, so a stream's hidden state after the
+    layers is bit-identical in a batch of 9 and stepped alone."""
+    wl = synth.workload("tiny_qwen2_b9")
+    p9 = build_pair(wl)
+    toks = list(range(200, 209))
+    h9 = step_both(p9, toks)[2]
+    for s in (0, 5, 8):
+        p1 = build_pair(wl, streams=[s], max_slots=1)
+        h1 = step_both(p1, [toks[s]])[2]
+        assert np.array_equal(h9[s].view(np.uint32), h1[0].view(np.uint32)), s
+        p1.gpu.close()
+    p9.gpu.close()

@@ -47,7 +47,9 @@ struct AttnArgs {
     long long out_bstride;
     float* part;           // [B * H * S * 68] partial states
     int* counters;         // [B * H] arrival counts, zero between launches
-    int S;                 // splits (gridDim.x)
+    int S;                 // splits (gridDim.x), the partial-state stride per row
+    int tps;               // 64-key tiles per split; 0: ceil(tiles / S) per row
+    int stages;            // shared-memory pipeline stages (1..3); 0: 3
     int* err;              // device status word
 };
 
@@ -64,7 +66,8 @@ __device__ __forceinline__ void attn_issue(float* sK, float* sV, uint64_t* bar, 
 static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArgs a) {
     extern __shared__ __align__(128) unsigned char attn_smem[];
     float* sK = reinterpret_cast<float*>(attn_smem);
-    float* sV = sK + kAttnStages * kAttnTile * kHeadDim;
+    const int NS = (a.stages > 0 && a.stages <= kAttnStages) ? a.stages : kAttnStages;
+    float* sV = sK + NS * kAttnTile * kHeadDim;
     __shared__ __align__(8) uint64_t bars[kAttnStages];
     __shared__ __align__(16) float sq[kHeadDim];
     __shared__ float wm[4], wl[4];
@@ -95,7 +98,9 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
         return;
     }
     const int ntiles = (n + kAttnTile - 1) / kAttnTile;
-    const int tps = (ntiles + a.S - 1) / a.S;
+    // a row's split boundaries depend only on its own length when tps is fixed, which
+    // keeps every row's summation order independent of the rest of the batch
+    const int tps = a.tps > 0 ? a.tps : (ntiles + a.S - 1) / a.S;
     const int active = (ntiles + tps - 1) / tps;
     const int t0 = s * tps;
     const int t1 = min(ntiles, t0 + tps);
@@ -109,9 +114,9 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
     const int first_new_tile = (a.mode == ATTN_SELF) ? (n - 1) / kAttnTile : ntiles;
     int pre = 0;
     if (tid == 0) {
-        for (int i = 0; i < kAttnStages; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
-        for (; pre < kAttnStages && t0 + pre < t1 && t0 + pre < first_new_tile; ++pre)
+        for (; pre < NS && t0 + pre < t1 && t0 + pre < first_new_tile; ++pre)
             attn_issue(sK + pre * kAttnTile * kHeadDim, sV + pre * kAttnTile * kHeadDim, &bars[pre], Kb,
                        Vb, t0 + pre, n);
     }
@@ -119,7 +124,7 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
     if (a.mode != ATTN_OP) pdl_wait();
     if (tid < kHeadDim) sq[tid] = a.q[b * a.q_bstride + h * kHeadDim + tid];
     if (tid == 0) {
-        for (int i = pre; i < kAttnStages && t0 + i < t1; ++i)
+        for (int i = pre; i < NS && t0 + i < t1; ++i)
             attn_issue(sK + i * kAttnTile * kHeadDim, sV + i * kAttnTile * kHeadDim, &bars[i], Kb,
                        Vb, t0 + i, n);
     }
@@ -131,18 +136,17 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
 
     for (int t = t0; t < t1; ++t) {
         const int it = t - t0;
-        const int stage = it % kAttnStages;
-        const uint32_t phase = static_cast<uint32_t>(it / kAttnStages) & 1u;
+        const int stage = it % NS;
+        const uint32_t phase = static_cast<uint32_t>(it / NS) & 1u;
         if (tid == 0) s_flag = mbar_wait_bounded(&bars[stage], phase, a.err) ? 1 : 0;
         __syncthreads();
         if (!s_flag) {
             // Give the copies still in flight a bounded chance to land before the
             // shared memory is released, then leave.
             if (tid == 0) {
-                for (int t2 = t; t2 < min(t1, t + kAttnStages); ++t2) {
+                for (int t2 = t; t2 < min(t1, t + NS); ++t2) {
                     const int it2 = t2 - t0;
-                    mbar_wait_bounded(&bars[it2 % kAttnStages],
-                                      static_cast<uint32_t>(it2 / kAttnStages) & 1u, nullptr);
+                    mbar_wait_bounded(&bars[it2 % NS], static_cast<uint32_t>(it2 / NS) & 1u, nullptr);
                 }
             }
             __syncthreads();
@@ -197,9 +201,9 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
             m = mnew;
         }
         __syncthreads();
-        if (tid == 0 && t + kAttnStages < t1)
+        if (tid == 0 && t + NS < t1)
             attn_issue(sK + stage * kAttnTile * kHeadDim, sV + stage * kAttnTile * kHeadDim,
-                       &bars[stage], Kb, Vb, t + kAttnStages, n);
+                       &bars[stage], Kb, Vb, t + NS, n);
     }
 
     // merge the four warps
@@ -242,15 +246,24 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
     if (!s_last) return;
     __threadfence();
     const float* base = a.part + (static_cast<long long>(b) * a.H + h) * a.S * kAttnPartStride;
+    // the split maxima and sums are fetched in parallel (one thread each, at most 32
+    // splits), then every output dim sums the splits in split order
+    __shared__ float pm[32], pl[32], pw[32];
+    if (tid < active) {
+        pm[tid] = __ldcg(base + tid * kAttnPartStride);
+        pl[tid] = __ldcg(base + tid * kAttnPartStride + 1);
+    }
+    __syncthreads();
+    float M2 = -INFINITY;
+    for (int i = 0; i < active; ++i) M2 = fmaxf(M2, pm[i]);
+    if (tid < active) pw[tid] = (pm[tid] == -INFINITY) ? 0.0f : expf(pm[tid] - M2);
+    __syncthreads();
     if (tid < kHeadDim) {
-        float M2 = -INFINITY;
-        for (int i = 0; i < active; ++i) M2 = fmaxf(M2, __ldcg(base + i * kAttnPartStride));
         float L2 = 0.0f, o = 0.0f;
+#pragma unroll 8
         for (int i = 0; i < active; ++i) {
-            const float mi = __ldcg(base + i * kAttnPartStride);
-            const float e = (mi == -INFINITY) ? 0.0f : expf(mi - M2);
-            L2 = fmaf(e, __ldcg(base + i * kAttnPartStride + 1), L2);
-            o = fmaf(e, __ldcg(base + i * kAttnPartStride + 4 + tid), o);
+            L2 = fmaf(pw[i], pl[i], L2);
+            o = fmaf(pw[i], __ldcg(base + i * kAttnPartStride + 4 + tid), o);
         }
         outp[tid] = (L2 > 0.0f && isfinite(L2)) ? o / L2 : 0.0f;
     }

@@ -22,6 +22,8 @@
 #include "gemv.cuh"
 #include "gemv_launch.cuh"
 #include "misc.cuh"
+#include "proj_i8mma.cuh"
+#include "proj_mma.cuh"
 
 using namespace dec;
 
@@ -52,7 +54,16 @@ struct LayerDev {
     float *s1 = nullptr, *s2 = nullptr, *b1 = nullptr, *b2 = nullptr;
     void *wg = nullptr, *wu = nullptr, *wd = nullptr;
     float *sg = nullptr, *su = nullptr, *sd = nullptr;
+    // Qwen tensor-core path: q|k|v rows in RoPE pair order, gate/up rows interleaved
+    void *wqkv_p = nullptr, *wgu = nullptr;
+    // 2-D TMA descriptors of the projections (tensor-core path); Qwen uses m_qkv (the
+    // permuted panel), m_o, m_1 (gate/up) and m_2 (down)
+    CUtensorMap m_qkv, m_o, m_xq, m_xo, m_1, m_2;
 };
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 }  // namespace
 
@@ -64,14 +75,24 @@ struct dec_handle {
     std::vector<void*> hallocs;
     float *tok_emb = nullptr, *pos_emb = nullptr, *final_w = nullptr, *final_b = nullptr;
     float2* rope = nullptr;
+    CUtensorMap m_head;            // TMA descriptor of the tied head (tensor-core path)
+    bool tma_ok = false;           // descriptors built (else the CUDA-core path is used)
     std::vector<LayerDev> layers;
     float *kc = nullptr, *vc = nullptr, *xkc = nullptr, *xvc = nullptr;
     long long self_slot_stride = 0, self_layer_stride = 0, cross_slot_stride = 0, cross_layer_stride = 0;
     int max_batch = 0;
+    int tps_self = 1, tps_cross = 1;   // attention tiles per split (handle constants)
     // workspace
     float *x = nullptr, *q = nullptr, *ctx = nullptr, *ffn = nullptr, *xq = nullptr;
     float* part = nullptr;
     int* counters = nullptr;
+    float* xn = nullptr;            // normalised activation rows (tensor-core path)
+    int8_t* xq8 = nullptr;          // quantised activation rows and their scales (int8 tensor-core path)
+    float* xs8 = nullptr;
+    void* mma_part = nullptr;       // split-K partial tiles (tensor-core path)
+    size_t mma_part_bytes = 0;
+    int* mma_cnt = nullptr;         // split-K arrival counts, zero between launches
+    int mma_cnt_len = 0;
     unsigned long long* keys = nullptr;
     int* head_counter = nullptr;
     int* last_tok = nullptr;
@@ -242,11 +263,109 @@ dec_status gemv(dec_handle* h, const GemvArgs& a, cudaStream_t st) {
     return DEC_OK;
 }
 
-// Whisper projections exist as f32 or W8A32.
+// Batches of at least this many rows take the tensor-core projection path.
+constexpr int kMmaMinBatch = 8;
+
+bool mma_eligible(const dec_handle* h, int N, int K, int elt, int B) {
+    if (!h->tma_ok || B < kMmaMinBatch) return false;
+    const MmaPlan p = mma_plan(N, K, elt, h->num_sms);
+    if (!p.ok || K > kRowprepMaxK) return false;
+    return p.n_ks == 1 || (mma_part_bytes(p, B) <= h->mma_part_bytes && mma_counters(p, B) <= h->mma_cnt_len);
+}
+
+// Norm prologue of the tensor-core path: normalised rows into h->xn, which becomes the
+// projection's input.
+template <int PRO>
+dec_status mma_input(dec_handle* h, GemvArgs& g, cudaStream_t st) {
+    if (PRO == PRO_NONE) return DEC_OK;
+    const cudaError_t e = rowprep_launch<PRO>(g, h->xn, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "row normalisation launch");
+    g.x = h->xn;
+    g.x_ld = g.K;
+    return DEC_OK;
+}
+
+template <typename WT, int PRO, int EPI>
+dec_status proj_mma(dec_handle* h, const GemvArgs& a, const CUtensorMap& map, cudaStream_t st) {
+    GemvArgs g = a;
+    DEC_TRY(mma_input<PRO>(h, g, st));
+    const cudaError_t e =
+        proj_mma_launch<WT, EPI>(h->num_sms, map, h->mma_part, h->mma_part_bytes, h->mma_cnt, h->mma_cnt_len, g, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "tensor-core projection launch");
+    return DEC_OK;
+}
+
+bool i8mma_eligible(const dec_handle* h, int n_rows, int K, int B) {
+    if (!h->tma_ok || B < kMmaMinBatch) return false;
+    const MmaPlan p = i8mma_plan(n_rows, K, h->num_sms);
+    if (!p.ok) return false;
+    return p.n_ks == 1 || (i8mma_part_bytes(p, B) <= h->mma_part_bytes && i8mma_counters(p, B) <= h->mma_cnt_len);
+}
+
+// W8A8 on int8 tensor cores: rows quantised by k_rowprep_i8, exact int32 products.
 template <int PRO, int EPI, int MAP>
-dec_status gemv_whisper(dec_handle* h, const GemvArgs& a, cudaStream_t st) {
-    if (h->cfg.proj_fmt == DEC_PROJ_F32) return gemv<float, false, PRO, EPI, MAP>(h, a, st);
+dec_status proj_w8a8_mma(dec_handle* h, const GemvArgs& a, const CUtensorMap& map, int n_rows, cudaStream_t st) {
+    cudaError_t e = rowprep_i8_launch<PRO>(a, h->xq8, h->xs8, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "row quantisation launch");
+    e = proj_i8mma_launch<EPI, MAP>(h->num_sms, map, n_rows, h->xq8, h->xs8, h->mma_part, h->mma_part_bytes,
+                                       h->mma_cnt, h->mma_cnt_len, a, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "int8 tensor-core projection launch");
+    return DEC_OK;
+}
+
+// Whisper projections exist as f32 or W8A32: tensor cores from batch 8 on, the
+// CUDA-core kernel below.
+template <int PRO, int EPI, int MAP>
+dec_status gemv_whisper(dec_handle* h, const GemvArgs& a, cudaStream_t st, const CUtensorMap* map = nullptr) {
+    const bool f32w = h->cfg.proj_fmt == DEC_PROJ_F32;
+    if (map != nullptr) {
+        if (f32w && mma_eligible(h, a.N, a.K, 4, a.B)) return proj_mma<float, PRO, EPI>(h, a, *map, st);
+        if (!f32w && mma_eligible(h, a.N, a.K, 1, a.B)) return proj_mma<int8_t, PRO, EPI>(h, a, *map, st);
+    }
+    if (f32w) return gemv<float, false, PRO, EPI, MAP>(h, a, st);
     return gemv<int8_t, false, PRO, EPI, MAP>(h, a, st);
+}
+
+// Qwen W8A8 projections: int8 tensor cores from batch 8 on, dp4a below (bit-identical).
+template <int PRO, int EPI, int MAP>
+dec_status gemv_qwen(dec_handle* h, const GemvArgs& a, const CUtensorMap& map, cudaStream_t st) {
+    const int n_rows = MAP == MAP_DUAL ? 2 * a.N : a.N;
+    if (i8mma_eligible(h, n_rows, a.K, a.B)) return proj_w8a8_mma<PRO, EPI, MAP>(h, a, map, n_rows, st);
+    return gemv<int8_t, true, PRO, EPI, MAP>(h, a, st);
+}
+
+// Final norm + tied head: tensor cores from batch 8 on, CUDA cores below.
+template <int PRO>
+dec_status head(dec_handle* h, const GemvArgs& a, cudaStream_t st) {
+    if (mma_eligible(h, a.N, a.K, 4, a.B)) return proj_mma<float, PRO, EPI_HEAD>(h, a, h->m_head, st);
+    return gemv<float, false, PRO, EPI_HEAD, MAP_ADJ>(h, a, st);
+}
+
+// 2-D TMA descriptor of a row-major [rows, cols] weight matrix (f32 or int8): boxes of
+// 128 rows x 128 bytes with the 128-byte swizzle, zero fill outside the matrix.
+dec_status make_wmap(dec_handle* h, CUtensorMap* m, const void* w, int rows, int cols, bool f32) {
+    static EncodeTiledFn encode = nullptr;
+    if (encode == nullptr) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr) {
+            cudaGetLastError();
+            return fail(h, DEC_ECUDA, "cuTensorMapEncodeTiled is not available");
+        }
+        encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    const int elt = f32 ? 4 : 1;
+    const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(cols) * elt};
+    const cuuint32_t box[2] = {cuuint32_t(128 / elt), cuuint32_t(kMmaBlockRows)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                              const_cast<void*>(w), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(h, DEC_ECUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(r) + ")");
+    return DEC_OK;
 }
 
 // Split count for one attention launch: minimise (waves x tiles per CTA).
@@ -269,7 +388,7 @@ int choose_splits(const dec_handle* h, int rows, int max_tiles) {
     return best;
 }
 
-dec_status attention(dec_handle* h, AttnArgs a, int B, int max_keys, cudaStream_t st) {
+dec_status attention(dec_handle* h, AttnArgs a, int B, int max_keys, int tps, cudaStream_t st) {
     static int configured = 0;
     if (!configured) {
         DEC_CUDA(h, cudaFuncSetAttribute(k_attention, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kAttnSmemBytes)));
@@ -277,10 +396,26 @@ dec_status attention(dec_handle* h, AttnArgs a, int B, int max_keys, cudaStream_
                                          cudaSharedmemCarveoutMaxShared));
         configured = 1;
     }
+    // fixed tiles per split (a handle constant): each row's split boundaries, hence its
+    // summation order, depend only on its own length
     const int max_tiles = (max_keys + kAttnTile - 1) / kAttnTile;
-    a.S = choose_splits(h, B * a.H, max_tiles);
-    DEC_CUDA(h, launch(k_attention, dim3(a.S, a.H, B), dim3(kAttnThreads), kAttnSmemBytes, st, a));
+    a.tps = tps;
+    a.S = std::max(1, (max_tiles + tps - 1) / tps);
+    // one stage per CTA (more resident CTAs) up to 4 tiles per split, two beyond:
+    // measured on B200 as the fastest for both ragged self-attention and cross-attention
+    a.stages = tps >= 8 ? 2 : 1;
+    const size_t smem = size_t(a.stages) * 2 * kAttnTile * kHeadDim * sizeof(float);
+    DEC_CUDA(h, launch(k_attention, dim3(a.S, a.H, B), dim3(kAttnThreads), smem, st, a));
     return DEC_OK;
+}
+
+// Tiles per split for a handle: finer splits when few (stream, head) rows exist, and
+// never more than kMaxSplits splits over the longest possible row.
+int tiles_per_split(const dec_handle* h, int max_keys) {
+    const int rows_cap = h->cfg.n_heads * h->max_batch;
+    int t = rows_cap <= 32 ? 1 : (rows_cap <= 1023 ? 4 : 8);
+    const int tiles_cap = (max_keys + kAttnTile - 1) / kAttnTile;
+    return std::max(t, (tiles_cap + kMaxSplits - 1) / kMaxSplits);
 }
 
 GemvArgs base_args(dec_handle* h, int B) {
@@ -321,10 +456,10 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
         g.ld = c.max_cache_len;
         g.d = d;
         if (c.family == DEC_FAMILY_WHISPER) {
-            DEC_TRY((gemv_whisper<PRO_LN, EPI_QKV, MAP_ADJ>(h, g, st)));
+            DEC_TRY((gemv_whisper<PRO_LN, EPI_QKV, MAP_ADJ>(h, g, st, &L.m_qkv)));
         } else {
             g.rope = h->rope;
-            DEC_TRY((gemv<int8_t, true, PRO_RMS, EPI_QKV, MAP_ROPE>(h, g, st)));
+            DEC_TRY((gemv_qwen<PRO_RMS, EPI_QKV, MAP_ROPE>(h, g, L.m_qkv, st)));
         }
         // ---- self-attention over rows 0..len ----
         AttnArgs at{};
@@ -342,7 +477,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
         at.part = h->part;
         at.counters = h->counters;
         at.err = h->dev_err;
-        DEC_TRY(attention(h, at, B, max_len_plus1, st));
+        DEC_TRY(attention(h, at, B, max_len_plus1, h->tps_self, st));
         // ---- output projection + residual ----
         g = base_args(h, B);
         g.x = h->ctx;
@@ -355,9 +490,9 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
         g.out = h->x;
         g.out_ld = d;
         if (c.family == DEC_FAMILY_WHISPER) {
-            DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st)));
+            DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st, &L.m_o)));
         } else {
-            DEC_TRY((gemv<int8_t, true, PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st)));
+            DEC_TRY((gemv_qwen<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, L.m_o, st)));
         }
         if (c.family == DEC_FAMILY_WHISPER) {
             // ---- cross-attention block ----
@@ -373,7 +508,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             g.bias = L.bxq;
             g.out = h->xq;
             g.out_ld = d;
-            DEC_TRY((gemv_whisper<PRO_LN, EPI_STORE, MAP_ADJ>(h, g, st)));
+            DEC_TRY((gemv_whisper<PRO_LN, EPI_STORE, MAP_ADJ>(h, g, st, &L.m_xq)));
             at.q = h->xq;
             at.k = h->xkc + l * h->cross_layer_stride;
             at.v = h->xvc + l * h->cross_layer_stride;
@@ -381,7 +516,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             at.ld = c.enc_len;
             at.mode = ATTN_CROSS;
             at.n_fixed = c.enc_len;
-            DEC_TRY(attention(h, at, B, c.enc_len, st));
+            DEC_TRY(attention(h, at, B, c.enc_len, h->tps_cross, st));
             g = base_args(h, B);
             g.x = h->ctx;
             g.x_ld = d;
@@ -392,7 +527,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             g.bias = L.bxo;
             g.out = h->x;
             g.out_ld = d;
-            DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st)));
+            DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st, &L.m_xo)));
             // ---- GELU FFN ----
             g = base_args(h, B);
             g.x = h->x;
@@ -406,7 +541,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             g.bias = L.b1;
             g.out = h->ffn;
             g.out_ld = F;
-            DEC_TRY((gemv_whisper<PRO_LN, EPI_GELU, MAP_ADJ>(h, g, st)));
+            DEC_TRY((gemv_whisper<PRO_LN, EPI_GELU, MAP_ADJ>(h, g, st, &L.m_1)));
             g = base_args(h, B);
             g.x = h->ffn;
             g.x_ld = F;
@@ -417,7 +552,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             g.bias = L.b2;
             g.out = h->x;
             g.out_ld = d;
-            DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st)));
+            DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st, &L.m_2)));
         } else {
             // ---- SwiGLU MLP ----
             g = base_args(h, B);
@@ -432,7 +567,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             g.scale2 = L.su;
             g.out = h->ffn;
             g.out_ld = F;
-            DEC_TRY((gemv<int8_t, true, PRO_RMS, EPI_SWIGLU, MAP_DUAL>(h, g, st)));
+            DEC_TRY((gemv_qwen<PRO_RMS, EPI_SWIGLU, MAP_DUAL>(h, g, L.m_1, st)));
             g = base_args(h, B);
             g.x = h->ffn;
             g.x_ld = F;
@@ -442,7 +577,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             g.scale = L.sd;
             g.out = h->x;
             g.out_ld = d;
-            DEC_TRY((gemv<int8_t, true, PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st)));
+            DEC_TRY((gemv_qwen<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, L.m_2, st)));
         }
     }
     // ---- final norm + tied head + greedy argmax ----
@@ -461,9 +596,9 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
     g.argmax_out = argmax;
     g.last_tok = h->last_tok;
     if (c.family == DEC_FAMILY_WHISPER) {
-        DEC_TRY((gemv<float, false, PRO_LN, EPI_HEAD, MAP_ADJ>(h, g, st)));
+        DEC_TRY(head<PRO_LN>(h, g, st));
     } else {
-        DEC_TRY((gemv<float, false, PRO_RMS, EPI_HEAD, MAP_ADJ>(h, g, st)));
+        DEC_TRY(head<PRO_RMS>(h, g, st));
     }
     return DEC_OK;
 }
@@ -639,6 +774,37 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
             DEC_TRY(upload_proj(h, W.down, d, F, false, &D.wd, &D.sd, &nobias, "down"));
         }
     }
+    // TMA descriptors of the tensor-core projection path (the head, every projection);
+    // without them the CUDA-core kernels run instead. The Qwen q|k|v and gate/up panels
+    // get row-permuted copies for the int8 kernel's RoPE and SwiGLU row maps.
+    {
+        const bool f32w = c.proj_fmt == DEC_PROJ_F32;
+        dec_status ts = make_wmap(h, &h->m_head, h->tok_emb, c.vocab, d, true);
+        for (int l = 0; l < L && ts == DEC_OK; ++l) {
+            LayerDev& D = h->layers[l];
+            if (wh) {
+                ts = make_wmap(h, &D.m_qkv, D.wqkv, 3 * d, d, f32w);
+                if (ts == DEC_OK) ts = make_wmap(h, &D.m_o, D.wo, d, d, f32w);
+                if (ts == DEC_OK) ts = make_wmap(h, &D.m_xq, D.wxq, d, d, f32w);
+                if (ts == DEC_OK) ts = make_wmap(h, &D.m_xo, D.wxo, d, d, f32w);
+                if (ts == DEC_OK) ts = make_wmap(h, &D.m_1, D.w1, F, d, f32w);
+                if (ts == DEC_OK) ts = make_wmap(h, &D.m_2, D.w2, d, F, f32w);
+            } else {
+                DEC_TRY(dalloc(h, &D.wqkv_p, size_t(3) * d * d));
+                DEC_TRY(dalloc(h, &D.wgu, size_t(2) * F * d));
+                DEC_CUDA(h, i8_rows_permute(MAP_ROPE, static_cast<int8_t*>(D.wqkv_p),
+                                            static_cast<const int8_t*>(D.wqkv), nullptr, 3 * d, d, 0));
+                DEC_CUDA(h, i8_rows_permute(MAP_DUAL, static_cast<int8_t*>(D.wgu), static_cast<const int8_t*>(D.wg),
+                                            static_cast<const int8_t*>(D.wu), 2 * F, d, 0));
+                ts = make_wmap(h, &D.m_qkv, D.wqkv_p, 3 * d, d, false);
+                if (ts == DEC_OK) ts = make_wmap(h, &D.m_o, D.wo, d, d, false);
+                if (ts == DEC_OK) ts = make_wmap(h, &D.m_1, D.wgu, 2 * F, d, false);
+                if (ts == DEC_OK) ts = make_wmap(h, &D.m_2, D.wd, d, F, false);
+            }
+        }
+        h->tma_ok = (ts == DEC_OK);
+        if (!h->tma_ok) h->err.clear();
+    }
     // caches
     h->self_slot_stride = (long long)H * c.max_cache_len * 64;
     h->self_layer_stride = h->self_slot_stride * c.max_slots;
@@ -656,6 +822,8 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
     }
     // workspace
     h->max_batch = std::min(c.max_slots, DEC_MAX_BATCH);
+    h->tps_self = tiles_per_split(h, c.max_cache_len);
+    h->tps_cross = wh ? tiles_per_split(h, c.enc_len) : 1;
     const int MB = h->max_batch;
     DEC_TRY(dalloc(h, &h->x, size_t(MB) * d * 4));
     DEC_TRY(dalloc(h, &h->q, size_t(MB) * d * 4));
@@ -665,6 +833,42 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
     DEC_TRY(dalloc(h, &h->part, size_t(MB) * H * kMaxSplits * kAttnPartStride * 4));
     DEC_TRY(dalloc(h, &h->counters, size_t(MB) * H * 4));
     DEC_CUDA(h, cudaMemset(h->counters, 0, size_t(MB) * H * 4));
+    // tensor-core path: normalised / quantised rows and the split-K scratch of the
+    // largest plan
+    if (h->tma_ok) {
+        DEC_TRY(dalloc(h, &h->xn, size_t(MB) * std::max(d, F) * 4));
+        DEC_TRY(dalloc(h, &h->xq8, size_t(MB) * std::max(d, F)));
+        DEC_TRY(dalloc(h, &h->xs8, size_t(MB) * 4));
+        size_t pb = 16;
+        int cl = 1;
+        const int welt = c.proj_fmt == DEC_PROJ_F32 ? 4 : 1;
+        auto need_f32 = [&](int n, int k, int elt) {
+            const MmaPlan p = mma_plan(n, k, elt, h->num_sms);
+            if (!p.ok) return;
+            pb = std::max(pb, mma_part_bytes(p, MB));
+            cl = std::max(cl, mma_counters(p, MB));
+        };
+        auto need_i8 = [&](int n, int k) {
+            const MmaPlan p = i8mma_plan(n, k, h->num_sms);
+            if (!p.ok) return;
+            pb = std::max(pb, i8mma_part_bytes(p, MB));
+            cl = std::max(cl, i8mma_counters(p, MB));
+        };
+        need_f32(c.vocab, d, 4);
+        const int shapes[4][2] = {{3 * d, d}, {d, d}, {F, d}, {d, F}};
+        for (const auto& sh : shapes) {
+            if (!wh) {
+                need_i8(sh[0] == F ? 2 * F : sh[0], sh[1]);
+            } else {
+                need_f32(sh[0], sh[1], welt);
+            }
+        }
+        DEC_TRY(dalloc(h, &h->mma_part, pb));
+        h->mma_part_bytes = pb;
+        DEC_TRY(dalloc(h, &h->mma_cnt, size_t(cl) * 4));
+        DEC_CUDA(h, cudaMemset(h->mma_cnt, 0, size_t(cl) * 4));
+        h->mma_cnt_len = cl;
+    }
     DEC_TRY(dalloc(h, &h->keys, size_t(MB) * 8));
     DEC_CUDA(h, cudaMemset(h->keys, 0, size_t(MB) * 8));
     DEC_TRY(dalloc(h, &h->head_counter, 16));
