@@ -141,6 +141,14 @@ MODELS: Dict[str, ModelConfig] = {
     "small_qwen2": _m(name="small_qwen2", family="qwen2", n_layers=3, d_model=256, n_heads=4,
                       head_dim=64, d_ff=704, vocab=4099, max_pos=32768, enc_len=0,
                       proj_fmt=PROJ_W8A8, norm_eps=1e-6, rope_theta=1e6),
+    # Mid-size models whose matrices are large enough that batches of 8+ take the
+    # tensor-core projection kernels (q|k|v, gate/up, down for W8A8; fc2 for f32).
+    "mid_whisper": _m(name="mid_whisper", family="whisper", n_layers=2, d_model=256, n_heads=4,
+                      head_dim=64, d_ff=2048, vocab=1031, max_pos=64, enc_len=40,
+                      proj_fmt=PROJ_F32, norm_eps=1e-5),
+    "mid_qwen2": _m(name="mid_qwen2", family="qwen2", n_layers=2, d_model=896, n_heads=14,
+                    head_dim=64, d_ff=2432, vocab=1009, max_pos=32768, enc_len=0,
+                    proj_fmt=PROJ_W8A8, norm_eps=1e-6, rope_theta=1e6),
 }
 
 WORKLOADS: Dict[str, Workload] = {
@@ -185,6 +193,10 @@ WORKLOADS: Dict[str, Workload] = {
                               cache_init="prefill", lens_lo=1, lens_hi=40, steps=6),
     "tiny_qwen2_b9": Workload("tiny_qwen2_b9", MODELS["tiny_qwen2"], batch=9, max_cache_len=96,
                               cache_init="prefill", lens_lo=1, lens_hi=40, steps=4),
+    "mid_whisper_b9": Workload("mid_whisper_b9", MODELS["mid_whisper"], batch=9, max_cache_len=64,
+                               cache_init="prefill", lens_lo=1, lens_hi=10, steps=3),
+    "mid_qwen2_b9": Workload("mid_qwen2_b9", MODELS["mid_qwen2"], batch=9, max_cache_len=64,
+                             cache_init="prefill", lens_lo=1, lens_hi=10, steps=3),
     "small_qwen2_kv_b5": Workload("small_qwen2_kv_b5", MODELS["small_qwen2"], batch=5,
                                   max_cache_len=700, cache_init="kv_seed", lens_lo=1,
                                   lens_hi=600, steps=4),

@@ -51,7 +51,7 @@ def _run(wl_name, steps=None, seed=0):
 
 @pytest.mark.parametrize("wl_name", ["tiny_whisper_b3", "tiny_qwen2_b3", "tiny_whisper_w8a32_b3",
                                      "small_qwen2_kv_b5", "tiny_whisper_b9", "tiny_whisper_w8a32_b9",
-                                     "tiny_qwen2_b9"])
+                                     "tiny_qwen2_b9", "mid_whisper_b9", "mid_qwen2_b9"])
 def test_step_matches_oracle(wl_name):
     _run(wl_name)
 
@@ -149,7 +149,7 @@ def test_tensor_core_path_is_batch_invariant_bitwise():
     """Batch 9 (two 8-column tiles) and batch 8 (one tile) give the same bits for the
     same stream: each output column of the tensor-core projections depends only on its
     own activation row."""
-    for wl_name in ("tiny_whisper_b9", "tiny_whisper_w8a32_b9"):
+    for wl_name in ("mid_whisper_b9", "tiny_whisper_w8a32_b9"):
         wl = synth.workload(wl_name)
         p9 = build_pair(wl)
         p8 = build_pair(wl, streams=list(range(8)), max_slots=8)
@@ -165,7 +165,7 @@ def test_w8a8_tensor_core_path_equals_dp4a_path_bitwise():
     """W8A8 products are exact integer sums on both paths (int8 tensor cores from batch 8
     on, dp4a below) and the quantiser is shared, so a stream's hidden state after the
     layers is bit-identical in a batch of 9 and stepped alone."""
-    wl = synth.workload("tiny_qwen2_b9")
+    wl = synth.workload("mid_qwen2_b9")
     p9 = build_pair(wl)
     toks = list(range(200, 209))
     h9 = step_both(p9, toks)[2]

@@ -22,6 +22,7 @@
 #include "gemv.cuh"
 #include "gemv_launch.cuh"
 #include "misc.cuh"
+#include "head_tc.cuh"
 #include "proj_i8mma.cuh"
 #include "proj_mma.cuh"
 
@@ -77,6 +78,12 @@ struct dec_handle {
     float2* rope = nullptr;
     CUtensorMap m_head;            // TMA descriptor of the tied head (tensor-core path)
     bool tma_ok = false;           // descriptors built (else the CUDA-core path is used)
+    // tcgen05 head: embedding and hidden rows as three int8 digit planes with row scales
+    int8_t *wdig = nullptr, *xdig = nullptr;
+    float *wsc = nullptr, *xsc = nullptr;
+    int xdig_rows = 0;             // rows per hidden digit plane (>= max batch, >= 32)
+    CUtensorMap m_wdig, m_xdig16, m_xdig32;
+    bool head_tc_ok = false;
     std::vector<LayerDev> layers;
     float *kc = nullptr, *vc = nullptr, *xkc = nullptr, *xvc = nullptr;
     long long self_slot_stride = 0, self_layer_stride = 0, cross_slot_stride = 0, cross_layer_stride = 0;
@@ -263,8 +270,18 @@ dec_status gemv(dec_handle* h, const GemvArgs& a, cudaStream_t st) {
     return DEC_OK;
 }
 
-// Batches of at least this many rows take the tensor-core projection path.
+// Batches of at least this many rows can take the tensor-core projection paths. Which
+// path runs also depends on the matrix (measured per shape on B200, PDL chains with
+// weights streamed from HBM): below about 2^21 weights with K < 2048 the tensor-core
+// kernels' fixed cost (activation slice load, split-K exchange) is larger than the
+// CUDA-core kernel's whole run, except for int8 weights with f32 activations, whose
+// CUDA-core kernel is arithmetic-bound from batch 8 on.
 constexpr int kMmaMinBatch = 8;
+constexpr long long kMmaMinWeights = 1LL << 21;
+
+bool mma_worth(int N, int K, bool w8a32) {
+    return w8a32 || K >= 2048 || static_cast<long long>(N) * K >= 4 * kMmaMinWeights;
+}
 
 bool mma_eligible(const dec_handle* h, int N, int K, int elt, int B) {
     if (!h->tma_ok || B < kMmaMinBatch) return false;
@@ -319,7 +336,8 @@ template <int PRO, int EPI, int MAP>
 dec_status gemv_whisper(dec_handle* h, const GemvArgs& a, cudaStream_t st, const CUtensorMap* map = nullptr) {
     const bool f32w = h->cfg.proj_fmt == DEC_PROJ_F32;
     if (map != nullptr) {
-        if (f32w && mma_eligible(h, a.N, a.K, 4, a.B)) return proj_mma<float, PRO, EPI>(h, a, *map, st);
+        if (f32w && mma_worth(a.N, a.K, false) && mma_eligible(h, a.N, a.K, 4, a.B))
+            return proj_mma<float, PRO, EPI>(h, a, *map, st);
         if (!f32w && mma_eligible(h, a.N, a.K, 1, a.B)) return proj_mma<int8_t, PRO, EPI>(h, a, *map, st);
     }
     if (f32w) return gemv<float, false, PRO, EPI, MAP>(h, a, st);
@@ -330,20 +348,51 @@ dec_status gemv_whisper(dec_handle* h, const GemvArgs& a, cudaStream_t st, const
 template <int PRO, int EPI, int MAP>
 dec_status gemv_qwen(dec_handle* h, const GemvArgs& a, const CUtensorMap& map, cudaStream_t st) {
     const int n_rows = MAP == MAP_DUAL ? 2 * a.N : a.N;
-    if (i8mma_eligible(h, n_rows, a.K, a.B)) return proj_w8a8_mma<PRO, EPI, MAP>(h, a, map, n_rows, st);
+    if (static_cast<long long>(n_rows) * a.K >= kMmaMinWeights && i8mma_eligible(h, n_rows, a.K, a.B))
+        return proj_w8a8_mma<PRO, EPI, MAP>(h, a, map, n_rows, st);
     return gemv<int8_t, true, PRO, EPI, MAP>(h, a, st);
 }
 
-// Final norm + tied head: tensor cores from batch 8 on, CUDA cores below.
+// Final norm + tied head with the greedy argmax: tcgen05 int8 tensor cores on digit
+// planes at every batch size when they were built, else TF32 tensor cores from batch 8
+// on and CUDA cores below.
 template <int PRO>
 dec_status head(dec_handle* h, const GemvArgs& a, cudaStream_t st) {
+    if (h->head_tc_ok) {
+        const int d = h->cfg.d_model;
+        cudaError_t e = rowprep_digits_launch<PRO>(a.x, a.x_ld, a.norm_w, a.norm_b, a.eps, d, a.B,
+                                                   static_cast<long long>(h->xdig_rows) * d, h->xdig, h->xsc, true, st);
+        if (e != cudaSuccess) return cuda_fail(h, e, "head row split launch");
+        HeadArgs ha;
+        ha.wmap = h->m_wdig;
+        ha.xmap16 = h->m_xdig16;
+        ha.xmap32 = h->m_xdig32;
+        ha.wscale = h->wsc;
+        ha.xscale = h->xsc;
+        ha.V = h->cfg.vocab;
+        ha.K = d;
+        ha.B = a.B;
+        ha.MB = h->xdig_rows;
+        ha.n_by = 1;
+        ha.logits = a.out;
+        ha.keys = a.keys;
+        ha.counter = a.counter;
+        ha.argmax_out = a.argmax_out;
+        ha.last_tok = a.last_tok;
+        ha.meta = a.meta;
+        ha.err = a.err;
+        e = head_tc_launch(h->num_sms, ha, st);
+        if (e != cudaSuccess) return cuda_fail(h, e, "tensor-core head launch");
+        return DEC_OK;
+    }
     if (mma_eligible(h, a.N, a.K, 4, a.B)) return proj_mma<float, PRO, EPI_HEAD>(h, a, h->m_head, st);
     return gemv<float, false, PRO, EPI_HEAD, MAP_ADJ>(h, a, st);
 }
 
-// 2-D TMA descriptor of a row-major [rows, cols] weight matrix (f32 or int8): boxes of
-// 128 rows x 128 bytes with the 128-byte swizzle, zero fill outside the matrix.
-dec_status make_wmap(dec_handle* h, CUtensorMap* m, const void* w, int rows, int cols, bool f32) {
+// 2-D TMA descriptor of a row-major [rows, cols] matrix (f32 or int8): boxes of box_rows
+// rows x 128 bytes with the 128-byte swizzle, zero fill outside the matrix.
+dec_status make_wmap(dec_handle* h, CUtensorMap* m, const void* w, int rows, int cols, bool f32,
+                      int box_rows = kMmaBlockRows) {
     static EncodeTiledFn encode = nullptr;
     if (encode == nullptr) {
         void* fn = nullptr;
@@ -358,7 +407,7 @@ dec_status make_wmap(dec_handle* h, CUtensorMap* m, const void* w, int rows, int
     const int elt = f32 ? 4 : 1;
     const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
     const cuuint64_t strides[1] = {cuuint64_t(cols) * elt};
-    const cuuint32_t box[2] = {cuuint32_t(128 / elt), cuuint32_t(kMmaBlockRows)};
+    const cuuint32_t box[2] = {cuuint32_t(128 / elt), cuuint32_t(box_rows)};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = encode(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
                               const_cast<void*>(w), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -804,6 +853,26 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
         }
         h->tma_ok = (ts == DEC_OK);
         if (!h->tma_ok) h->err.clear();
+    }
+    // tcgen05 head: the embedding's digit planes (once) and the hidden rows' buffers
+    if (h->tma_ok && head_tc_stages(d, 32) > 0) {
+        const long long V = c.vocab;
+        DEC_TRY(dalloc(h, &h->wdig, size_t(3) * V * d));
+        DEC_TRY(dalloc(h, &h->wsc, size_t(V) * 4));
+        DEC_CUDA(h, rowprep_digits_launch<PRO_NONE>(h->tok_emb, d, nullptr, nullptr, 0.0f, d, c.vocab, V * d, h->wdig,
+                                                   h->wsc, false, 0));
+        h->xdig_rows = std::max(std::min(c.max_slots, DEC_MAX_BATCH), 32);
+        const size_t xb = size_t(3) * h->xdig_rows * d;
+        DEC_TRY(dalloc(h, &h->xdig, xb));
+        DEC_CUDA(h, cudaMemset(h->xdig, 0, xb));
+        DEC_TRY(dalloc(h, &h->xsc, size_t(h->xdig_rows) * 4));
+        DEC_CUDA(h, cudaMemset(h->xsc, 0, size_t(h->xdig_rows) * 4));
+        dec_status ts = make_wmap(h, &h->m_wdig, h->wdig, int(3 * V), d, false);
+        if (ts == DEC_OK) ts = make_wmap(h, &h->m_xdig16, h->xdig, 3 * h->xdig_rows, d, false, 16);
+        if (ts == DEC_OK) ts = make_wmap(h, &h->m_xdig32, h->xdig, 3 * h->xdig_rows, d, false, 32);
+        h->head_tc_ok = (ts == DEC_OK);
+        if (!h->head_tc_ok) h->err.clear();
+        DEC_CUDA(h, cudaDeviceSynchronize());
     }
     // caches
     h->self_slot_stride = (long long)H * c.max_cache_len * 64;

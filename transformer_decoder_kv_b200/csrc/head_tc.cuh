@@ -1,0 +1,530 @@
+// Tied LM head on the 5th-generation tensor cores (tcgen05, TMEM accumulators), with the
+// greedy argmax fused: logits[b, n] = sum_k E[n, k] h[b, k] over the f32 token embedding E
+// and the final-normed hidden rows h (cera whisper.rs / franken_ocr decoder_qwen2.rs: the
+// head is tied to the embedding; argmax picks the lowest index among equal maxima).
+//
+// f32 products on integer tensor cores (the splitting idea of Ozaki et al., "Error-free
+// transformations of matrix multiplication by using fast routines of matrix
+// multiplication", 2012; and of Ootomo, Ozaki and Yokota, "DGEMM on integer matrix
+// multiplication unit", 2024): every row r of E and of h is written with a per-row scale
+// s_r = amax_r / 127 as three base-254 int8 digits,
+//     v ~ s_r (d1 + d2 / 254 + d3 / 254^2),  |error| <= 2^-22 amax_r  (digits3 below),
+// the embedding once when the weights are loaded (3 bytes per weight instead of 4), the
+// hidden rows once per step (k_rowprep_digits). The six digit products whose weight is at
+// least 254^-2 go through tcgen05.mma .kind::i8 with exact int32 accumulation in TMEM,
+// grouped by weight into three accumulators
+//     A0 = D1 E1,  A1 = D1 E2 + D2 E1,  A2 = D1 E3 + D2 E2 + D3 E1,
+// and the logit is s_n s_b (A0 + (A1 + A2 / 254) / 254) in f32. The dropped products are
+// below 254^-3 relative; |A| <= 3 * 127^2 * K stays inside int32 for K <= 4096. Because the
+// sums are exact integers, a stream's logits do not depend on which other streams share
+// the batch.
+//
+// CTA (192 threads, one per SM): warp 0 streams the three digit planes of 128-row
+// embedding blocks with 2-D TMA loads (128 rows x 128 bytes per plane, 128-byte swizzle,
+// no multicast) into a ring of 48 KB stages; warp 1 owns the TMEM allocation and issues
+// the MMAs (M = 128 embedding rows, N = BT batch columns, K = 32 per instruction) into one
+// of two TMEM accumulator sets, committing each stage back to the producer and each block
+// to the epilogue; warps 2..5 read the accumulators (tcgen05.ld, one TMEM lane quarter
+// each), write the logits and keep a running argmax key per batch column. The hidden
+// digit planes of the CTA's batch tile are loaded once, by TMA, in the same swizzled
+// K-major layout.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "gemv.cuh"
+
+namespace dec {
+
+constexpr int kHeadThreads = 192;
+constexpr int kHeadRows = 128;                      // embedding rows per block (MMA M)
+constexpr int kHeadKC = 128;                        // K per stage (one 128-byte box per plane)
+constexpr int kHeadPlaneBox = kHeadRows * kHeadKC;  // 16 KB
+constexpr int kHeadStageBytes = 3 * kHeadPlaneBox;  // 48 KB
+constexpr int kHeadMaxStages = 4;
+constexpr int kHeadMaxK = 4096;
+
+struct HeadArgs {
+    CUtensorMap wmap;      // embedding digit planes [3 V, K] int8: box {128 bytes, 128 rows}
+    CUtensorMap xmap16;    // hidden digit planes [3 MB, K] int8: box {128 bytes, 16 rows}
+    CUtensorMap xmap32;    // the same with boxes of 32 rows
+    const float* wscale;   // [V] embedding row scales
+    const float* xscale;   // [MB] hidden row scales
+    int V, K, B, MB;
+    int n_by;              // batch tiles (fastest-varying CTA index)
+    float* logits;         // [B, V] or null
+    unsigned long long* keys;  // [B] argmax keys, zero between launches
+    int* counter;              // CTA arrival count, zero between launches
+    int* argmax_out;           // [B] or null
+    int* last_tok;             // [slots]
+    const StepMeta* meta;
+    int* err;
+};
+
+// Three base-254 digits of v / s with inv = 1 / s (|v| <= amax, so |v inv| <= 127).
+__device__ __forceinline__ void digits3(float v, float inv, int& d1, int& d2, int& d3) {
+    const float r0 = v * inv;
+    const float e1 = fminf(fmaxf(rintf(r0), -127.0f), 127.0f);
+    const float r1 = (r0 - e1) * 254.0f;
+    const float e2 = fminf(fmaxf(rintf(r1), -127.0f), 127.0f);
+    const float r2 = (r1 - e2) * 254.0f;
+    const float e3 = fminf(fmaxf(rintf(r2), -127.0f), 127.0f);
+    d1 = static_cast<int>(e1);
+    d2 = static_cast<int>(e2);
+    d3 = static_cast<int>(e3);
+}
+
+// Digit planes of rows of a row-major f32 matrix: out[p][r][k], scale[r]. One warp per
+// row; `norm` applies the final LayerNorm / RMSNorm first (PRO) with the CUDA-core
+// prologue's arithmetic.
+template <int PRO>
+__global__ void __launch_bounds__(128) k_rowprep_digits(const float* __restrict__ x, int x_ld,
+                                                        const float* __restrict__ gw, const float* __restrict__ gb,
+                                                        float eps, int K, int rows, long long plane_stride,
+                                                        int8_t* __restrict__ out, float* __restrict__ scale) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int r = blockIdx.x * 4 + (threadIdx.x >> 5);
+    if (r >= rows) return;
+    const float4* xr = reinterpret_cast<const float4*>(x + static_cast<long long>(r) * x_ld);
+    const int K4 = K >> 2;
+    float mu = 0.0f, rstd = 1.0f;
+    if (PRO == PRO_LN) {
+        float sum = 0.0f;
+        for (int k = lane; k < K4; k += 32) {
+            const float4 v = xr[k];
+            sum += (v.x + v.y) + (v.z + v.w);
+        }
+        mu = warp_sum(sum) / static_cast<float>(K);
+        float var = 0.0f;
+        for (int k = lane; k < K4; k += 32) {
+            const float4 v = xr[k];
+            const float d0 = v.x - mu, d1 = v.y - mu, d2 = v.z - mu, d3 = v.w - mu;
+            var = fmaf(d0, d0, var);
+            var = fmaf(d1, d1, var);
+            var = fmaf(d2, d2, var);
+            var = fmaf(d3, d3, var);
+        }
+        var = warp_sum(var) / static_cast<float>(K);
+        rstd = 1.0f / sqrtf(var + eps);
+    } else if (PRO == PRO_RMS) {
+        float ss = 0.0f;
+        for (int k = lane; k < K4; k += 32) {
+            const float4 v = xr[k];
+            ss = fmaf(v.x, v.x, ss);
+            ss = fmaf(v.y, v.y, ss);
+            ss = fmaf(v.z, v.z, ss);
+            ss = fmaf(v.w, v.w, ss);
+        }
+        ss = warp_sum(ss) / static_cast<float>(K);
+        rstd = 1.0f / sqrtf(ss + eps);
+    }
+    auto normed = [&](int k) {
+        float4 v = xr[k];
+        if (PRO != PRO_NONE) {
+            const float4 g = __ldg(reinterpret_cast<const float4*>(gw) + k);
+            float4 be = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (PRO == PRO_LN) be = __ldg(reinterpret_cast<const float4*>(gb) + k);
+            v = make_float4(norm_value(PRO, v.x, mu, rstd, g.x, be.x), norm_value(PRO, v.y, mu, rstd, g.y, be.y),
+                            norm_value(PRO, v.z, mu, rstd, g.z, be.z), norm_value(PRO, v.w, mu, rstd, g.w, be.w));
+        }
+        return v;
+    };
+    float amax = 0.0f;
+    for (int k = lane; k < K4; k += 32) {
+        const float4 v = normed(k);
+        amax = fmaxf(fmaxf(amax, fabsf(v.x)), fmaxf(fabsf(v.y), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+    amax = warp_max(amax);
+    const float inv = amax > 0.0f ? 127.0f / amax : 0.0f;
+    uint32_t* o1 = reinterpret_cast<uint32_t*>(out + static_cast<long long>(r) * K);
+    uint32_t* o2 = reinterpret_cast<uint32_t*>(out + plane_stride + static_cast<long long>(r) * K);
+    uint32_t* o3 = reinterpret_cast<uint32_t*>(out + 2 * plane_stride + static_cast<long long>(r) * K);
+    for (int k = lane; k < K4; k += 32) {
+        const float4 v = normed(k);
+        const float e[4] = {v.x, v.y, v.z, v.w};
+        uint32_t p1 = 0, p2 = 0, p3 = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            int a, b, c;
+            digits3(e[j], inv, a, b, c);
+            p1 |= (static_cast<uint32_t>(a) & 0xffu) << (8 * j);
+            p2 |= (static_cast<uint32_t>(b) & 0xffu) << (8 * j);
+            p3 |= (static_cast<uint32_t>(c) & 0xffu) << (8 * j);
+        }
+        o1[k] = p1;
+        o2[k] = p2;
+        o3[k] = p3;
+    }
+    if (lane == 0) scale[r] = amax / 127.0f;
+}
+
+// ---- tcgen05 / TMEM primitives ----------------------------------------------------
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, int8 x int8 -> int32
+__device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// arrive on `bar` once every tcgen05 operation issued so far by this thread has completed
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major operand in the 128-byte-swizzled layout that
+// TMA writes: rows of 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), the
+// leading byte offset unused (1), descriptor version 1, layout type 2 (SWIZZLE_128B).
+__device__ __forceinline__ uint64_t smem_desc_sw128(const void* p) {
+    const uint64_t addr = smem_u32(p);
+    return ((addr & 0x3FFFFull) >> 4) | (1ull << 16) | (uint64_t(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor: int32 accumulator, signed int8 A and B, both K-major, N = n, M = 128.
+__host__ __device__ constexpr uint32_t idesc_i8(int n) {
+    return (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(kHeadRows >> 4) << 24);
+}
+
+template <int BT>
+struct HeadTmemLd;
+template <>
+struct HeadTmemLd<16> {
+    __device__ __forceinline__ static void run(uint32_t taddr, int (&r)[16]) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+              "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+            : "r"(taddr));
+    }
+};
+template <>
+struct HeadTmemLd<32> {
+    __device__ __forceinline__ static void run(uint32_t taddr, int (&r)[32]) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+            "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+              "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+              "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+              "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+            : "r"(taddr));
+    }
+};
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+template <int BT>
+__global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_constant__ HeadArgs A, int NS) {
+    static_assert(BT == 16 || BT == 32, "batch tile");
+    constexpr int ACC = 3 * BT;                           // TMEM columns of one accumulator set
+    constexpr uint32_t TCOLS = BT == 16 ? 128 : 256;      // two sets, power of two
+    constexpr uint32_t IDESC = idesc_i8(BT);
+    const int nch = (A.K + kHeadKC - 1) / kHeadKC;
+    const int xplane = nch * BT * 128;                    // bytes of one hidden digit plane
+
+    extern __shared__ unsigned char head_smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(head_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    unsigned char* ring = smem;                                             // NS x 48 KB
+    unsigned char* sx = smem + static_cast<size_t>(NS) * kHeadStageBytes;   // 3 x xplane
+    __shared__ __align__(8) uint64_t full[kHeadMaxStages], empty[kHeadMaxStages];
+    __shared__ __align__(8) uint64_t tfull[2], tempty[2], bar_x, bar_done;
+    __shared__ uint32_t s_tmem;
+    __shared__ unsigned long long s_key[BT];
+    __shared__ int s_fail, s_last;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n_by = A.n_by;
+    const int by = blockIdx.x % n_by, b0 = by * BT;
+    const int nb = min(BT, A.B - b0);
+    const int n_blocks = (A.V + kHeadRows - 1) / kHeadRows;
+    const int cps = gridDim.x / n_by;
+    const int c0 = blockIdx.x / n_by;
+    const int my_blocks = c0 < n_blocks ? (n_blocks - 1 - c0) / cps + 1 : 0;
+    const int n_items = my_blocks * nch;
+
+    if (tid == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], 4);
+        }
+        mbar_init(&bar_x, 1);
+        mbar_init(&bar_done, 1);
+        mbar_fence_init();
+        s_fail = 0;
+    }
+    if (tid < BT) s_key[tid] = 0ull;
+    if (warp == 1) {
+        tmem_alloc(&s_tmem, TCOLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = s_tmem;
+
+    // weights do not depend on earlier kernels: the first stages go out before the wait
+    auto issue = [&](int it) {
+        const int jb = c0 + (it / nch) * cps;
+        const int c = it % nch;
+        unsigned char* dst = ring + static_cast<size_t>(it % NS) * kHeadStageBytes;
+        mbar_arrive_expect_tx(&full[it % NS], kHeadStageBytes);
+#pragma unroll
+        for (int p = 0; p < 3; ++p)
+            tma_load_2d(dst + p * kHeadPlaneBox, &A.wmap, c * kHeadKC, p * A.V + jb * kHeadRows, &full[it % NS]);
+    };
+    int n_issued = 0;
+    if (warp == 0 && lane == 0)
+        for (; n_issued < NS && n_issued < n_items; ++n_issued) issue(n_issued);
+    pdl_launch_dependents();
+    pdl_wait();
+
+    if (warp == 0 && lane == 0) {
+        // hidden digit planes of this batch tile (written by k_rowprep_digits)
+        mbar_arrive_expect_tx(&bar_x, 3 * xplane);
+        for (int p = 0; p < 3; ++p)
+            for (int c = 0; c < nch; ++c)
+                tma_load_2d(sx + p * xplane + c * BT * 128, BT == 16 ? &A.xmap16 : &A.xmap32, c * kHeadKC,
+                            p * A.MB + b0, &bar_x);
+        // remaining weight stages
+        for (int it = n_issued; it < n_items; ++it) {
+            if (!mbar_wait_bounded(&empty[it % NS], static_cast<uint32_t>(it / NS - 1) & 1u, A.err)) {
+                s_fail = 1;
+                break;
+            }
+            issue(it);
+            n_issued = it + 1;
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---- MMA issuer ----
+        bool ok = mbar_wait_bounded(&bar_x, 0, A.err);
+        tc_fence_after();
+        int it = 0;
+        for (int i = 0; ok && i < my_blocks; ++i) {
+            const int ab = i & 1;
+            if (i >= 2 && !mbar_wait_bounded(&tempty[ab], static_cast<uint32_t>((i >> 1) - 1) & 1u, A.err)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t dacc = tbase + static_cast<uint32_t>(ab * (TCOLS / 2));
+            for (int c = 0; c < nch; ++c, ++it) {
+                const int stage = it % NS;
+                if (!mbar_wait_bounded(&full[stage], static_cast<uint32_t>(it / NS) & 1u, A.err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const unsigned char* st = ring + static_cast<size_t>(stage) * kHeadStageBytes;
+#pragma unroll
+                for (int s = 0; s < kHeadKC / 32; ++s) {
+                    // six digit products, grouped by weight into three accumulators
+                    const uint64_t w1 = smem_desc_sw128(st) + 2 * s, w2 = smem_desc_sw128(st + kHeadPlaneBox) + 2 * s,
+                                   w3 = smem_desc_sw128(st + 2 * kHeadPlaneBox) + 2 * s;
+                    const unsigned char* xc = sx + c * BT * 128;
+                    const uint64_t x1 = smem_desc_sw128(xc) + 2 * s, x2 = smem_desc_sw128(xc + xplane) + 2 * s,
+                                   x3 = smem_desc_sw128(xc + 2 * xplane) + 2 * s;
+                    const uint32_t first = (c == 0 && s == 0) ? 0u : 1u;
+                    umma_i8(dacc, w1, x1, IDESC, first);
+                    umma_i8(dacc + BT, w1, x2, IDESC, first);
+                    umma_i8(dacc + BT, w2, x1, IDESC, 1u);
+                    umma_i8(dacc + 2 * BT, w1, x3, IDESC, first);
+                    umma_i8(dacc + 2 * BT, w2, x2, IDESC, 1u);
+                    umma_i8(dacc + 2 * BT, w3, x1, IDESC, 1u);
+                }
+                umma_commit(&empty[stage]);   // stage free once these MMAs have read it
+            }
+            if (!ok) break;
+            umma_commit(&tfull[ab]);          // accumulator set ready for the epilogue
+        }
+        if (!ok) s_fail = 1;
+        // every MMA issued has completed before TMEM is released
+        umma_commit(&bar_done);
+        mbar_wait_bounded(&bar_done, 0, nullptr);
+    } else if (warp >= 2) {
+        // ---- epilogue: TMEM lane quarter q holds embedding rows 32 q .. 32 q + 31 ----
+        const int q = warp & 3;
+        unsigned long long best[BT];
+#pragma unroll
+        for (int b = 0; b < BT; ++b) best[b] = 0ull;
+        for (int i = 0; i < my_blocks; ++i) {
+            const int ab = i & 1;
+            if (!mbar_wait_bounded(&tfull[ab], static_cast<uint32_t>(i >> 1) & 1u, A.err)) {
+                s_fail = 1;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t t0 = tbase + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * (TCOLS / 2));
+            int a0[BT], a1[BT], a2[BT];
+            HeadTmemLd<BT>::run(t0, a0);
+            HeadTmemLd<BT>::run(t0 + BT, a1);
+            HeadTmemLd<BT>::run(t0 + 2 * BT, a2);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[ab]);
+            const int jb = c0 + i * cps;
+            const int n = jb * kHeadRows + q * 32 + lane;
+            if (n < A.V) {
+                const float sn = __ldg(A.wscale + n);
+#pragma unroll
+                for (int b = 0; b < BT; ++b) {
+                    if (b >= nb) break;
+                    const float u = static_cast<float>(a1[b]) + static_cast<float>(a2[b]) * (1.0f / 254.0f);
+                    const float w = static_cast<float>(a0[b]) + u * (1.0f / 254.0f);
+                    const float y = __fmul_rn(sn * A.xscale[b0 + b], w);
+                    if (A.logits) A.logits[static_cast<long long>(b0 + b) * A.V + n] = y;
+                    const unsigned long long key = argmax_key(y, n);
+                    best[b] = key > best[b] ? key : best[b];
+                }
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < BT; ++b) {
+            unsigned long long v = best[b];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, off);
+                v = o > v ? o : v;
+            }
+            if (lane == 0 && b < nb && v != 0ull) atomicMax(&s_key[b], v);
+        }
+    }
+    // in-flight weight copies land before the CTA can exit
+    if (warp == 0 && lane == 0 && s_fail)
+        for (int i2 = max(0, n_issued - NS); i2 < n_issued; ++i2)
+            mbar_wait_bounded(&full[i2 % NS], static_cast<uint32_t>(i2 / NS) & 1u, nullptr);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, TCOLS);
+    }
+    // fold into the grid-wide keys; the last CTA writes the picks and resets the keys
+    if (tid < nb && s_key[tid] != 0ull) atomicMax(&A.keys[b0 + tid], s_key[tid]);
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        s_last = (atomicAdd(A.counter, 1) == static_cast<int>(gridDim.x) - 1);
+    }
+    __syncthreads();
+    if (s_last) {
+        __threadfence();
+        for (int b = tid; b < A.B; b += kHeadThreads) {
+            const unsigned long long k = atomicExch(&A.keys[b], 0ull);
+            const int idx = (k == 0ull) ? 0 : argmax_key_index(k);
+            if (A.argmax_out) A.argmax_out[b] = idx;
+            if (A.last_tok) A.last_tok[A.meta->slot[b]] = idx;
+        }
+        if (tid == 0) *A.counter = 0;
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+inline size_t head_tc_smem(int K, int bt, int ns) {
+    const int nch = (K + kHeadKC - 1) / kHeadKC;
+    return 1024 + size_t(ns) * kHeadStageBytes + size_t(3) * nch * bt * 128;
+}
+inline int head_tc_bt(int B) { return B <= 16 ? 16 : 32; }
+// stages that fit next to the hidden planes (0: the head does not fit)
+inline int head_tc_stages(int K, int bt) {
+    if (K % 16 != 0 || K > kHeadMaxK) return 0;
+    for (int ns = kHeadMaxStages; ns >= 2; --ns)
+        if (head_tc_smem(K, bt, ns) <= size_t(227 * 1024 - 1024)) return ns;   // room for static smem
+    return 0;
+}
+
+template <int PRO>
+cudaError_t rowprep_digits_launch(const float* x, int x_ld, const float* gw, const float* gb, float eps, int K,
+                                  int rows, long long plane_stride, int8_t* out, float* scale, bool pdl,
+                                  cudaStream_t st);
+cudaError_t head_tc_launch(int num_sms, const HeadArgs& a, cudaStream_t st);
+
+#ifdef DEC_HEAD_TC_DEFINE
+
+template <int PRO>
+cudaError_t rowprep_digits_launch(const float* x, int x_ld, const float* gw, const float* gb, float eps, int K,
+                                  int rows, long long plane_stride, int8_t* out, float* scale, bool pdl,
+                                  cudaStream_t st) {
+    if (K % 4 != 0 || rows <= 0) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((rows + 3) / 4);
+    cfg.blockDim = dim3(128);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_rowprep_digits<PRO>, x, x_ld, gw, gb, eps, K, rows, plane_stride, out, scale);
+}
+
+template <int BT>
+cudaError_t head_tc_launch_bt(int num_sms, HeadArgs a, cudaStream_t st) {
+    const int ns = head_tc_stages(a.K, BT);
+    if (ns == 0) return cudaErrorNotSupported;
+    const size_t smem = head_tc_smem(a.K, BT, ns);
+    static int attr_dev = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (attr_dev != dev) {
+        e = cudaFuncSetAttribute(k_head_tc<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024 - 1024);
+        if (e != cudaSuccess) return e;
+        attr_dev = dev;
+    }
+    const int gy = (a.B + BT - 1) / BT;
+    a.n_by = gy;
+    const int n_blocks = (a.V + kHeadRows - 1) / kHeadRows;
+    const int cps = std::max(1, std::min(n_blocks, num_sms / gy));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cps * gy);
+    cfg.blockDim = dim3(kHeadThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_head_tc<BT>, a, ns);
+}
+
+cudaError_t head_tc_launch(int num_sms, const HeadArgs& a, cudaStream_t st) {
+    if (a.B < 1 || a.B > a.MB) return cudaErrorInvalidValue;
+    if (head_tc_bt(a.B) == 16) return head_tc_launch_bt<16>(num_sms, a, st);
+    return head_tc_launch_bt<32>(num_sms, a, st);
+}
+
+#endif  // DEC_HEAD_TC_DEFINE
+
+}  // namespace dec
