@@ -211,7 +211,6 @@ def run_ours(args, wl: synth.Workload, rank: int, world: int) -> dict:
     gw = GpuWorkload(wl, seed, fast_setup=args.fast_setup)
     stream = torch.cuda.Stream()
     sh = stream.cuda_stream
-    kernels_per_step = 2 + cfg.n_layers * (8 if cfg.is_whisper else 5)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             gw.step(sh)
@@ -226,13 +225,19 @@ def run_ours(args, wl: synth.Workload, rank: int, world: int) -> dict:
         e1 = torch.cuda.Event(enable_timing=True)
         tokens = 0
         lens_seen = []
+        launches = 0
+        if args.profile_range:
+            torch.cuda.profiler.start()
         e0.record(stream)
         for _ in range(args.steps):
             b, pos = gw.step(sh)
             tokens += b
             lens_seen.append(pos)
+            launches += gw.dec.step_kernels()
         e1.record(stream)
         torch.cuda.synchronize()
+        if args.profile_range:
+            torch.cuda.profiler.stop()
         clocks = clk.stop()
         ms = e0.elapsed_time(e1)
         gw.dec.sync(sh)
@@ -280,7 +285,7 @@ def run_ours(args, wl: synth.Workload, rank: int, world: int) -> dict:
     roof = dominant_kernel_roofline(wl, cfg, lens_at_start) if rank == 0 else None
     gw.dec.close()
     return dict(value=value, ms=ms_max, tokens=tokens_all, clocks=clocks, e2e=e2e, roofline=roof,
-                achieved_gbs=achieved_gbs, launches=kernels_per_step * args.steps,
+                achieved_gbs=achieved_gbs, launches=launches,
                 step_bytes=statistics.mean(per_step_bytes))
 
 
@@ -434,6 +439,8 @@ def main():
     ap.add_argument("--config", default="c2", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-range", action="store_true",
+                    help="bracket the timed steps with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
     ap.add_argument("--fast-setup", action="store_true",
                     help="seed caches with N(0,1) K/V instead of prefilling tokens (profiling runs)")
     args = ap.parse_args()

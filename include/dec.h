@@ -229,6 +229,11 @@ dec_status dec_hidden(dec_handle* h, float* out, int32_t batch, void* stream);
  * bounded wait inside a kernel gave up). Clears the device status word. */
 dec_status dec_sync(dec_handle* h, void* stream);
 
+/* Number of kernels one step of the most recent dec_step / dec_step_host call
+ * launches (the kernel nodes of its captured CUDA graph), or -1 when that step's
+ * launch sequence could not be captured. Host-only; never blocks. */
+dec_status dec_step_kernels(const dec_handle* h, int32_t* kernels);
+
 /*
  * Kernel-level entry points (no handle). They run one kernel of the step on
  * caller-provided device buffers, for testing each kernel on its own.

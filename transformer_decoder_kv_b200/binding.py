@@ -24,7 +24,7 @@ PROJ = {"f32": 0, "w8a8": 1, "w8a32": 2}
 
 # Every symbol include/dec.h declares.
 EXPORTS = ["dec_create", "dec_destroy", "dec_last_error", "dec_prefill", "dec_kv_append", "dec_step",
-           "dec_step_host", "dec_slot_len", "dec_kv_read", "dec_hidden", "dec_sync",
+           "dec_step_host", "dec_slot_len", "dec_kv_read", "dec_hidden", "dec_sync", "dec_step_kernels",
            "dec_attention_workspace_size", "dec_attention", "dec_attention_noalloc", "dec_i8_dot"]
 
 
@@ -80,6 +80,7 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
         "dec_kv_read": (C.c_int, [vp, i32, i32, i32, i32, vp, vp, vp]),
         "dec_hidden": (C.c_int, [vp, vp, i32, vp]),
         "dec_sync": (C.c_int, [vp, vp]),
+        "dec_step_kernels": (C.c_int, [vp, pi32]),
         "dec_attention_workspace_size": (C.c_size_t, [i32, i32, i32]),
         "dec_attention": (C.c_int, [vp, vp, vp, vp, i32, i32, i32, vp, vp, C.c_size_t, vp]),
         "dec_attention_noalloc": (C.c_int, [vp, vp, vp, vp, i32, i32, i32, vp, vp]),
@@ -216,6 +217,12 @@ class Decoder:
 
     def sync(self, stream: int = 0):
         self._check(self._lib.dec_sync(self._h, stream))
+
+    def step_kernels(self) -> int:
+        """Kernels launched by one step of the most recent step call (-1: not captured)."""
+        n = C.c_int32(0)
+        self._check(self._lib.dec_step_kernels(self._h, C.byref(n)))
+        return int(n.value)
 
 
 def attention(q, k, v, lens, batch: int, n_heads: int, ld: int, out, workspace, workspace_bytes: int,

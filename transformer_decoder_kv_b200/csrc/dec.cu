@@ -115,7 +115,12 @@ struct dec_handle {
     // CUDA graphs of the step's launch sequence, keyed by what changes its launches:
     // batch size, self-attention tile count, output pointers. A null entry means
     // capture failed for that key and the step runs eagerly.
-    std::map<std::array<long long, 4>, cudaGraphExec_t> graphs;
+    struct StepGraph {
+        cudaGraphExec_t exec;
+        int kernels;   // kernel launches in one step of this key (-1: not captured)
+    };
+    std::map<std::array<long long, 4>, StepGraph> graphs;
+    int last_step_kernels = -1;
     cudaStream_t cap_stream = nullptr;
     float* stage_logits = nullptr;   // dec_step_host result staging
     int* stage_argmax = nullptr;
@@ -716,10 +721,11 @@ void capture_step(dec_handle* h, const std::array<long long, 4>& key, int B, int
                   int* argmax) {
     if (h->graphs.size() >= 256) {
         for (auto& kv : h->graphs)
-            if (kv.second) cudaGraphExecDestroy(kv.second);
+            if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
         h->graphs.clear();
     }
     cudaGraphExec_t exec = nullptr;
+    int kernels = -1;
     if (cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal) == cudaSuccess) {
         const std::string saved = h->err;
         const dec_status s = run_step(h, B, max_len, logits, argmax, h->cap_stream);
@@ -727,12 +733,23 @@ void capture_step(dec_handle* h, const std::array<long long, 4>& key, int B, int
         const cudaError_t e = cudaStreamEndCapture(h->cap_stream, &g);
         if (s == DEC_OK && e == cudaSuccess && g != nullptr) {
             if (cudaGraphInstantiate(&exec, g, 0) != cudaSuccess) exec = nullptr;
+            size_t n = 0;
+            if (exec && cudaGraphGetNodes(g, nullptr, &n) == cudaSuccess) {
+                std::vector<cudaGraphNode_t> nodes(n);
+                if (n && cudaGraphGetNodes(g, nodes.data(), &n) == cudaSuccess) {
+                    kernels = 0;
+                    for (auto nd : nodes) {
+                        cudaGraphNodeType t;
+                        if (cudaGraphNodeGetType(nd, &t) == cudaSuccess && t == cudaGraphNodeTypeKernel) ++kernels;
+                    }
+                }
+            }
         }
         if (g) cudaGraphDestroy(g);
         h->err = saved;
     }
     cudaGetLastError();
-    h->graphs[key] = exec;
+    h->graphs[key] = {exec, kernels};
 }
 
 dec_status step_validated(dec_handle* h, const StepMeta& m, int max_len, float* logits, int* argmax,
@@ -741,12 +758,13 @@ dec_status step_validated(dec_handle* h, const StepMeta& m, int max_len, float* 
     const std::array<long long, 4> key = {m.B, (max_len + kAttnTile - 1) / kAttnTile,
                                           reinterpret_cast<long long>(logits), reinterpret_cast<long long>(argmax)};
     auto it = h->graphs.find(key);
-    if (it != h->graphs.end() && it->second != nullptr) {
-        DEC_CUDA(h, cudaGraphLaunch(it->second, st));
+    if (it != h->graphs.end() && it->second.exec != nullptr) {
+        DEC_CUDA(h, cudaGraphLaunch(it->second.exec, st));
     } else {
         DEC_TRY(run_step(h, m.B, max_len, logits, argmax, st));
         if (it == h->graphs.end()) capture_step(h, key, m.B, max_len, logits, argmax);
     }
+    h->last_step_kernels = h->graphs[key].kernels;
     for (int b = 0; b < m.B; ++b) {
         h->slot_len[m.slot[b]] += 1;
         h->has_tok[m.slot[b]] = 1;
@@ -767,7 +785,7 @@ dec_status dec_destroy(dec_handle* h) {
     if (!h) return DEC_OK;
     cudaDeviceSynchronize();
     for (auto& kv : h->graphs)
-        if (kv.second) cudaGraphExecDestroy(kv.second);
+        if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
     if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
     for (void* p : h->dallocs) cudaFree(p);
     for (void* p : h->hallocs) cudaFreeHost(p);
@@ -1122,6 +1140,12 @@ dec_status dec_hidden(dec_handle* h, float* out, int32_t batch, void* stream) {
     if (!out || batch < 1 || batch > h->last_batch) return fail(h, DEC_EINVAL, "bad output or batch");
     DEC_CUDA(h, cudaMemcpyAsync(out, h->x, size_t(batch) * h->cfg.d_model * 4, cudaMemcpyDeviceToDevice,
                                 static_cast<cudaStream_t>(stream)));
+    return DEC_OK;
+}
+
+dec_status dec_step_kernels(const dec_handle* h, int32_t* kernels) {
+    if (!h || !kernels) return DEC_EINVAL;
+    *kernels = h->last_step_kernels;
     return DEC_OK;
 }
 

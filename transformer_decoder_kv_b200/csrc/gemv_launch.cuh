@@ -78,32 +78,56 @@ cudaError_t gemv_launch_bt(int num_sms, const GemvArgs& a, cudaStream_t st) {
     const int n_tasks = (n_pairs + pairs_per_task - 1) / pairs_per_task;
     const int n_blocks = (n_tasks + gemv_consumer_warps(BT) - 1) / gemv_consumer_warps(BT);
     // occupancy for this instantiation, cached per shared-memory size
-    static size_t occ_smem[4] = {~size_t(0), ~size_t(0), ~size_t(0), ~size_t(0)};
-    static int occ_val[4] = {0, 0, 0, 0};
+    static size_t occ_smem[8] = {~size_t(0), ~size_t(0), ~size_t(0), ~size_t(0),
+                                 ~size_t(0), ~size_t(0), ~size_t(0), ~size_t(0)};
+    static int occ_val[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     static int occ_next = 0;
-    int occ = -1;
-    for (int i = 0; i < 4; ++i)
-        if (occ_smem[i] == p.smem) occ = occ_val[i];
-    if (occ < 0) {
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, gemv_threads(BT), p.smem);
-        if (e != cudaSuccess) return e;
-        occ_smem[occ_next] = p.smem;
-        occ_val[occ_next] = occ;
-        occ_next = (occ_next + 1) & 3;
-    }
+    auto occupancy = [&](size_t smem, int* occ) -> cudaError_t {
+        for (int i = 0; i < 8; ++i)
+            if (occ_smem[i] == smem) {
+                *occ = occ_val[i];
+                return cudaSuccess;
+            }
+        const cudaError_t r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, kern, gemv_threads(BT), smem);
+        if (r != cudaSuccess) return r;
+        occ_smem[occ_next] = smem;
+        occ_val[occ_next] = *occ;
+        occ_next = (occ_next + 1) & 7;
+        return cudaSuccess;
+    };
+    // The ring holds no more stages than a CTA streams, so a small matrix leaves shared
+    // memory free and the next kernel's CTAs can become resident early and prefetch
+    // their weights while this one runs (programmatic dependent launch).
     const int gy = (a.B + BT - 1) / BT;
-    const int gx = std::max(1, std::min(n_blocks, (num_sms * std::max(1, occ)) / gy));
+    const int elt_w = sizeof(WT);
+    const int rows_per_block = gemv_rows_per_task(BT) * gemv_consumer_warps(BT);
+    const size_t stage = size_t(rows_per_block) * p.KC * elt_w;
+    const size_t xbytes = p.smem - size_t(p.NS) * stage;
+    const int chunks = (a.K + p.KC - 1) / p.KC;
+    int occ = 0, gx = 1, ns = p.NS;
+    for (int pass = 0; pass < 2; ++pass) {
+        e = occupancy(xbytes + size_t(pass == 0 ? 2 : ns) * stage, &occ);
+        if (e != cudaSuccess) return e;
+        gx = std::max(1, std::min(n_blocks, (num_sms * std::max(1, occ)) / gy));
+        const int items = ((n_blocks + gx - 1) / gx) * chunks;
+        ns = std::min(p.NS, std::max(2, items));
+    }
+    const size_t smem = xbytes + size_t(ns) * stage;
+    // one wave at the final ring depth
+    e = occupancy(smem, &occ);
+    if (e != cudaSuccess) return e;
+    gx = std::max(1, std::min(gx, (num_sms * std::max(1, occ)) / gy));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(gx, gy);
     cfg.blockDim = dim3(gemv_threads(BT));
-    cfg.dynamicSmemBytes = p.smem;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a, p.KC, p.NS);
+    return cudaLaunchKernelEx(&cfg, kern, a, p.KC, ns);
 }
 
 template <typename WT, bool I8, int PRO, int EPI, int MAP>

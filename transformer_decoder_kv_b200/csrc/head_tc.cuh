@@ -255,6 +255,7 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
     __shared__ __align__(8) uint64_t tfull[2], tempty[2], bar_x, bar_done;
     __shared__ uint32_t s_tmem;
     __shared__ unsigned long long s_key[BT];
+    __shared__ float s_xs[BT];
     __shared__ int s_fail, s_last;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -307,6 +308,8 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
     pdl_launch_dependents();
     pdl_wait();
 
+    if (tid < BT) s_xs[tid] = tid < nb ? A.xscale[b0 + tid] : 0.0f;
+    __syncthreads();
     if (warp == 0 && lane == 0) {
         // hidden digit planes of this batch tile (written by k_rowprep_digits)
         mbar_arrive_expect_tx(&bar_x, 3 * xplane);
@@ -400,7 +403,7 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
                     if (b >= nb) break;
                     const float u = static_cast<float>(a1[b]) + static_cast<float>(a2[b]) * (1.0f / 254.0f);
                     const float w = static_cast<float>(a0[b]) + u * (1.0f / 254.0f);
-                    const float y = __fmul_rn(sn * A.xscale[b0 + b], w);
+                    const float y = __fmul_rn(sn * s_xs[b], w);
                     if (A.logits) A.logits[static_cast<long long>(b0 + b) * A.V + n] = y;
                     const unsigned long long key = argmax_key(y, n);
                     best[b] = key > best[b] ? key : best[b];

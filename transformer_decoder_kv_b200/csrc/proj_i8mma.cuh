@@ -508,9 +508,8 @@ cudaError_t proj_i8mma_launch_bt(int num_sms, I8MmaArgs A, int n_blocks, cudaStr
     auto kern = k_proj_i8mma<BT, EPI, MAP>;
     const size_t xbytes = size_t(BT) * (A.ksl + kI8XPad);
     const size_t avail = size_t(227 * 1024) - 1024 - 1024 - xbytes;
-    const int NS = int(std::min<size_t>(kMmaMaxStages, avail / kMmaStageBytes));
-    if (NS < 2) return cudaErrorNotSupported;
-    const size_t smem = 1024 + size_t(NS) * kMmaStageBytes + xbytes;
+    const int ns_max = int(std::min<size_t>(kMmaMaxStages, avail / kMmaStageBytes));
+    if (ns_max < 2) return cudaErrorNotSupported;
     static int attr_dev = -1;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -522,13 +521,25 @@ cudaError_t proj_i8mma_launch_bt(int num_sms, I8MmaArgs A, int n_blocks, cudaStr
         if (e != cudaSuccess) return e;
         attr_dev = dev;
     }
-    int occ = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kMmaThreads, smem);
-    if (e != cudaSuccess) return e;
+    // the ring holds no more stages than a CTA streams (room for the next kernel's CTAs)
     const int gy = (A.g.B + BT - 1) / BT;
     A.n_by = gy;
-    const int slots = std::max(1, num_sms * std::max(1, occ) / gy);
-    const int cps = std::max(1, std::min(n_blocks, slots / A.n_ks));
+    const int stage_k = kI8KC;
+    const int nkc = (A.ksl + stage_k - 1) / stage_k;
+    int occ = 0, cps = 1, NS = ns_max;
+    for (int pass = 0; pass < 2; ++pass) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kMmaThreads,
+                                                          1024 + size_t(pass == 0 ? 2 : NS) * kMmaStageBytes + xbytes);
+        if (e != cudaSuccess) return e;
+        const int slots = std::max(1, num_sms * std::max(1, occ) / gy);
+        cps = std::max(1, std::min(n_blocks, slots / A.n_ks));
+        NS = std::min(ns_max, std::max(2, ((n_blocks + cps - 1) / cps) * nkc));
+    }
+    const size_t smem = 1024 + size_t(NS) * kMmaStageBytes + xbytes;
+    // one wave at the final ring depth
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kMmaThreads, smem);
+    if (e != cudaSuccess) return e;
+    cps = std::max(1, std::min(cps, std::max(1, num_sms * std::max(1, occ) / gy) / A.n_ks));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cps * A.n_ks * gy);
     cfg.blockDim = dim3(kMmaThreads);
