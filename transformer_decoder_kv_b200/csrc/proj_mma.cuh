@@ -42,9 +42,10 @@ constexpr int kMmaConsumerWarps = 4;
 constexpr int kMmaThreads = (kMmaConsumerWarps + 1) * 32;
 constexpr int kMmaBlockRows = 32 * kMmaConsumerWarps;           // 128
 constexpr int kMmaBoxBytes = kMmaBlockRows * 128;               // 16 KB: 128 rows x 128 bytes
-constexpr int kMmaBoxesPerStage = 2;
+constexpr int kMmaBoxesPerStage = 2;                              // int8 tensor-core kernel
 constexpr int kMmaStageBytes = kMmaBoxBytes * kMmaBoxesPerStage;  // 32 KB
 constexpr int kMmaMaxStages = 6;
+constexpr int kMmaMaxStagesTF = 12;   // TF32 kernel: stages of one or two boxes
 
 struct MmaArgs {
     CUtensorMap tmap;        // weights [N, K]: box {128 bytes of K, 128 rows}, 128-byte swizzle
@@ -172,13 +173,15 @@ __global__ void __launch_bounds__(kRowprepThreads) k_rowprep(const float* __rest
     }
 }
 
-template <int BT, typename WT, int EPI>
+// NBX: 128-byte boxes per stage (1 for int8 weights, 2 for f32)
+template <int BT, typename WT, int EPI, int NBX>
 __global__ void __launch_bounds__(kMmaThreads, 1) k_proj_mma(const __grid_constant__ MmaArgs A, int NS) {
     const GemvArgs& a = A.g;
     constexpr int NT = BT / 8;
     constexpr int ELT = sizeof(WT);
     constexpr int BOXK = 128 / ELT;                       // K elements per box row
-    constexpr int KC = BOXK * kMmaBoxesPerStage;          // K elements per stage
+    constexpr int KC = BOXK * NBX;                        // K elements per stage
+    constexpr int SB = kMmaBoxBytes * NBX;                // stage bytes
     constexpr bool F32W = std::is_same<WT, float>::value;
     static_assert(BT % 8 == 0, "batch tile must be a multiple of 8");
 
@@ -187,9 +190,9 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_proj_mma(const __grid_consta
         (reinterpret_cast<uintptr_t>(mma_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     unsigned char* ring = smem;
     const int XS = A.ksl + mma_xpad<WT>();   // padded activation row (floats)
-    float* sX = reinterpret_cast<float*>(smem + static_cast<size_t>(NS) * kMmaStageBytes);
-    __shared__ __align__(8) uint64_t full[kMmaMaxStages];
-    __shared__ __align__(8) uint64_t empty[kMmaMaxStages];
+    float* sX = reinterpret_cast<float*>(smem + static_cast<size_t>(NS) * SB);
+    __shared__ __align__(8) uint64_t full[kMmaMaxStagesTF];
+    __shared__ __align__(8) uint64_t empty[kMmaMaxStagesTF];
     __shared__ __align__(8) uint64_t bar_x;
     __shared__ unsigned long long s_key[BT];
     __shared__ int s_flag, s_last;   // staging succeeded; this CTA arrived last (head)
@@ -215,10 +218,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_proj_mma(const __grid_consta
         const int jb = c0 + (it / nkc) * cps;
         const int c = it % nkc;
         const int stage = it % NS;
-        unsigned char* dst = ring + static_cast<size_t>(stage) * kMmaStageBytes;
-        mbar_arrive_expect_tx(&full[stage], kMmaStageBytes);
+        unsigned char* dst = ring + static_cast<size_t>(stage) * SB;
+        mbar_arrive_expect_tx(&full[stage], SB);
 #pragma unroll
-        for (int bx = 0; bx < kMmaBoxesPerStage; ++bx)
+        for (int bx = 0; bx < NBX; ++bx)
             tma_load_2d(dst + bx * kMmaBoxBytes, &A.tmap, kstart + c * KC + bx * BOXK, jb * kMmaBlockRows,
                         &full[stage]);
     };
@@ -327,7 +330,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_proj_mma(const __grid_consta
 #pragma unroll
                         for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.0f;
             }
-            const unsigned char* st = ring + static_cast<size_t>(stage) * kMmaStageBytes;
+            const unsigned char* st = ring + static_cast<size_t>(stage) * SB;
             // 32-column groups of this stage (slices and K are multiples of 32); the group
             // body is unrolled, the group loop is not, so the code stays in the
             // instruction cache
@@ -557,12 +560,16 @@ struct MmaPlan {
     int n_blocks;   // 128-row blocks
     int n_ks;       // K slices
     int ksl;        // K elements per slice
+    int nbx;        // 128-byte boxes per pipeline stage (TF32 kernel)
     bool ok;
 };
 
 inline MmaPlan mma_plan(int N, int K, int elt, int num_sms) {
     MmaPlan p{};
-    const int KC = kMmaBoxesPerStage * 128 / elt;
+    // int8 weights stream 128 columns (16 KB) per stage: finer K slices, so that the
+    // 2xTF32 work of a slice spreads over every SM
+    p.nbx = elt == 1 ? 1 : 2;
+    const int KC = p.nbx * 128 / elt;
     const int pad = elt == 4 ? 4 : 16;
     p.n_blocks = (N + kMmaBlockRows - 1) / kMmaBlockRows;
     if (K % 32 != 0 || N <= 0) return p;
@@ -596,12 +603,13 @@ cudaError_t rowprep_launch(const GemvArgs& g, float* out, cudaStream_t st);
 
 #ifdef DEC_MMA_DEFINE
 
-template <int BT, typename WT, int EPI>
+template <int BT, typename WT, int EPI, int NBX>
 cudaError_t proj_mma_launch_bt(int num_sms, MmaArgs A, int n_blocks, cudaStream_t st) {
-    auto kern = k_proj_mma<BT, WT, EPI>;
+    auto kern = k_proj_mma<BT, WT, EPI, NBX>;
+    constexpr int SB = kMmaBoxBytes * NBX;
     const size_t xbytes = size_t(BT) * (A.ksl + mma_xpad<WT>()) * 4;
     const size_t avail = size_t(227 * 1024) - 1024 - 1024 - xbytes;
-    const int ns_max = int(std::min<size_t>(kMmaMaxStages, avail / kMmaStageBytes));
+    const int ns_max = int(std::min<size_t>(kMmaMaxStagesTF, avail / SB));
     if (ns_max < 2) return cudaErrorNotSupported;
     static int attr_dev = -1;
     int dev = 0;
@@ -617,18 +625,18 @@ cudaError_t proj_mma_launch_bt(int num_sms, MmaArgs A, int n_blocks, cudaStream_
     // the ring holds no more stages than a CTA streams (room for the next kernel's CTAs)
     const int gy = (A.g.B + BT - 1) / BT;
     A.n_by = gy;
-    const int stage_k = kMmaBoxesPerStage * 128 / int(sizeof(WT));
+    const int stage_k = NBX * 128 / int(sizeof(WT));
     const int nkc = (A.ksl + stage_k - 1) / stage_k;
     int occ = 0, cps = 1, NS = ns_max;
     for (int pass = 0; pass < 2; ++pass) {
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kMmaThreads,
-                                                          1024 + size_t(pass == 0 ? 2 : NS) * kMmaStageBytes + xbytes);
+                                                          1024 + size_t(pass == 0 ? 2 : NS) * SB + xbytes);
         if (e != cudaSuccess) return e;
         const int slots = std::max(1, num_sms * std::max(1, occ) / gy);
         cps = std::max(1, std::min(n_blocks, slots / A.n_ks));
         NS = std::min(ns_max, std::max(2, ((n_blocks + cps - 1) / cps) * nkc));
     }
-    const size_t smem = 1024 + size_t(NS) * kMmaStageBytes + xbytes;
+    const size_t smem = 1024 + size_t(NS) * SB + xbytes;
     // one wave at the final ring depth
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kMmaThreads, smem);
     if (e != cudaSuccess) return e;
@@ -664,10 +672,17 @@ cudaError_t proj_mma_launch(int num_sms, const CUtensorMap& map, void* part, siz
     A.ksl = p.ksl;
     A.n_by = 1;
     A.g = g;
+    if (p.nbx == 1) {
+        switch (bt) {
+            case 8: return proj_mma_launch_bt<8, WT, EPI, 1>(num_sms, A, p.n_blocks, st);
+            case 16: return proj_mma_launch_bt<16, WT, EPI, 1>(num_sms, A, p.n_blocks, st);
+            default: return proj_mma_launch_bt<32, WT, EPI, 1>(num_sms, A, p.n_blocks, st);
+        }
+    }
     switch (bt) {
-        case 8: return proj_mma_launch_bt<8, WT, EPI>(num_sms, A, p.n_blocks, st);
-        case 16: return proj_mma_launch_bt<16, WT, EPI>(num_sms, A, p.n_blocks, st);
-        default: return proj_mma_launch_bt<32, WT, EPI>(num_sms, A, p.n_blocks, st);
+        case 8: return proj_mma_launch_bt<8, WT, EPI, 2>(num_sms, A, p.n_blocks, st);
+        case 16: return proj_mma_launch_bt<16, WT, EPI, 2>(num_sms, A, p.n_blocks, st);
+        default: return proj_mma_launch_bt<32, WT, EPI, 2>(num_sms, A, p.n_blocks, st);
     }
 }
 
