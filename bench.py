@@ -20,6 +20,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -88,7 +89,8 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        # samples go to a scratch file; the summary is part of the JSON line
+        self.path = os.path.join(tempfile.gettempdir(), f"dec_bench_clocks_{os.getpid()}.csv")
 
     def start(self):
         try:

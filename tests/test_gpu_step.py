@@ -175,3 +175,19 @@ def test_w8a8_tensor_core_path_equals_dp4a_path_bitwise():
         assert np.array_equal(h9[s].view(np.uint32), h1[0].view(np.uint32)), s
         p1.gpu.close()
     p9.gpu.close()
+
+
+def test_step_kernel_count_is_reported():
+    """dec_step_kernels gives the kernel count of the step's captured graph: positive, the
+    same for repeated steps of one shape, and the layer count sets it for a fixed path."""
+    wl = synth.workload("tiny_whisper_b3")
+    p = build_pair(wl)
+    counts = []
+    for t in range(3):
+        step_both(p, [5, 6, 7])
+        counts.append(p.gpu.step_kernels())
+    p.gpu.close()
+    assert counts[0] > 0 and len(set(counts)) == 1, counts
+    # embed, then per layer: q|k|v, self-attention, o, cross q, cross-attention, cross o,
+    # fc1, fc2; then the head's row split and the head
+    assert counts[0] == 1 + wl.model.n_layers * 8 + 2, counts
