@@ -461,8 +461,10 @@ def main():
         if rank != 0:
             return
         cb = oracle_sample(wl, 0, budget_s=max(5.0, min(60.0, 8.0 * max(1, args.steps) / 8)))
+        # one step = one token for each of the workload's streams, at the oracle's rate
         line = {"impl": "reference", "metric": metric, "value": cb["value"], "unit": "tokens/s",
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(1e3 * wl.batch / cb["value"], 3),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": config, "cpu_baseline": cb,
                 "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
