@@ -243,9 +243,7 @@ def run_ours(args, wl: synth.Workload, rank: int, world: int) -> dict:
         clocks = clk.stop()
         ms = e0.elapsed_time(e1)
         gw.dec.sync(sh)
-    ms_max = _max_over_ranks(ms, world)
-    tokens_all = _sum_over_ranks(tokens, world)
-    value = tokens_all / (ms_max / 1e3)
+    value, ms_max, tokens_all = combine_ranks(ms, tokens, world)
 
     # bytes actually moved per step at the lengths seen
     per_step_bytes = [step_bytes(cfg, p)["total"] for p in lens_seen]
@@ -278,8 +276,7 @@ def run_ours(args, wl: synth.Workload, rank: int, world: int) -> dict:
         ee1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = ee0.elapsed_time(ee1)
-    e2e_ms_max = _max_over_ranks(e2e_ms, world)
-    e2e_value = _sum_over_ranks(e2e_tokens, world) / (e2e_ms_max / 1e3)
+    e2e_value = combine_ranks(e2e_ms, e2e_tokens, world)[0]
     meta_bytes = 4 * 4 * wl.batch  # slots, tokens, positions, lengths
     e2e = {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": meta_bytes,
            "d2h_bytes_per_step": wl.batch * (cfg.vocab * 4 + 4)}
@@ -422,6 +419,14 @@ def _max_over_ranks(v: float, world: int) -> float:
     t = torch.tensor([v], dtype=torch.float64)
     _PG.all_reduce(t, op=_PG.ReduceOp.MAX)
     return float(t.item())
+
+
+def combine_ranks(ms: float, tokens: int, world: int):
+    """Whole-job throughput: every rank's tokens over the slowest rank's device time.
+    Returns (tokens/s, max ms, total tokens); every rank takes the same collective steps."""
+    ms_max = _max_over_ranks(ms, world)
+    tokens_all = _sum_over_ranks(tokens, world)
+    return tokens_all / (ms_max / 1e3), ms_max, tokens_all
 
 
 def _sum_over_ranks(v: float, world: int) -> float:
