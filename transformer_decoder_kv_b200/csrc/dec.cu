@@ -455,9 +455,9 @@ dec_status attention(dec_handle* h, AttnArgs a, int B, int max_keys, int tps, cu
     const int max_tiles = (max_keys + kAttnTile - 1) / kAttnTile;
     a.tps = tps;
     a.S = std::max(1, (max_tiles + tps - 1) / tps);
-    // one stage per CTA (more resident CTAs) up to 4 tiles per split, two beyond:
-    // measured on B200 as the fastest for both ragged self-attention and cross-attention
-    a.stages = tps >= 8 ? 2 : 1;
+    // one stage per CTA (more resident CTAs) at 1 and 4 tiles per split, two at 2 and 8+:
+    // measured on B200 (HBM-resident caches) as the fastest for each split size
+    a.stages = (tps == 2 || tps >= 8) ? 2 : 1;
     const size_t smem = size_t(a.stages) * 2 * kAttnTile * kHeadDim * sizeof(float);
     DEC_CUDA(h, launch(k_attention, dim3(a.S, a.H, B), dim3(kAttnThreads), smem, st, a));
     return DEC_OK;
@@ -467,8 +467,10 @@ dec_status attention(dec_handle* h, AttnArgs a, int B, int max_keys, int tps, cu
 // never more than kMaxSplits splits over the longest possible row.
 int tiles_per_split(const dec_handle* h, int max_keys) {
     const int rows_cap = h->cfg.n_heads * h->max_batch;
-    int t = rows_cap <= 32 ? 1 : (rows_cap <= 1023 ? 4 : 8);
     const int tiles_cap = (max_keys + kAttnTile - 1) / kAttnTile;
+    // measured on B200 with HBM-resident caches: few rows and short caches favour two
+    // tiles per split (double-buffered), more rows or longer caches four or eight
+    int t = rows_cap <= 32 ? 1 : (rows_cap <= 256 && tiles_cap <= 8) ? 2 : (rows_cap <= 1023 ? 4 : 8);
     return std::max(t, (tiles_cap + kMaxSplits - 1) / kMaxSplits);
 }
 
