@@ -23,7 +23,8 @@
 #include "gemv_launch.cuh"
 #include "misc.cuh"
 #include "head_tc.cuh"
-#include "proj_i8mma.cuh"
+#include "rowprep_i8.cuh"
+#include "proj_tc.cuh"
 #include "proj_mma.cuh"
 
 using namespace dec;
@@ -95,6 +96,8 @@ struct dec_handle {
     int* counters = nullptr;
     float* xn = nullptr;            // normalised activation rows (tensor-core path)
     int8_t* xq8 = nullptr;          // quantised activation rows and their scales (int8 tensor-core path)
+    int xq8_rows = 0;               // rows of xq8 (>= max batch, >= 32)
+    CUtensorMap m_xq8[2][2];        // xq8 as [rows, K] for K = d, F and boxes of 16, 32 rows
     float* xs8 = nullptr;
     void* mma_part = nullptr;       // split-K partial tiles (tensor-core path)
     size_t mma_part_bytes = 0;
@@ -317,21 +320,22 @@ dec_status proj_mma(dec_handle* h, const GemvArgs& a, const CUtensorMap& map, cu
     return DEC_OK;
 }
 
-bool i8mma_eligible(const dec_handle* h, int n_rows, int K, int B) {
+bool tc_eligible(const dec_handle* h, int n_rows, int K, int B) {
     if (!h->tma_ok || B < kMmaMinBatch) return false;
-    const MmaPlan p = i8mma_plan(n_rows, K, h->num_sms);
+    const MmaPlan p = tc_plan(n_rows, K, h->num_sms);
     if (!p.ok) return false;
-    return p.n_ks == 1 || (i8mma_part_bytes(p, B) <= h->mma_part_bytes && i8mma_counters(p, B) <= h->mma_cnt_len);
+    return p.n_ks == 1 || (tc_part_bytes(p, B) <= h->mma_part_bytes && tc_counters(p, B) <= h->mma_cnt_len);
 }
 
-// W8A8 on int8 tensor cores: rows quantised by k_rowprep_i8, exact int32 products.
+// W8A8 on tcgen05 int8 tensor cores: rows quantised by k_rowprep_i8, exact int32 products.
 template <int PRO, int EPI, int MAP>
-dec_status proj_w8a8_mma(dec_handle* h, const GemvArgs& a, const CUtensorMap& map, int n_rows, cudaStream_t st) {
+dec_status proj_w8a8_tc(dec_handle* h, const GemvArgs& a, const CUtensorMap& map, int n_rows, cudaStream_t st) {
     cudaError_t e = rowprep_i8_launch<PRO>(a, h->xq8, h->xs8, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "row quantisation launch");
-    e = proj_i8mma_launch<EPI, MAP>(h->num_sms, map, n_rows, h->xq8, h->xs8, h->mma_part, h->mma_part_bytes,
-                                       h->mma_cnt, h->mma_cnt_len, a, st);
-    if (e != cudaSuccess) return cuda_fail(h, e, "int8 tensor-core projection launch");
+    const int kx = a.K == h->cfg.d_model ? 0 : 1;
+    e = proj_tc_launch<EPI, MAP>(h->num_sms, map, h->m_xq8[kx][0], h->m_xq8[kx][1], n_rows, h->xs8, h->mma_part,
+                                 h->mma_part_bytes, h->mma_cnt, h->mma_cnt_len, a, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "tcgen05 projection launch");
     return DEC_OK;
 }
 
@@ -349,12 +353,13 @@ dec_status gemv_whisper(dec_handle* h, const GemvArgs& a, cudaStream_t st, const
     return gemv<int8_t, false, PRO, EPI, MAP>(h, a, st);
 }
 
-// Qwen W8A8 projections: int8 tensor cores from batch 8 on, dp4a below (bit-identical).
+// Qwen W8A8 projections: tcgen05 int8 tensor cores from batch 8 on for matrices of 2^21
+// weights or more, dp4a otherwise (bit-identical).
 template <int PRO, int EPI, int MAP>
 dec_status gemv_qwen(dec_handle* h, const GemvArgs& a, const CUtensorMap& map, cudaStream_t st) {
     const int n_rows = MAP == MAP_DUAL ? 2 * a.N : a.N;
-    if (static_cast<long long>(n_rows) * a.K >= kMmaMinWeights && i8mma_eligible(h, n_rows, a.K, a.B))
-        return proj_w8a8_mma<PRO, EPI, MAP>(h, a, map, n_rows, st);
+    if (static_cast<long long>(n_rows) * a.K >= kMmaMinWeights && tc_eligible(h, n_rows, a.K, a.B))
+        return proj_w8a8_tc<PRO, EPI, MAP>(h, a, map, n_rows, st);
     return gemv<int8_t, true, PRO, EPI, MAP>(h, a, st);
 }
 
@@ -861,9 +866,9 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
             } else {
                 DEC_TRY(dalloc(h, &D.wqkv_p, size_t(3) * d * d));
                 DEC_TRY(dalloc(h, &D.wgu, size_t(2) * F * d));
-                DEC_CUDA(h, i8_rows_permute(MAP_ROPE, static_cast<int8_t*>(D.wqkv_p),
+                DEC_CUDA(h, tc_rows_permute(MAP_ROPE, static_cast<int8_t*>(D.wqkv_p),
                                             static_cast<const int8_t*>(D.wqkv), nullptr, 3 * d, d, 0));
-                DEC_CUDA(h, i8_rows_permute(MAP_DUAL, static_cast<int8_t*>(D.wgu), static_cast<const int8_t*>(D.wg),
+                DEC_CUDA(h, tc_rows_permute(MAP_DUAL, static_cast<int8_t*>(D.wgu), static_cast<const int8_t*>(D.wg),
                                             static_cast<const int8_t*>(D.wu), 2 * F, d, 0));
                 ts = make_wmap(h, &D.m_qkv, D.wqkv_p, 3 * d, d, false);
                 if (ts == DEC_OK) ts = make_wmap(h, &D.m_o, D.wo, d, d, false);
@@ -926,7 +931,15 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
     // largest plan
     if (h->tma_ok) {
         DEC_TRY(dalloc(h, &h->xn, size_t(MB) * std::max(d, F) * 4));
-        DEC_TRY(dalloc(h, &h->xq8, size_t(MB) * std::max(d, F)));
+        h->xq8_rows = std::max(MB, 32);
+        DEC_TRY(dalloc(h, &h->xq8, size_t(h->xq8_rows) * std::max(d, F)));
+        DEC_CUDA(h, cudaMemset(h->xq8, 0, size_t(h->xq8_rows) * std::max(d, F)));
+        if (!wh) {
+            const int ks[2] = {d, F};
+            for (int i = 0; i < 2; ++i)
+                for (int j = 0; j < 2; ++j)
+                    DEC_TRY(make_wmap(h, &h->m_xq8[i][j], h->xq8, h->xq8_rows, ks[i], false, j ? 32 : 16));
+        }
         DEC_TRY(dalloc(h, &h->xs8, size_t(MB) * 4));
         size_t pb = 16;
         int cl = 1;
@@ -938,10 +951,10 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
             cl = std::max(cl, mma_counters(p, MB));
         };
         auto need_i8 = [&](int n, int k) {
-            const MmaPlan p = i8mma_plan(n, k, h->num_sms);
+            const MmaPlan p = tc_plan(n, k, h->num_sms);
             if (!p.ok) return;
-            pb = std::max(pb, i8mma_part_bytes(p, MB));
-            cl = std::max(cl, i8mma_counters(p, MB));
+            pb = std::max(pb, tc_part_bytes(p, MB));
+            cl = std::max(cl, tc_counters(p, MB));
         };
         need_f32(c.vocab, d, 4);
         const int shapes[4][2] = {{3 * d, d}, {d, d}, {F, d}, {d, F}};
