@@ -141,6 +141,17 @@ typedef struct dec_handle dec_handle;
  * `DecoderScratch`: per-token buffers allocated once). The caller may free
  * its weight buffers after the call. On error *out is NULL and nothing leaks;
  * the message is available from dec_last_error(NULL) on the same thread.
+ * Besides the packed weights the handle keeps, for the tensor-core paths:
+ * the embedding as three int8 digit planes plus row scales (3 bytes per
+ * element, for the LM head) and, for qwen2, row-permuted copies of the
+ * q|k|v and gate/up panels.
+ * Numerics: W8A8 products are exact int32 sums on every path; the LM head is
+ * computed from exact-integer products of three-digit splits of its f32
+ * operands (error below 2^-22 of each row's largest element per operand);
+ * f32 and W8A32 projections of batches of 8 or more may run on TF32 tensor
+ * cores with split operands (three / two products). A stream's logits never
+ * depend on the other streams of the batch for the head and W8A8 layers, and
+ * for f32 / W8A32 layers not within batches below 8 or within batches of 8+.
  */
 dec_status dec_create(const dec_config* cfg, const dec_weights* w, dec_handle** out);
 
