@@ -450,10 +450,21 @@ def main():
                     help="bracket the timed steps with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
     ap.add_argument("--fast-setup", action="store_true",
                     help="seed caches with N(0,1) K/V instead of prefilling tokens (profiling runs)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="profiling only: fewer streams than the workload (same model and kernels)")
+    ap.add_argument("--max-cache-len", type=int, default=0,
+                    help="profiling only: shorter caches, for ncu captures with a small device footprint")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     wl = synth.workload(CONFIGS[args.config])
+    if args.batch or args.max_cache_len:
+        # a reduced variant of the workload for profiling captures; named as such
+        L = min(args.max_cache_len or wl.max_cache_len, wl.max_cache_len)
+        hi = max(1, min(wl.lens_hi, L - wl.steps - 1))
+        wl = synth.scaled(wl, name=f"{wl.name} (profiling variant)", batch=args.batch or wl.batch,
+                          max_cache_len=L, lens_lo=min(wl.lens_lo, hi), lens_hi=hi,
+                          retire_at=min(wl.retire_at, L) if wl.retire_at else wl.retire_at)
     cfg = wl.model
     config = {"workload": wl.name, "batch": wl.batch, "n_layers": cfg.n_layers, "d_model": cfg.d_model,
               "vocab": cfg.vocab, "proj": cfg.proj_fmt, "cache_init": wl.cache_init,
