@@ -189,5 +189,5 @@ def test_step_kernel_count_is_reported():
     p.gpu.close()
     assert counts[0] > 0 and len(set(counts)) == 1, counts
     # embed, then per layer: q|k|v, self-attention, o, cross q, cross-attention, cross o,
-    # fc1, fc2; then the head's row split and the head
-    assert counts[0] == 1 + wl.model.n_layers * 8 + 2, counts
+    # fc1, fc2; then the head (which splits the hidden rows itself at batches up to 16)
+    assert counts[0] == 1 + wl.model.n_layers * 8 + 1, counts

@@ -370,15 +370,26 @@ template <int PRO>
 dec_status head(dec_handle* h, const GemvArgs& a, cudaStream_t st) {
     if (h->head_tc_ok) {
         const int d = h->cfg.d_model;
-        cudaError_t e = rowprep_digits_launch<PRO>(a.x, a.x_ld, a.norm_w, a.norm_b, a.eps, d, a.B,
-                                                   static_cast<long long>(h->xdig_rows) * d, h->xdig, h->xsc, true, st);
-        if (e != cudaSuccess) return cuda_fail(h, e, "head row split launch");
+        // batches above 16: the hidden rows' digit planes come from their own kernel;
+        // smaller batches make them inside the head kernel (same arithmetic)
+        const bool own = head_tc_makes_planes(a.B);
+        cudaError_t e = cudaSuccess;
+        if (!own) {
+            e = rowprep_digits_launch<PRO>(a.x, a.x_ld, a.norm_w, a.norm_b, a.eps, d, a.B,
+                                           static_cast<long long>(h->xdig_rows) * d, h->xdig, h->xsc, true, st);
+            if (e != cudaSuccess) return cuda_fail(h, e, "head row split launch");
+        }
         HeadArgs ha;
         ha.wmap = h->m_wdig;
         ha.xmap16 = h->m_xdig16;
         ha.xmap32 = h->m_xdig32;
         ha.wscale = h->wsc;
         ha.xscale = h->xsc;
+        ha.x = a.x;
+        ha.x_ld = a.x_ld;
+        ha.norm_w = a.norm_w;
+        ha.norm_b = a.norm_b;
+        ha.eps = a.eps;
         ha.V = h->cfg.vocab;
         ha.K = d;
         ha.B = a.B;
@@ -391,7 +402,7 @@ dec_status head(dec_handle* h, const GemvArgs& a, cudaStream_t st) {
         ha.last_tok = a.last_tok;
         ha.meta = a.meta;
         ha.err = a.err;
-        e = head_tc_launch(h->num_sms, ha, st);
+        e = head_tc_launch(h->num_sms, ha, own ? PRO : kHeadXExternal, st);
         if (e != cudaSuccess) return cuda_fail(h, e, "tensor-core head launch");
         return DEC_OK;
     }

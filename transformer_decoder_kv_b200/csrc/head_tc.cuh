@@ -50,7 +50,12 @@ struct HeadArgs {
     CUtensorMap xmap16;    // hidden digit planes [3 MB, K] int8: box {128 bytes, 16 rows}
     CUtensorMap xmap32;    // the same with boxes of 32 rows
     const float* wscale;   // [V] embedding row scales
-    const float* xscale;   // [MB] hidden row scales
+    const float* xscale;   // [MB] hidden row scales (hidden planes made by k_rowprep_digits)
+    const float* x;        // residual rows [B, K] (hidden planes made in the head kernel)
+    int x_ld;
+    const float* norm_w;   // final norm
+    const float* norm_b;
+    float eps;
     int V, K, B, MB;
     int n_by;              // batch tiles (fastest-varying CTA index)
     float* logits;         // [B, V] or null
@@ -75,20 +80,15 @@ __device__ __forceinline__ void digits3(float v, float inv, int& d1, int& d2, in
     d3 = static_cast<int>(e3);
 }
 
-// Digit planes of rows of a row-major f32 matrix: out[p][r][k], scale[r]. One warp per
-// row; `norm` applies the final LayerNorm / RMSNorm first (PRO) with the CUDA-core
-// prologue's arithmetic.
-template <int PRO>
-__global__ void __launch_bounds__(128) k_rowprep_digits(const float* __restrict__ x, int x_ld,
-                                                        const float* __restrict__ gw, const float* __restrict__ gb,
-                                                        float eps, int K, int rows, long long plane_stride,
-                                                        int8_t* __restrict__ out, float* __restrict__ scale) {
-    pdl_launch_dependents();
-    pdl_wait();
-    const int lane = threadIdx.x & 31;
-    const int r = blockIdx.x * 4 + (threadIdx.x >> 5);
-    if (r >= rows) return;
-    const float4* xr = reinterpret_cast<const float4*>(x + static_cast<long long>(r) * x_ld);
+// One row's three digit planes, computed by one warp (the final LayerNorm / RMSNorm first
+// when PRO says so, with the CUDA-core projection prologue's arithmetic): `sink(k4, p1, p2,
+// p3)` receives the packed digits of elements 4 k4 .. 4 k4 + 3; returns the row scale.
+// Every caller uses this one function, so the digits do not depend on where they are made.
+template <int PRO, class Sink>
+__device__ __forceinline__ float row_digits_warp(const float* __restrict__ x, const float* __restrict__ gw,
+                                                 const float* __restrict__ gb, float eps, int K, int lane,
+                                                 Sink sink) {
+    const float4* xr = reinterpret_cast<const float4*>(x);
     const int K4 = K >> 2;
     float mu = 0.0f, rstd = 1.0f;
     if (PRO == PRO_LN) {
@@ -139,9 +139,6 @@ __global__ void __launch_bounds__(128) k_rowprep_digits(const float* __restrict_
     }
     amax = warp_max(amax);
     const float inv = amax > 0.0f ? 127.0f / amax : 0.0f;
-    uint32_t* o1 = reinterpret_cast<uint32_t*>(out + static_cast<long long>(r) * K);
-    uint32_t* o2 = reinterpret_cast<uint32_t*>(out + plane_stride + static_cast<long long>(r) * K);
-    uint32_t* o3 = reinterpret_cast<uint32_t*>(out + 2 * plane_stride + static_cast<long long>(r) * K);
     for (int k = lane; k < K4; k += 32) {
         const float4 v = normed(k);
         const float e[4] = {v.x, v.y, v.z, v.w};
@@ -154,11 +151,33 @@ __global__ void __launch_bounds__(128) k_rowprep_digits(const float* __restrict_
             p2 |= (static_cast<uint32_t>(b) & 0xffu) << (8 * j);
             p3 |= (static_cast<uint32_t>(c) & 0xffu) << (8 * j);
         }
-        o1[k] = p1;
-        o2[k] = p2;
-        o3[k] = p3;
+        sink(k, p1, p2, p3);
     }
-    if (lane == 0) scale[r] = amax / 127.0f;
+    return amax / 127.0f;
+}
+
+// Digit planes of rows of a row-major f32 matrix: out[p][r][k], scale[r]. One warp per
+// row (the embedding once at load; the hidden rows of batches above 16 every step).
+template <int PRO>
+__global__ void __launch_bounds__(128) k_rowprep_digits(const float* __restrict__ x, int x_ld,
+                                                        const float* __restrict__ gw, const float* __restrict__ gb,
+                                                        float eps, int K, int rows, long long plane_stride,
+                                                        int8_t* __restrict__ out, float* __restrict__ scale) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int r = blockIdx.x * 4 + (threadIdx.x >> 5);
+    if (r >= rows) return;
+    uint32_t* o1 = reinterpret_cast<uint32_t*>(out + static_cast<long long>(r) * K);
+    uint32_t* o2 = reinterpret_cast<uint32_t*>(out + plane_stride + static_cast<long long>(r) * K);
+    uint32_t* o3 = reinterpret_cast<uint32_t*>(out + 2 * plane_stride + static_cast<long long>(r) * K);
+    const float sc = row_digits_warp<PRO>(x + static_cast<long long>(r) * x_ld, gw, gb, eps, K, lane,
+                                          [&](int k4, uint32_t p1, uint32_t p2, uint32_t p3) {
+                                              o1[k4] = p1;
+                                              o2[k4] = p2;
+                                              o3[k4] = p3;
+                                          });
+    if (lane == 0) scale[r] = sc;
 }
 
 // ---- tcgen05 / TMEM primitives ----------------------------------------------------
@@ -237,7 +256,11 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-template <int BT>
+// XPRO: kHeadXExternal when k_rowprep_digits made the hidden planes (read by TMA), else the
+// final norm (PRO_LN / PRO_RMS) with which this kernel makes them itself.
+constexpr int kHeadXExternal = -1;
+
+template <int BT, int XPRO>
 __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_constant__ HeadArgs A, int NS) {
     static_assert(BT == 16 || BT == 32, "batch tile");
     constexpr int ACC = 3 * BT;                           // TMEM columns of one accumulator set
@@ -308,15 +331,40 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
     pdl_launch_dependents();
     pdl_wait();
 
-    if (tid < BT) s_xs[tid] = tid < nb ? A.xscale[b0 + tid] : 0.0f;
+    if (XPRO == kHeadXExternal) {
+        if (tid < BT) s_xs[tid] = tid < nb ? A.xscale[b0 + tid] : 0.0f;
+    } else {
+        // the hidden planes in the swizzled K-major layout the MMA reads: zero first (rows past
+        // the batch, columns past K), then one warp per row writes its digits
+        for (int o = tid * 16; o < 3 * xplane; o += kHeadThreads * 16)
+            *reinterpret_cast<uint4*>(sx + o) = make_uint4(0u, 0u, 0u, 0u);
+        if (tid < BT) s_xs[tid] = 0.0f;
+        __syncthreads();
+        for (int b = warp; b < nb; b += kHeadThreads / 32) {
+            const float sc = row_digits_warp<(XPRO < 0 ? PRO_NONE : XPRO)>(
+                A.x + static_cast<long long>(b0 + b) * A.x_ld, A.norm_w, A.norm_b, A.eps, A.K, lane,
+                [&](int k4, uint32_t p1, uint32_t p2, uint32_t p3) {
+                    const int j = (4 * k4) & 127;   // byte within the 128-byte row of chunk (4 k4) / 128
+                    const int off = ((4 * k4) >> 7) * BT * 128 + b * 128 + (((j >> 4) ^ (b & 7)) << 4) + (j & 15);
+                    *reinterpret_cast<uint32_t*>(sx + off) = p1;
+                    *reinterpret_cast<uint32_t*>(sx + xplane + off) = p2;
+                    *reinterpret_cast<uint32_t*>(sx + 2 * xplane + off) = p3;
+                });
+            if (lane == 0) s_xs[b] = sc;
+        }
+        // generic-proxy shared-memory writes become visible to the tensor core
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
     __syncthreads();
     if (warp == 0 && lane == 0) {
-        // hidden digit planes of this batch tile (written by k_rowprep_digits)
-        mbar_arrive_expect_tx(&bar_x, 3 * xplane);
-        for (int p = 0; p < 3; ++p)
-            for (int c = 0; c < nch; ++c)
-                tma_load_2d(sx + p * xplane + c * BT * 128, BT == 16 ? &A.xmap16 : &A.xmap32, c * kHeadKC,
-                            p * A.MB + b0, &bar_x);
+        if (XPRO == kHeadXExternal) {
+            // hidden digit planes of this batch tile (written by k_rowprep_digits)
+            mbar_arrive_expect_tx(&bar_x, 3 * xplane);
+            for (int p = 0; p < 3; ++p)
+                for (int c = 0; c < nch; ++c)
+                    tma_load_2d(sx + p * xplane + c * BT * 128, BT == 16 ? &A.xmap16 : &A.xmap32, c * kHeadKC,
+                                p * A.MB + b0, &bar_x);
+        }
         // remaining weight stages
         for (int it = n_issued; it < n_items; ++it) {
             if (!mbar_wait_bounded(&empty[it % NS], static_cast<uint32_t>(it / NS - 1) & 1u, A.err)) {
@@ -328,7 +376,7 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
         }
     } else if (warp == 1 && lane == 0) {
         // ---- MMA issuer ----
-        bool ok = mbar_wait_bounded(&bar_x, 0, A.err);
+        bool ok = XPRO != kHeadXExternal || mbar_wait_bounded(&bar_x, 0, A.err);
         tc_fence_after();
         int it = 0;
         for (int i = 0; ok && i < my_blocks; ++i) {
@@ -470,7 +518,10 @@ template <int PRO>
 cudaError_t rowprep_digits_launch(const float* x, int x_ld, const float* gw, const float* gb, float eps, int K,
                                   int rows, long long plane_stride, int8_t* out, float* scale, bool pdl,
                                   cudaStream_t st);
-cudaError_t head_tc_launch(int num_sms, const HeadArgs& a, cudaStream_t st);
+// pro: the final norm when the head kernel makes the hidden planes itself (batches up to
+// 16), kHeadXExternal when k_rowprep_digits made them
+cudaError_t head_tc_launch(int num_sms, const HeadArgs& a, int pro, cudaStream_t st);
+inline bool head_tc_makes_planes(int B) { return B <= 16; }
 
 #ifdef DEC_HEAD_TC_DEFINE
 
@@ -491,7 +542,7 @@ cudaError_t rowprep_digits_launch(const float* x, int x_ld, const float* gw, con
     return cudaLaunchKernelEx(&cfg, k_rowprep_digits<PRO>, x, x_ld, gw, gb, eps, K, rows, plane_stride, out, scale);
 }
 
-template <int BT>
+template <int BT, int XPRO>
 cudaError_t head_tc_launch_bt(int num_sms, HeadArgs a, cudaStream_t st) {
     const int ns = head_tc_stages(a.K, BT);
     if (ns == 0) return cudaErrorNotSupported;
@@ -501,7 +552,7 @@ cudaError_t head_tc_launch_bt(int num_sms, HeadArgs a, cudaStream_t st) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (attr_dev != dev) {
-        e = cudaFuncSetAttribute(k_head_tc<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024 - 1024);
+        e = cudaFuncSetAttribute(k_head_tc<BT, XPRO>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024 - 1024);
         if (e != cudaSuccess) return e;
         attr_dev = dev;
     }
@@ -519,13 +570,18 @@ cudaError_t head_tc_launch_bt(int num_sms, HeadArgs a, cudaStream_t st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_head_tc<BT>, a, ns);
+    return cudaLaunchKernelEx(&cfg, k_head_tc<BT, XPRO>, a, ns);
 }
 
-cudaError_t head_tc_launch(int num_sms, const HeadArgs& a, cudaStream_t st) {
+cudaError_t head_tc_launch(int num_sms, const HeadArgs& a, int pro, cudaStream_t st) {
     if (a.B < 1 || a.B > a.MB) return cudaErrorInvalidValue;
-    if (head_tc_bt(a.B) == 16) return head_tc_launch_bt<16>(num_sms, a, st);
-    return head_tc_launch_bt<32>(num_sms, a, st);
+    if (head_tc_makes_planes(a.B)) {
+        if (pro == PRO_LN) return head_tc_launch_bt<16, PRO_LN>(num_sms, a, st);
+        if (pro == PRO_RMS) return head_tc_launch_bt<16, PRO_RMS>(num_sms, a, st);
+        return cudaErrorInvalidValue;
+    }
+    if (pro != kHeadXExternal) return cudaErrorInvalidValue;
+    return head_tc_launch_bt<32, kHeadXExternal>(num_sms, a, st);
 }
 
 #endif  // DEC_HEAD_TC_DEFINE
