@@ -191,3 +191,18 @@ def test_step_kernel_count_is_reported():
     # embed, then per layer: q|k|v, self-attention, o, cross q, cross-attention, cross o,
     # fc1, fc2; then the head (which splits the hidden rows itself at batches up to 16)
     assert counts[0] == 1 + wl.model.n_layers * 8 + 1, counts
+
+
+def test_head_digit_planes_made_in_kernel_or_by_row_kernel_give_same_bits():
+    """Up to batch 16 the tensor-core head splits the hidden rows itself; above 16 a row
+    kernel does it first. Both call one device function, and the products are exact integer
+    sums, so a stream's logits are the same bits in a batch of 17 and in a batch of 9."""
+    wl = synth.scaled(synth.workload("mid_whisper_b9"), batch=17)
+    p17 = build_pair(wl)
+    p9 = build_pair(wl, streams=list(range(9)), max_slots=9)
+    toks = list(range(300, 317))
+    l17 = step_both(p17, toks)[0]
+    l9 = step_both(p9, toks[:9])[0]
+    assert np.array_equal(l17[:9].view(np.uint32), l9.view(np.uint32))
+    p17.gpu.close()
+    p9.gpu.close()
