@@ -459,12 +459,12 @@ int choose_splits(const dec_handle* h, int rows, int max_tiles) {
 }
 
 dec_status attention(dec_handle* h, AttnArgs a, int B, int max_keys, int tps, cudaStream_t st) {
-    static int configured = 0;
-    if (!configured) {
+    thread_local int configured_dev = -1;   // attributes are per device
+    if (configured_dev != h->device) {
         DEC_CUDA(h, cudaFuncSetAttribute(k_attention, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kAttnSmemBytes)));
         DEC_CUDA(h, cudaFuncSetAttribute(k_attention, cudaFuncAttributePreferredSharedMemoryCarveout,
                                          cudaSharedmemCarveoutMaxShared));
-        configured = 1;
+        configured_dev = h->device;
     }
     // fixed tiles per split (a handle constant): each row's split boundaries, hence its
     // summation order, depend only on its own length
@@ -1202,15 +1202,15 @@ dec_status dec_attention(const float* q, const float* k, const float* v, const i
     if (batch < 1 || n_heads < 1 || ld < 1) return DEC_EINVAL;
     if (workspace_bytes < dec_attention_workspace_size(batch, n_heads, ld)) return DEC_EINVAL;
     if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15) return DEC_EINVAL;
-    static int configured = 0;
-    if (!configured) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    thread_local int configured_dev = -1;   // attributes are per device
+    if (configured_dev != dev) {
         if (cudaFuncSetAttribute(k_attention, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kAttnSmemBytes)) !=
             cudaSuccess)
             return DEC_ECUDA;
-        configured = 1;
+        configured_dev = dev;
     }
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     AttnArgs a{};
     a.q = q;

@@ -62,26 +62,28 @@ template <int BT, typename WT, bool I8, int PRO, int EPI, int MAP>
 cudaError_t gemv_launch_bt(int num_sms, const GemvArgs& a, cudaStream_t st) {
     auto kern = k_gemv<BT, WT, I8, PRO, EPI, MAP>;
     const GemvPlan p = gemv_plan<WT, I8, PRO>(BT, a.K);
-    static bool attr_set = false;  // per instantiation
-    cudaError_t e;
-    if (!attr_set) {
+    thread_local int attr_dev = -1;   // attributes are per device; set again when it changes
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (attr_dev != dev) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemvSmemMax - 2048));
         if (e != cudaSuccess) return e;
         // one shared-memory carveout for every kernel of the step, so that consecutive
         // kernels can share an SM without reconfiguring it
         e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        attr_dev = dev;
     }
     const int n_pairs = (MAP == MAP_DUAL) ? a.N : (a.N + 1) / 2;
     const int pairs_per_task = gemv_rows_per_task(BT) / 2;
     const int n_tasks = (n_pairs + pairs_per_task - 1) / pairs_per_task;
     const int n_blocks = (n_tasks + gemv_consumer_warps(BT) - 1) / gemv_consumer_warps(BT);
-    // occupancy for this instantiation, cached per shared-memory size
-    static size_t occ_smem[8] = {~size_t(0), ~size_t(0), ~size_t(0), ~size_t(0),
+    // occupancy for this instantiation, cached per shared-memory size (per thread)
+    thread_local size_t occ_smem[8] = {~size_t(0), ~size_t(0), ~size_t(0), ~size_t(0),
                                  ~size_t(0), ~size_t(0), ~size_t(0), ~size_t(0)};
-    static int occ_val[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    static int occ_next = 0;
+    thread_local int occ_val[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    thread_local int occ_next = 0;
     auto occupancy = [&](size_t smem, int* occ) -> cudaError_t {
         for (int i = 0; i < 8; ++i)
             if (occ_smem[i] == smem) {

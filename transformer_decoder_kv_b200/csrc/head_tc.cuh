@@ -547,7 +547,7 @@ cudaError_t head_tc_launch_bt(int num_sms, HeadArgs a, cudaStream_t st) {
     const int ns = head_tc_stages(a.K, BT);
     if (ns == 0) return cudaErrorNotSupported;
     const size_t smem = head_tc_smem(a.K, BT, ns);
-    static int attr_dev = -1;
+    thread_local int attr_dev = -1;   // attributes are per device; set again when it changes
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;

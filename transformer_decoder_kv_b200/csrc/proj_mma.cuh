@@ -611,7 +611,7 @@ cudaError_t proj_mma_launch_bt(int num_sms, MmaArgs A, int n_blocks, cudaStream_
     const size_t avail = size_t(227 * 1024) - 1024 - 1024 - xbytes;
     const int ns_max = int(std::min<size_t>(kMmaMaxStagesTF, avail / SB));
     if (ns_max < 2) return cudaErrorNotSupported;
-    static int attr_dev = -1;
+    thread_local int attr_dev = -1;   // attributes are per device; set again when it changes
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
