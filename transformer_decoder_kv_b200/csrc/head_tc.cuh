@@ -505,7 +505,6 @@ inline size_t head_tc_smem(int K, int bt, int ns) {
     const int nch = (K + kHeadKC - 1) / kHeadKC;
     return 1024 + size_t(ns) * kHeadStageBytes + size_t(3) * nch * bt * 128;
 }
-inline int head_tc_bt(int B) { return B <= 16 ? 16 : 32; }
 // stages that fit next to the hidden planes (0: the head does not fit)
 inline int head_tc_stages(int K, int bt) {
     if (K % 16 != 0 || K > kHeadMaxK) return 0;
