@@ -132,6 +132,19 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def clocks_rejected(clocks: dict) -> bool:
+    """A timed region whose clock record shows a hardware or thermal slowdown, or SM clocks
+    held well below their maximum with no reason given (a leftover clock lock), does not
+    give a valid number; power capping alone is kept (normal on a 1 kW part)."""
+    reasons = set(clocks.get("reasons") or [])
+    if reasons & {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}:
+        return True
+    sm, smax = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    if sm and smax and sm < 0.8 * smax and not (reasons & {"sw_power_cap"}):
+        return True
+    return False
+
+
 # ---------------------------------------------------------------- workload setup (GPU)
 
 class GpuWorkload:
@@ -241,6 +254,7 @@ def run_ours(args, wl: synth.Workload, rank: int, world: int) -> dict:
         if args.profile_range:
             torch.cuda.profiler.stop()
         clocks = clk.stop()
+        clocks["rejected"] = clocks_rejected(clocks)
         ms = e0.elapsed_time(e1)
         gw.dec.sync(sh)
     value, ms_max, tokens_all = combine_ranks(ms, tokens, world)
