@@ -195,6 +195,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_proj_mma(const __grid_consta
     __shared__ __align__(8) uint64_t empty[kMmaMaxStagesTF];
     __shared__ __align__(8) uint64_t bar_x;
     __shared__ unsigned long long s_key[BT];
+    __shared__ int s_slot[BT], s_len[BT];   // EPI_QKV: the batch tile's cache slots and rows
     __shared__ int s_flag, s_last;   // staging succeeded; this CTA arrived last (head)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -249,6 +250,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_proj_mma(const __grid_consta
         s_flag = mbar_wait_bounded(&bar_x, 0, a.err) ? 1 : 0;
     }
     if (EPI == EPI_HEAD && tid < BT) s_key[tid] = 0ull;
+    if (EPI == EPI_QKV && tid < BT) {
+        s_slot[tid] = tid < nb ? a.meta->slot[b0 + tid] : 0;
+        s_len[tid] = tid < nb ? a.meta->len[b0 + tid] : 0;
+    }
     __syncthreads();
     if (!s_flag) {
         if (producer && lane == 0)
@@ -265,18 +270,31 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_proj_mma(const __grid_consta
     for (int nt = 0; nt < NT; ++nt) best[nt][0] = best[nt][1] = 0ull;
 
     const int g = lane >> 2, t = lane & 3;
+    // Global inputs of one output element's epilogue (row scale, bias, residual value).
+    // A warp loads all of them for its elements before its first store: a load placed
+    // after a store to memory it might alias waits for that store, one L2 round trip
+    // per element.
+    struct EpiIn {
+        float s, bias, prev;
+    };
+    auto load_in = [&](int n, int b) {
+        EpiIn v{1.0f, 0.0f, 0.0f};
+        if (!F32W) v.s = a.scale[n];
+        if (EPI != EPI_HEAD && a.bias != nullptr) v.bias = a.bias[n];
+        if (EPI == EPI_RESID) v.prev = a.out[static_cast<long long>(b0 + b) * a.out_ld + n];
+        return v;
+    };
     // epilogue of one output element
     // (nt, e: the argmax accumulator of column b = 8 nt + 2 t + e, compile-time at every
     // call; nt < 0 folds into the CTA's shared keys instead)
-    auto finish = [&](int n, int b, float y, int nt, int e) {
-        if (!F32W) y = __fmul_rn(y, a.scale[n]);
-        if (EPI != EPI_HEAD && a.bias != nullptr) y = __fadd_rn(y, a.bias[n]);
+    auto finish = [&](int n, int b, float y, const EpiIn& in, int nt, int e) {
+        if (!F32W) y = __fmul_rn(y, in.s);
+        if (EPI != EPI_HEAD && a.bias != nullptr) y = __fadd_rn(y, in.bias);
         const int gb = b0 + b;
         if (EPI == EPI_STORE) {
             a.out[static_cast<long long>(gb) * a.out_ld + n] = y;
         } else if (EPI == EPI_RESID) {
-            float* p = a.out + static_cast<long long>(gb) * a.out_ld + n;
-            *p = __fadd_rn(*p, y);
+            a.out[static_cast<long long>(gb) * a.out_ld + n] = __fadd_rn(in.prev, y);
         } else if (EPI == EPI_GELU) {
             a.out[static_cast<long long>(gb) * a.out_ld + n] = gelu_tanh_f(y);
         } else if (EPI == EPI_QKV) {
@@ -285,9 +303,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_proj_mma(const __grid_consta
             if (sec == 0) {
                 a.out[static_cast<long long>(gb) * a.out_ld + within] = y;
             } else {
-                const int slot = a.meta->slot[gb], row = a.meta->len[gb];
                 float* cache = (sec == 1) ? a.kc : a.vc;
-                cache[slot * a.slot_stride + (static_cast<long long>(hh) * a.ld + row) * kHeadDim + i] = y;
+                cache[s_slot[b] * a.slot_stride + (static_cast<long long>(hh) * a.ld + s_len[b]) * kHeadDim + i] = y;
             }
         } else if (EPI == EPI_HEAD) {
             if (a.out != nullptr) a.out[static_cast<long long>(gb) * a.out_ld + n] = y;
@@ -419,6 +436,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_proj_mma(const __grid_consta
             // ---- block done: epilogue directly, or through the split-K reduction ----
             // C fragment: e = 0,1 -> row g, columns 2t, 2t+1; e = 2,3 -> row g + 8
             if (A.n_ks == 1) {
+                EpiIn in[2][NT][4];
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -427,7 +445,17 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_proj_mma(const __grid_consta
                         for (int e = 0; e < 4; ++e) {
                             const int n = jb * kMmaBlockRows + 32 * warp + 16 * mt + g + 8 * (e >> 1);
                             const int b = nt * 8 + 2 * t + (e & 1);
-                            if (b < nb && n < a.N) finish(n, b, acc[mt][nt][e], nt, e & 1);
+                            if (b < nb && n < a.N) in[mt][nt][e] = load_in(n, b);
+                        }
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int n = jb * kMmaBlockRows + 32 * warp + 16 * mt + g + 8 * (e >> 1);
+                            const int b = nt * 8 + 2 * t + (e & 1);
+                            if (b < nb && n < a.N) finish(n, b, acc[mt][nt][e], in[mt][nt][e], nt, e & 1);
                         }
             } else {
                 float* tile = reinterpret_cast<float*>(A.part) +
@@ -490,16 +518,26 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_proj_mma(const __grid_consta
                             sum[j].w += v.w;
                         }
                     }
+                    EpiIn in[V][4];
+#pragma unroll
+                    for (int j = 0; j < V; ++j) {
+                        const int e0 = (lane + 32 * j) * 4;
+                        const int n = jb * kMmaBlockRows + 32 * warp + e0 / BT;
+                        const int bc = e0 % BT;
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            if (n < a.N && bc + u < nb) in[j][u] = load_in(n, bc + u);
+                    }
 #pragma unroll
                     for (int j = 0; j < V; ++j) {
                         const int e0 = (lane + 32 * j) * 4;
                         const int n = jb * kMmaBlockRows + 32 * warp + e0 / BT;
                         const int bc = e0 % BT;
                         if (n < a.N) {
-                            if (bc < nb) finish(n, bc, sum[j].x, -1, 0);
-                            if (bc + 1 < nb) finish(n, bc + 1, sum[j].y, -1, 0);
-                            if (bc + 2 < nb) finish(n, bc + 2, sum[j].z, -1, 0);
-                            if (bc + 3 < nb) finish(n, bc + 3, sum[j].w, -1, 0);
+                            if (bc < nb) finish(n, bc, sum[j].x, in[j][0], -1, 0);
+                            if (bc + 1 < nb) finish(n, bc + 1, sum[j].y, in[j][1], -1, 0);
+                            if (bc + 2 < nb) finish(n, bc + 2, sum[j].z, in[j][2], -1, 0);
+                            if (bc + 3 < nb) finish(n, bc + 3, sum[j].w, in[j][3], -1, 0);
                         }
                     }
                     if (lane == 0) *cw = 0;
@@ -689,6 +727,9 @@ cudaError_t proj_mma_launch(int num_sms, const CUtensorMap& map, void* part, siz
 template <int PRO>
 cudaError_t rowprep_launch(const GemvArgs& g, float* out, cudaStream_t st) {
     if (g.K > kRowprepMaxK || g.K % 4 != 0) return cudaErrorNotSupported;
+    thread_local int attr_dev = -1;
+    const cudaError_t e = prefer_max_shared_once(k_rowprep<PRO>, attr_dev);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(g.B);
     cfg.blockDim = dim3(kRowprepThreads);

@@ -9,4 +9,5 @@ namespace dec {
 DEC_PROJ_TC_INSTANTIATE(EPI_QKV, MAP_ROPE)
 DEC_PROJ_TC_INSTANTIATE(EPI_RESID, MAP_ADJ)
 DEC_PROJ_TC_INSTANTIATE(EPI_SWIGLU, MAP_DUAL)
+DEC_PROJ_TC_INSTANTIATE(EPI_I32, MAP_ADJ)
 }  // namespace dec

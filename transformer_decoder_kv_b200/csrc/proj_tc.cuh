@@ -74,6 +74,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
     __shared__ __align__(8) uint64_t tfull[2], tempty[2], bar_x, bar_done;
     __shared__ uint32_t s_tmem;
     __shared__ float s_xs[BT];
+    __shared__ int s_pos[BT], s_slot[BT], s_len[BT];   // EPI_QKV: the batch tile's step description
     __shared__ int s_fail;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -126,7 +127,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
         for (; n_issued < NS && n_issued < n_items; ++n_issued) issue(n_issued);
     pdl_launch_dependents();
     pdl_wait();
-    if (tid < BT) s_xs[tid] = tid < nb ? A.xs[b0 + tid] : 0.0f;
+    if (tid < BT) {
+        s_xs[tid] = tid < nb ? A.xs[b0 + tid] : 0.0f;
+        if (EPI == EPI_QKV) {
+            s_pos[tid] = tid < nb ? a.meta->pos[b0 + tid] : 0;
+            s_slot[tid] = tid < nb ? a.meta->slot[b0 + tid] : 0;
+            s_len[tid] = tid < nb ? a.meta->len[b0 + tid] : 0;
+        }
+    }
     __syncthreads();
 
     if (warp == 0 && lane == 0) {
@@ -223,12 +231,45 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
                 if (lane == 0) A.cnt[grp] = 0;
             }
             // ---- dequantise and finish row p for every batch column ----
+            // Every global input of the epilogue (row scale, bias, the residual values, the
+            // RoPE table entries) is loaded before the first store: a load placed after a
+            // store to memory it might alias would wait for that store, one L2 round trip
+            // per batch column.
             const int p = jb * 128 + q * 32 + lane;
             const bool row_live = p < A.n_rows;
             const int n = tc_logical_row<MAP>(p);
             const float* sc = (MAP == MAP_DUAL && (p & 1)) ? a.scale2 : a.scale;
             const float sn = row_live ? sc[n] : 0.0f;
             const float bn = (EPI != EPI_SWIGLU && a.bias != nullptr && row_live) ? a.bias[n] : 0.0f;
+            int sec = 0, within = n, hh = 0, col = 0;
+            if (EPI == EPI_QKV) {
+                sec = n / a.d;
+                within = n - sec * a.d;
+                hh = within >> 6;
+                col = within & 63;
+            }
+            constexpr bool kRope = EPI == EPI_QKV && MAP == MAP_ROPE;
+            float prev[EPI == EPI_RESID ? BT : 1];
+            float2 cs[kRope ? BT : 1];
+            if (EPI == EPI_RESID) {
+#pragma unroll
+                for (int b = 0; b < BT; ++b)
+                    prev[b] = (b < nb && row_live) ? a.out[static_cast<long long>(b0 + b) * a.out_ld + n] : 0.0f;
+            }
+            if (kRope) {
+                const bool rot = a.rope != nullptr && sec < 2 && row_live;
+#pragma unroll
+                for (int b = 0; b < BT; ++b)
+                    cs[b] = (rot && b < nb) ? a.rope[static_cast<long long>(s_pos[b]) * 32 + (col & 31)]
+                                            : make_float2(1.0f, 0.0f);
+            }
+            if (EPI == EPI_I32) {
+                // the exact int32 sums themselves (kernel-level check of the integer products)
+#pragma unroll
+                for (int b = 0; b < BT; ++b)
+                    if (b < nb && row_live) a.out_i32[static_cast<long long>(b0 + b) * a.out_ld + n] = acc[b];
+                continue;
+            }
 #pragma unroll
             for (int b = 0; b < BT; ++b) {
                 float y = __fmul_rn(static_cast<float>(acc[b]), __fmul_rn(s_xs[b], sn));
@@ -237,28 +278,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
                 if (b >= nb || !row_live) continue;
                 const int gb = b0 + b;
                 if (EPI == EPI_RESID) {
-                    float* o = a.out + static_cast<long long>(gb) * a.out_ld + n;
-                    *o = __fadd_rn(*o, y);
+                    a.out[static_cast<long long>(gb) * a.out_ld + n] = __fadd_rn(prev[EPI == EPI_RESID ? b : 0], y);
                 } else if (EPI == EPI_SWIGLU) {
                     if ((p & 1) == 0) a.out[static_cast<long long>(gb) * a.out_ld + n] = __fmul_rn(silu_f(y), yp);
                 } else if (EPI == EPI_QKV) {
-                    const int sec = n / a.d, within = n - sec * a.d;
-                    const int hh = within >> 6, i = within & 63;
                     float val = y;
-                    if (MAP == MAP_ROPE && a.rope != nullptr && sec < 2) {
-                        const float2 cs = a.rope[static_cast<long long>(a.meta->pos[gb]) * 32 + (i & 31)];
+                    if (kRope && a.rope != nullptr && sec < 2) {
+                        const float2 c = cs[kRope ? b : 0];
                         // pair (i, i + 32): x_i' = x_i c - x_{i+32} s ; x_{i+32}' = x_i s + x_{i+32} c
-                        if (i < 32)
-                            val = __fsub_rn(__fmul_rn(y, cs.x), __fmul_rn(yp, cs.y));
+                        if (col < 32)
+                            val = __fsub_rn(__fmul_rn(y, c.x), __fmul_rn(yp, c.y));
                         else
-                            val = __fadd_rn(__fmul_rn(yp, cs.y), __fmul_rn(y, cs.x));
+                            val = __fadd_rn(__fmul_rn(yp, c.y), __fmul_rn(y, c.x));
                     }
                     if (sec == 0) {
                         a.out[static_cast<long long>(gb) * a.out_ld + within] = val;
                     } else {
-                        const int slot = a.meta->slot[gb], row = a.meta->len[gb];
                         float* cache = (sec == 1) ? a.kc : a.vc;
-                        cache[slot * a.slot_stride + (static_cast<long long>(hh) * a.ld + row) * kHeadDim + i] = val;
+                        cache[s_slot[b] * a.slot_stride + (static_cast<long long>(hh) * a.ld + s_len[b]) * kHeadDim + col] =
+                            val;
                     }
                 } else if (EPI == EPI_STORE) {
                     a.out[static_cast<long long>(gb) * a.out_ld + n] = y;
@@ -352,6 +390,8 @@ cudaError_t proj_tc_launch_bt(int num_sms, TcArgs A, int n_blocks, cudaStream_t 
     if (e != cudaSuccess) return e;
     if (attr_dev != dev) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024 - 1024);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         attr_dev = dev;
     }
