@@ -255,19 +255,31 @@ dec_status dec_step_kernels(const dec_handle* h, int32_t* kernels);
  * s_j = q . k_j / 8, max-subtracted softmax, sum_j p_j v_j; a row whose
  * softmax sum is not finite and positive gives zeros, [q8] full-attention step).
  *   q        device f32 [batch, n_heads, 64]
- *   k, v     device f32 [batch, n_heads, ld, 64] (head-first, ld rows per head)
+ *   k, v     device f32 [batch, n_heads, ld, 64] (head-first, ld rows per head),
+ *            16-byte aligned
  *   lens     device int32 [batch]: keys attended per stream (rows 0..lens[b]-1),
  *            0 <= lens[b] <= ld; lens[b] == 0 gives zeros
+ *   tiles_per_split  64-key tiles per CTA of a row: 0 splits every row alike
+ *            (the split count minimising waves x tiles per CTA); a positive value
+ *            fixes each row's split boundaries from its own length, as the decode
+ *            step does (dec_attention_plan gives a handle's value); at most 32
+ *            splits over ld rows (DEC_EINVAL otherwise)
  *   out      device f32 [batch, n_heads, 64]
  *   workspace device scratch of at least dec_attention_workspace_size(batch,
  *            n_heads, ld) bytes, 16-byte aligned; its first
  *            batch * n_heads int32 must be zero before the first call (each call
  *            leaves them zero again)
+ * Errors set dec_last_error(NULL).
  */
 size_t dec_attention_workspace_size(int32_t batch, int32_t n_heads, int32_t ld);
 dec_status dec_attention(const float* q, const float* k, const float* v, const int32_t* lens,
-                         int32_t batch, int32_t n_heads, int32_t ld, float* out,
+                         int32_t batch, int32_t n_heads, int32_t ld, int32_t tiles_per_split, float* out,
                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Tiles per split of a handle's self-attention (cross = 0) or cross-attention
+ * (cross = 1, whisper) launches in dec_step, for timing the step's own launch
+ * shape through dec_attention. Host-only. */
+dec_status dec_attention_plan(const dec_handle* h, int32_t cross, int32_t* tiles_per_split);
 
 /*
  * Allocation-free variant of dec_attention, for callers that cannot allocate
@@ -275,16 +287,19 @@ dec_status dec_attention(const float* q, const float* k, const float* v, const i
  * owns the whole device and hands plug-ins no workspace, or latency-critical
  * paths where cudaMalloc's implicit device synchronisation is not acceptable.
  * (It has no counterpart in the pages; it is an interface convenience only.)
- * Same arguments, numerics and output as dec_attention, minus the workspace:
- * the split-K scratch lives in one fixed array of about 2.2 MB inside this
- * library, which every GPU that loads the library holds until the process exits.
+ * Same arguments as dec_attention with tiles_per_split = 0, minus the workspace,
+ * and the same launch, hence the same output bits: the split-K scratch lives in
+ * one fixed array of about 8.9 MB inside this library, which every GPU that loads
+ * the library holds until the process exits.
  * Limits: batch * n_heads <= 1024 (DEC_EINVAL otherwise, message from
- * dec_last_error(NULL)). The first call on a device looks up that array's device
- * address (cudaGetSymbolAddress) with the device current; make that first call
- * before any stream capture. Every call clears the arrival counters it needs
- * (cudaMemsetAsync on `stream`) and shares the one array, which keeps the last
- * call's contents: calls that overlap on the GPU (different streams, no ordering)
- * race on it. It allocates nothing.
+ * dec_last_error(NULL)). Every call looks up that array's device address
+ * (cudaGetSymbolAddress) with the calling thread's current device; make the first
+ * call on a device before any stream capture (it may load the module). Every call
+ * clears the status word and the arrival counters it needs (cudaMemsetAsync on
+ * `stream`) and shares the one array, which keeps the last call's contents: calls
+ * that overlap on the GPU (different streams, no ordering) race on it. A bounded
+ * device wait that gives up (about a second) leaves `out` undefined; it is noted in
+ * the array's status word only and not reported by this call. It allocates nothing.
  */
 dec_status dec_attention_noalloc(const float* q, const float* k, const float* v, const int32_t* lens,
                                  int32_t batch, int32_t n_heads, int32_t ld, float* out, void* stream);
@@ -293,9 +308,15 @@ dec_status dec_attention_noalloc(const float* q, const float* k, const float* v,
  * int8 x int8 -> int32 dot products acc[m, n] = sum_k xq[m, k] * wq[n, k]
  * (the accumulator of [focr] `gemv_i8_bias_prequant`). xq device int8 [m, kdim],
  * wq device int8 [n, kdim], acc device int32 [m, n]; kdim a multiple of 16,
- * 1 <= m <= 64.
+ * 1 <= m <= 64, xq and wq 16-byte aligned. `path` selects the kernel the decode
+ * step uses for that batch size: DEC_I8_PATH_DP4A (CUDA cores, dp4a, batches
+ * below 8) or DEC_I8_PATH_TCGEN05 (tcgen05.mma kind::i8 with TMEM accumulators,
+ * batches of 8 or more; this path allocates its split-K scratch with
+ * cudaMallocAsync on `stream` and frees it after the launch). Errors set
+ * dec_last_error(NULL).
  */
-dec_status dec_i8_dot(const int8_t* xq, const int8_t* wq, int32_t m, int32_t n, int32_t kdim,
+enum { DEC_I8_PATH_DP4A = 0, DEC_I8_PATH_TCGEN05 = 1 };
+dec_status dec_i8_dot(const int8_t* xq, const int8_t* wq, int32_t m, int32_t n, int32_t kdim, int32_t path,
                       int32_t* acc, void* stream);
 
 #ifdef __cplusplus

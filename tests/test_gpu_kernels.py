@@ -62,6 +62,28 @@ def test_i8_dot_is_bit_exact(torch_cuda, m, n, k):
     assert np.array_equal(acc.cpu().numpy().astype(np.int64), oracle.int8_dot_acc(xq, wq))
 
 
+@pytest.mark.parametrize("m", [8, 16, 17, 32, 64])
+@pytest.mark.parametrize("n,k", [(3072, 1024), (5632, 1024), (1024, 2816), (200, 384)])
+def test_i8_dot_tcgen05_is_bit_exact(torch_cuda, m, n, k):
+    """The tcgen05 kind::i8 kernel the W8A8 step uses from batch 8 on: its int32
+    accumulators (TMEM, split-K partials added by the last arriving warp) equal the
+    exact integer dot products, including the largest magnitudes (127 * 127 * K)."""
+    torch = torch_cuda
+    from transformer_decoder_kv_b200 import i8_dot
+    rng = np.random.default_rng(m * 7919 + n + k)
+    xq = rng.integers(-127, 128, size=(m, k)).astype(np.int8)
+    wq = rng.integers(-127, 128, size=(n, k)).astype(np.int8)
+    xq[0, :] = 127
+    wq[0, :] = 127
+    wq[1, :] = -127
+    acc = torch.full((m, n), -1, dtype=torch.int32, device="cuda")
+    i8_dot(torch.from_numpy(xq).cuda(), torch.from_numpy(wq).cuda(), m, n, k, acc, path="tcgen05")
+    torch.cuda.synchronize()
+    want = oracle.int8_dot_acc(xq, wq)
+    assert want[0, 0] == 127 * 127 * k
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), want)
+
+
 @pytest.mark.parametrize("lens,ld", [([1, 0, 64, 65], 80), ([31, 1500, 7], 1500),
                                      ([4129, 128, 2000, 4096], 4129)])
 def test_attention_op_matches_oracle(torch_cuda, lens, ld):

@@ -25,7 +25,9 @@ PROJ = {"f32": 0, "w8a8": 1, "w8a32": 2}
 # Every symbol include/dec.h declares.
 EXPORTS = ["dec_create", "dec_destroy", "dec_last_error", "dec_prefill", "dec_kv_append", "dec_step",
            "dec_step_host", "dec_slot_len", "dec_kv_read", "dec_hidden", "dec_sync", "dec_step_kernels",
-           "dec_attention_workspace_size", "dec_attention", "dec_attention_noalloc", "dec_i8_dot"]
+           "dec_attention_workspace_size", "dec_attention", "dec_attention_plan", "dec_attention_noalloc",
+           "dec_i8_dot"]
+I8_PATH = {"dp4a": 0, "tcgen05": 1}
 
 
 class DecError(RuntimeError):
@@ -82,9 +84,10 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
         "dec_sync": (C.c_int, [vp, vp]),
         "dec_step_kernels": (C.c_int, [vp, pi32]),
         "dec_attention_workspace_size": (C.c_size_t, [i32, i32, i32]),
-        "dec_attention": (C.c_int, [vp, vp, vp, vp, i32, i32, i32, vp, vp, C.c_size_t, vp]),
+        "dec_attention": (C.c_int, [vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, C.c_size_t, vp]),
+        "dec_attention_plan": (C.c_int, [vp, i32, pi32]),
         "dec_attention_noalloc": (C.c_int, [vp, vp, vp, vp, i32, i32, i32, vp, vp]),
-        "dec_i8_dot": (C.c_int, [vp, vp, i32, i32, i32, vp, vp]),
+        "dec_i8_dot": (C.c_int, [vp, vp, i32, i32, i32, i32, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -218,6 +221,12 @@ class Decoder:
     def sync(self, stream: int = 0):
         self._check(self._lib.dec_sync(self._h, stream))
 
+    def attention_plan(self, cross: bool = False) -> int:
+        """Tiles per split of the step's self- (or cross-) attention launches."""
+        n = C.c_int32(0)
+        self._check(self._lib.dec_attention_plan(self._h, 1 if cross else 0, C.byref(n)))
+        return int(n.value)
+
     def step_kernels(self) -> int:
         """Kernels launched by one step of the most recent step call (-1: not captured)."""
         n = C.c_int32(0)
@@ -225,27 +234,27 @@ class Decoder:
         return int(n.value)
 
 
-def attention(q, k, v, lens, batch: int, n_heads: int, ld: int, out, workspace, workspace_bytes: int,
-              stream: int = 0):
-    st = lib().dec_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(lens), batch, n_heads, ld, _ptr(out),
-                             _ptr(workspace), workspace_bytes, stream)
+def _raise_thread_error(st: int):
     if st != DEC_OK:
-        raise DecError(st, "dec_attention failed")
+        raise DecError(st, lib().dec_last_error(None).decode())
+
+
+def attention(q, k, v, lens, batch: int, n_heads: int, ld: int, out, workspace, workspace_bytes: int,
+              stream: int = 0, tiles_per_split: int = 0):
+    _raise_thread_error(lib().dec_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(lens), batch, n_heads, ld,
+                                            tiles_per_split, _ptr(out), _ptr(workspace), workspace_bytes,
+                                            stream))
 
 
 def attention_noalloc(q, k, v, lens, batch: int, n_heads: int, ld: int, out, stream: int = 0):
     """dec_attention without a caller workspace: the library's fixed scratch array is used."""
-    st = lib().dec_attention_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(lens), batch, n_heads, ld,
-                                     _ptr(out), stream)
-    if st != DEC_OK:
-        raise DecError(st, lib().dec_last_error(None).decode())
+    _raise_thread_error(lib().dec_attention_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(lens), batch, n_heads, ld,
+                                                    _ptr(out), stream))
 
 
 def attention_workspace_size(batch: int, n_heads: int, ld: int) -> int:
     return int(lib().dec_attention_workspace_size(batch, n_heads, ld))
 
 
-def i8_dot(xq, wq, m: int, n: int, kdim: int, acc, stream: int = 0):
-    st = lib().dec_i8_dot(_ptr(xq), _ptr(wq), m, n, kdim, _ptr(acc), stream)
-    if st != DEC_OK:
-        raise DecError(st, "dec_i8_dot failed")
+def i8_dot(xq, wq, m: int, n: int, kdim: int, acc, stream: int = 0, path: str = "dp4a"):
+    _raise_thread_error(lib().dec_i8_dot(_ptr(xq), _ptr(wq), m, n, kdim, I8_PATH[path], _ptr(acc), stream))

@@ -141,8 +141,10 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
         if (tid == 0) s_flag = mbar_wait_bounded(&bars[stage], phase, a.err) ? 1 : 0;
         __syncthreads();
         if (!s_flag) {
-            // Give the copies still in flight a bounded chance to land before the
-            // shared memory is released, then leave.
+            // Give the copies still in flight a bounded chance to land, then stop reading
+            // tiles. The CTA still merges and arrives below, so the row's arrival count
+            // returns to zero for the next launch; the status word already says that this
+            // launch's output is not valid.
             if (tid == 0) {
                 for (int t2 = t; t2 < min(t1, t + NS); ++t2) {
                     const int it2 = t2 - t0;
@@ -150,7 +152,7 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
                 }
             }
             __syncthreads();
-            return;
+            break;
         }
         // the phase is complete; each thread observes it itself (acquire of the bulk writes)
         if (tid != 0) (void)mbar_try_wait(&bars[stage], phase);

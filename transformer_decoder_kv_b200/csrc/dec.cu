@@ -18,6 +18,7 @@
 
 #include "../../include/dec.h"
 #include "attention.cuh"
+#include "attn_plan.h"
 #include "common.cuh"
 #include "gemv.cuh"
 #include "gemv_launch.cuh"
@@ -32,7 +33,7 @@ using namespace dec;
 namespace {
 
 constexpr int kMetaRing = 8;
-constexpr int kMaxSplits = 32;
+constexpr int kMaxSplits = kAttnMaxSplits;
 
 thread_local std::string g_create_error;
 
@@ -438,26 +439,6 @@ dec_status make_wmap(dec_handle* h, CUtensorMap* m, const void* w, int rows, int
     return DEC_OK;
 }
 
-// Split count for one attention launch: minimise (waves x tiles per CTA).
-int choose_splits(const dec_handle* h, int rows, int max_tiles) {
-    if (max_tiles <= 1) return 1;
-    const int slots = h->num_sms * 2;
-    int best = 1;
-    double best_cost = 1e30;
-    for (int s = 1; s <= std::min(kMaxSplits, max_tiles); ++s) {
-        const int tps = (max_tiles + s - 1) / s;
-        const int eff = (max_tiles + tps - 1) / tps;
-        if (eff != s) continue;
-        const double waves = std::ceil(double(rows) * s / slots);
-        const double cost = waves * (tps + 1.5) + (s > 1 ? 0.5 : 0.0);
-        if (cost < best_cost) {
-            best_cost = cost;
-            best = s;
-        }
-    }
-    return best;
-}
-
 dec_status attention(dec_handle* h, AttnArgs a, int B, int max_keys, int tps, cudaStream_t st) {
     thread_local int configured_dev = -1;   // attributes are per device
     if (configured_dev != h->device) {
@@ -468,26 +449,17 @@ dec_status attention(dec_handle* h, AttnArgs a, int B, int max_keys, int tps, cu
     }
     // fixed tiles per split (a handle constant): each row's split boundaries, hence its
     // summation order, depend only on its own length
-    const int max_tiles = (max_keys + kAttnTile - 1) / kAttnTile;
-    a.tps = tps;
-    a.S = std::max(1, (max_tiles + tps - 1) / tps);
-    // one stage per CTA (more resident CTAs) at 1 and 4 tiles per split, two at 2 and 8+:
-    // measured on B200 (HBM-resident caches) as the fastest for each split size
-    a.stages = (tps == 2 || tps >= 8) ? 2 : 1;
-    const size_t smem = size_t(a.stages) * 2 * kAttnTile * kHeadDim * sizeof(float);
-    DEC_CUDA(h, launch(k_attention, dim3(a.S, a.H, B), dim3(kAttnThreads), smem, st, a));
+    const AttnLaunch p = attn_launch_plan(h->num_sms, B * a.H, max_keys, tps);
+    a.tps = p.tps;
+    a.S = p.S;
+    a.stages = p.stages;
+    DEC_CUDA(h, launch(k_attention, dim3(a.S, a.H, B), dim3(kAttnThreads), attn_smem_bytes(p.stages), st, a));
     return DEC_OK;
 }
 
-// Tiles per split for a handle: finer splits when few (stream, head) rows exist, and
-// never more than kMaxSplits splits over the longest possible row.
+// Tiles per split of the handle's self- or cross-attention launches.
 int tiles_per_split(const dec_handle* h, int max_keys) {
-    const int rows_cap = h->cfg.n_heads * h->max_batch;
-    const int tiles_cap = (max_keys + kAttnTile - 1) / kAttnTile;
-    // measured on B200 with HBM-resident caches: few rows and short caches favour two
-    // tiles per split (double-buffered), more rows or longer caches four or eight
-    int t = rows_cap <= 32 ? 1 : (rows_cap <= 256 && tiles_cap <= 8) ? 2 : (rows_cap <= 1023 ? 4 : 8);
-    return std::max(t, (tiles_cap + kMaxSplits - 1) / kMaxSplits);
+    return attn_tiles_per_split(h->cfg.n_heads * h->max_batch, max_keys);
 }
 
 GemvArgs base_args(dec_handle* h, int B) {
@@ -503,6 +475,10 @@ GemvArgs base_args(dec_handle* h, int B) {
 dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int* argmax, cudaStream_t st) {
     const dec_config& c = h->cfg;
     const int d = c.d_model, F = c.d_ff, H = c.n_heads;
+    {
+        thread_local int attr_dev = -1;
+        DEC_CUDA(h, prefer_max_shared_once(k_embed, attr_dev));
+    }
     DEC_CUDA(h, launch(k_embed, dim3(B), dim3(128), 0, st, (const float*)h->tok_emb, (const float*)h->pos_emb,
                        (const StepMeta*)h->dmeta, (const int*)h->last_tok, h->x, d));
     for (int l = 0; l < c.n_layers; ++l) {
@@ -1196,22 +1172,24 @@ size_t dec_attention_workspace_size(int32_t batch, int32_t n_heads, int32_t ld) 
 }
 
 dec_status dec_attention(const float* q, const float* k, const float* v, const int32_t* lens, int32_t batch,
-                         int32_t n_heads, int32_t ld, float* out, void* workspace, size_t workspace_bytes,
-                         void* stream) {
-    if (!q || !k || !v || !lens || !out || !workspace) return DEC_EINVAL;
-    if (batch < 1 || n_heads < 1 || ld < 1) return DEC_EINVAL;
-    if (workspace_bytes < dec_attention_workspace_size(batch, n_heads, ld)) return DEC_EINVAL;
-    if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15) return DEC_EINVAL;
+                         int32_t n_heads, int32_t ld, int32_t tiles_per_split, float* out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    auto bad = [](const char* m) { return fail(nullptr, DEC_EINVAL, std::string("dec_attention: ") + m); };
+    if (!q || !k || !v || !lens || !out || !workspace) return bad("null pointer");
+    if (batch < 1 || n_heads < 1 || ld < 1) return bad("batch, n_heads and ld must be >= 1");
+    if (tiles_per_split < 0) return bad("tiles_per_split must be >= 0");
+    if (workspace_bytes < dec_attention_workspace_size(batch, n_heads, ld)) return bad("workspace too small");
+    if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(workspace)) &
+        15)
+        return bad("k, v and workspace must be 16-byte aligned");
     int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    thread_local int configured_dev = -1;   // attributes are per device
-    if (configured_dev != dev) {
-        if (cudaFuncSetAttribute(k_attention, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kAttnSmemBytes)) !=
-            cudaSuccess)
-            return DEC_ECUDA;
-        configured_dev = dev;
-    }
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_attention, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kAttnSmemBytes));
+    if (e != cudaSuccess) return cuda_fail(nullptr, e, "dec_attention: device set-up");
+    const AttnLaunch p = attn_launch_plan(sms, batch * n_heads, ld, tiles_per_split);
+    if (p.S > kMaxSplits) return bad("tiles_per_split gives more than 32 splits over ld rows");
     AttnArgs a{};
     a.q = q;
     a.q_bstride = (long long)n_heads * 64;
@@ -1229,23 +1207,37 @@ dec_status dec_attention(const float* q, const float* k, const float* v, const i
     a.counters = static_cast<int*>(workspace);
     a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + counters);
     a.err = nullptr;
-    dec_handle tmp;
-    tmp.num_sms = sms;
-    const int max_tiles = (ld + kAttnTile - 1) / kAttnTile;
-    a.S = choose_splits(&tmp, batch * n_heads, max_tiles);
-    cudaError_t e = launch(k_attention, dim3(a.S, n_heads, batch), dim3(kAttnThreads), kAttnSmemBytes,
-                           static_cast<cudaStream_t>(stream), a);
-    return e == cudaSuccess ? DEC_OK : DEC_ECUDA;
+    a.S = p.S;
+    a.tps = p.tps;
+    a.stages = p.stages;
+    e = launch(k_attention, dim3(a.S, n_heads, batch), dim3(kAttnThreads), attn_smem_bytes(p.stages),
+               static_cast<cudaStream_t>(stream), a);
+    if (e != cudaSuccess) return cuda_fail(nullptr, e, "dec_attention: k_attention launch");
+    return DEC_OK;
 }
 
-dec_status dec_i8_dot(const int8_t* xq, const int8_t* wq, int32_t m, int32_t n, int32_t kdim, int32_t* acc,
-                      void* stream) {
-    if (!xq || !wq || !acc) return DEC_EINVAL;
-    if (m < 1 || m > 64 || n < 1 || kdim < 16 || kdim % 16) return DEC_EINVAL;
+dec_status dec_attention_plan(const dec_handle* h, int32_t cross, int32_t* tiles_per_split) {
+    if (!h || !tiles_per_split) return fail(nullptr, DEC_EINVAL, "dec_attention_plan: null pointer");
+    if (cross && h->cfg.family != DEC_FAMILY_WHISPER)
+        return fail(const_cast<dec_handle*>(h), DEC_EINVAL, "dec_attention_plan: the model has no cross-attention");
+    *tiles_per_split = cross ? h->tps_cross : h->tps_self;
+    return DEC_OK;
+}
+
+dec_status dec_i8_dot(const int8_t* xq, const int8_t* wq, int32_t m, int32_t n, int32_t kdim, int32_t path,
+                      int32_t* acc, void* stream) {
+    auto bad = [](const char* msg) { return fail(nullptr, DEC_EINVAL, std::string("dec_i8_dot: ") + msg); };
+    if (!xq || !wq || !acc) return bad("null pointer");
+    if (m < 1 || m > 64 || n < 1 || kdim < 16 || kdim % 16) return bad("need 1 <= m <= 64, n >= 1, kdim a multiple of 16");
+    if (path != DEC_I8_PATH_DP4A && path != DEC_I8_PATH_TCGEN05) return bad("unknown path");
+    if ((reinterpret_cast<uintptr_t>(xq) | reinterpret_cast<uintptr_t>(wq)) & 15)
+        return bad("xq and wq must be 16-byte aligned");
     dec_handle tmp;
     int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&tmp.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&tmp.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(nullptr, e, "dec_i8_dot: device query");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
     GemvArgs g{};
     g.xq = xq;
     g.x_ld = kdim;
@@ -1255,8 +1247,38 @@ dec_status dec_i8_dot(const int8_t* xq, const int8_t* wq, int32_t m, int32_t n, 
     g.W = wq;
     g.out_i32 = acc;
     g.out_ld = n;
-    dec_status st = gemv<int8_t, true, PRO_RAW_I8, EPI_I32, MAP_ADJ>(&tmp, g, static_cast<cudaStream_t>(stream));
-    return st;
+    if (path == DEC_I8_PATH_DP4A) {
+        e = gemv_launch<int8_t, true, PRO_RAW_I8, EPI_I32, MAP_ADJ>(tmp.num_sms, g, st);
+        if (e != cudaSuccess) return cuda_fail(nullptr, e, "dec_i8_dot: k_gemv launch");
+        return DEC_OK;
+    }
+    // tcgen05: TMA maps of both operands, split-K scratch of the plan, then the same
+    // kernel the decode step runs (EPI_I32 stores the exact int32 sums).
+    const MmaPlan p = tc_plan(n, kdim, tmp.num_sms);
+    if (!p.ok) return bad("shape not supported by the tensor-core plan");
+    tmp.device = dev;
+    CUtensorMap wmap, x16, x32;
+    if (make_wmap(&tmp, &wmap, wq, n, kdim, false) != DEC_OK || make_wmap(&tmp, &x16, xq, m, kdim, false, 16) != DEC_OK ||
+        make_wmap(&tmp, &x32, xq, m, kdim, false, 32) != DEC_OK)
+        return fail(nullptr, DEC_ECUDA, "dec_i8_dot: " + tmp.err);
+    const size_t pb = std::max<size_t>(16, tc_part_bytes(p, m));
+    const int cl = std::max(1, tc_counters(p, m));
+    void* part = nullptr;
+    int* cnt = nullptr;
+    float* xs = nullptr;
+    e = cudaMallocAsync(&part, pb, st);
+    if (e == cudaSuccess) e = cudaMallocAsync(reinterpret_cast<void**>(&cnt), size_t(cl) * 4, st);
+    if (e == cudaSuccess) e = cudaMallocAsync(reinterpret_cast<void**>(&xs), size_t(m) * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(cnt, 0, size_t(cl) * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(xs, 0, size_t(m) * 4, st);
+    if (e == cudaSuccess)
+        e = proj_tc_launch<EPI_I32, MAP_ADJ>(tmp.num_sms, wmap, x16, x32, n, xs, part, pb, cnt, cl, g, st);
+    const cudaError_t launch_err = e;
+    if (part) cudaFreeAsync(part, st);
+    if (cnt) cudaFreeAsync(cnt, st);
+    if (xs) cudaFreeAsync(xs, st);
+    if (launch_err != cudaSuccess) return cuda_fail(nullptr, launch_err, "dec_i8_dot: tcgen05 path");
+    return DEC_OK;
 }
 
 }  // extern "C"

@@ -4,73 +4,34 @@
 
 #include <cuda_runtime.h>
 
-#include <mutex>
 #include <string>
 
 #include "../../include/dec.h"
-#include "attention.cuh"
+#include "attn_plan.h"
 
 void dec_set_thread_error(const char* msg);
 
 namespace {
 
 constexpr int kNoAllocMaxRows = 1024;   // batch * n_heads
-constexpr int kNoAllocMaxSplits = 8;
+constexpr int kNoAllocMaxSplits = dec::kAttnMaxSplits;   // the same split cap as dec_attention
+constexpr size_t kStatusBytes = 256;    // device status word, padded to the array's alignment
 constexpr size_t kCounterBytes = size_t(kNoAllocMaxRows) * sizeof(int);   // 4 KB, 256-aligned
 constexpr size_t kPartBytes = size_t(kNoAllocMaxRows) * kNoAllocMaxSplits * dec::kAttnPartStride * sizeof(float);
-constexpr size_t kScratchBytes = kCounterBytes + kPartBytes;
-constexpr int kMaxDevices = 64;
+constexpr size_t kScratchBytes = kStatusBytes + kCounterBytes + kPartBytes;
 
 }  // namespace
 
-// The scratch: counters [1024] int32, then partial states [1024][8][68] f32. In host
-// code this name is only a stand-in; the device address comes from cudaGetSymbolAddress.
+// The scratch: a status word (padded to 256 bytes), arrival counters [1024] int32, then
+// partial states [1024][32][68] f32 -- about 8.9 MB. In host code this name is only a
+// stand-in; the device address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_attn_noalloc_scratch[kScratchBytes];
 
 namespace {
 
-std::mutex g_setup_mu;
-void* g_scratch_addr[kMaxDevices] = {};
-
 dec_status fail(dec_status st, const std::string& msg) {
     dec_set_thread_error(msg.c_str());
     return st;
-}
-
-// Once per device, with that device current: the array's device address, and the
-// kernel's shared-memory opt-in.
-dec_status setup(int dev, void** addr) {
-    std::lock_guard<std::mutex> lock(g_setup_mu);
-    if (g_scratch_addr[dev] == nullptr) {
-        void* p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, g_attn_noalloc_scratch);
-        if (e != cudaSuccess) return fail(DEC_ECUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
-        e = cudaFuncSetAttribute(dec::k_attention, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(dec::kAttnSmemBytes));
-        if (e != cudaSuccess) return fail(DEC_ECUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
-        g_scratch_addr[dev] = p;
-    }
-    *addr = g_scratch_addr[dev];
-    return DEC_OK;
-}
-
-// Split count: fewest waves x tiles per CTA, at most kNoAllocMaxSplits.
-int splits_for(int num_sms, int rows, int max_tiles) {
-    if (max_tiles <= 1) return 1;
-    const int slots = num_sms * 2;
-    int best = 1;
-    double best_cost = 1e30;
-    for (int s = 1; s <= (max_tiles < kNoAllocMaxSplits ? max_tiles : kNoAllocMaxSplits); ++s) {
-        const int tps = (max_tiles + s - 1) / s;
-        if ((max_tiles + tps - 1) / tps != s) continue;
-        const double waves = double((rows * s + slots - 1) / slots);
-        const double cost = waves * (tps + 1.5) + (s > 1 ? 0.5 : 0.0);
-        if (cost < best_cost) {
-            best_cost = cost;
-            best = s;
-        }
-    }
-    return best;
 }
 
 }  // namespace
@@ -89,16 +50,24 @@ extern "C" dec_status dec_attention_noalloc(const float* q, const float* k, cons
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return fail(DEC_ECUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
-    if (dev < 0 || dev >= kMaxDevices) return fail(DEC_EINVAL, "dec_attention_noalloc: device index too large");
+    // The array's device address on the current device, looked up on every call (cheap once
+    // the module is loaded, and valid again after a device reset reloads it), and the
+    // kernel's shared-memory opt-in, which is per device as well.
     void* base = nullptr;
-    dec_status st = setup(dev, &base);
-    if (st != DEC_OK) return st;
+    e = cudaGetSymbolAddress(&base, g_attn_noalloc_scratch);
+    if (e != cudaSuccess) return fail(DEC_ECUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+    e = cudaFuncSetAttribute(dec::k_attention, cudaFuncAttributeMaxDynamicSharedMemorySize, int(dec::kAttnSmemBytes));
+    if (e != cudaSuccess) return fail(DEC_ECUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
     int sms = 148;
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return fail(DEC_ECUDA, std::string("cudaDeviceGetAttribute: ") + cudaGetErrorString(e));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the arrival counters must start at zero
-    e = cudaMemsetAsync(base, 0, size_t(batch) * n_heads * sizeof(int), s);
+    // the status word and the arrival counters must start at zero
+    e = cudaMemsetAsync(base, 0, kStatusBytes + size_t(batch) * n_heads * sizeof(int), s);
     if (e != cudaSuccess) return fail(DEC_ECUDA, std::string("cudaMemsetAsync: ") + cudaGetErrorString(e));
+    unsigned char* arr = static_cast<unsigned char*>(base);
+    // the launch dec_attention makes for the same arguments with tiles_per_split = 0
+    const dec::AttnLaunch p = dec::attn_launch_plan(sms, batch * n_heads, ld, 0);
     dec::AttnArgs a{};
     a.q = q;
     a.q_bstride = static_cast<long long>(n_heads) * dec::kHeadDim;
@@ -112,11 +81,13 @@ extern "C" dec_status dec_attention_noalloc(const float* q, const float* k, cons
     a.lens = lens;
     a.out = out;
     a.out_bstride = static_cast<long long>(n_heads) * dec::kHeadDim;
-    a.counters = static_cast<int*>(base);
-    a.part = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + kCounterBytes);
-    a.err = nullptr;
-    a.S = splits_for(sms, batch * n_heads, (ld + dec::kAttnTile - 1) / dec::kAttnTile);
-    dec::k_attention<<<dim3(a.S, n_heads, batch), dec::kAttnThreads, dec::kAttnSmemBytes, s>>>(a);
+    a.err = reinterpret_cast<int*>(arr);
+    a.counters = reinterpret_cast<int*>(arr + kStatusBytes);
+    a.part = reinterpret_cast<float*>(arr + kStatusBytes + kCounterBytes);
+    a.S = p.S;
+    a.tps = p.tps;
+    a.stages = p.stages;
+    dec::k_attention<<<dim3(a.S, n_heads, batch), dec::kAttnThreads, dec::attn_smem_bytes(p.stages), s>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(DEC_ECUDA, std::string("k_attention launch: ") + cudaGetErrorString(e));
     return DEC_OK;
