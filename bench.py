@@ -295,16 +295,18 @@ def run_ours(args, wl: synth.Workload, rank: int, world: int) -> dict:
     e2e = {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": meta_bytes,
            "d2h_bytes_per_step": wl.batch * (cfg.vocab * 4 + 4)}
 
-    roof = dominant_kernel_roofline(wl, cfg, lens_at_start) if rank == 0 else None
+    tps = gw.dec.attention_plan(cross=cfg.is_whisper)
+    roof = dominant_kernel_roofline(wl, cfg, lens_at_start, tps) if rank == 0 else None
     gw.dec.close()
     return dict(value=value, ms=ms_max, tokens=tokens_all, clocks=clocks, e2e=e2e, roofline=roof,
                 achieved_gbs=achieved_gbs, launches=launches,
                 step_bytes=statistics.mean(per_step_bytes))
 
 
-def dominant_kernel_roofline(wl, cfg, lens) -> dict:
-    """Time the workload's dominant kernel on its own (same kernel, same shapes) with CUDA
-    events; achieved = algorithmic bytes per launch / mean launch time."""
+def dominant_kernel_roofline(wl, cfg, lens, tiles_per_split: int) -> dict:
+    """Time the workload's dominant kernel on its own with CUDA events, in the launch shape
+    the decode step uses (the same grid: the handle's tiles per split over the step's
+    longest row); achieved = algorithmic bytes per launch / mean launch time."""
     import torch
     from transformer_decoder_kv_b200 import attention, attention_workspace_size
 
@@ -331,20 +333,23 @@ def dominant_kernel_roofline(wl, cfg, lens) -> dict:
     ws = torch.zeros(wsb // 4 + 1, dtype=torch.int32, device="cuda")
     s = torch.cuda.current_stream()
     for i in range(3):
-        attention(q, ks[i % nbuf], vs[i % nbuf], lens_d, B, H, ld, out, ws, wsb, s.cuda_stream)
+        attention(q, ks[i % nbuf], vs[i % nbuf], lens_d, B, H, ld, out, ws, wsb, s.cuda_stream, tiles_per_split)
     reps = 20
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(s)
     for i in range(reps):
-        attention(q, ks[i % nbuf], vs[i % nbuf], lens_d, B, H, ld, out, ws, wsb, s.cuda_stream)
+        attention(q, ks[i % nbuf], vs[i % nbuf], lens_d, B, H, ld, out, ws, wsb, s.cuda_stream, tiles_per_split)
     e1.record(s)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
     alg = sum(n * 64 * 4 * 2 for n in n_keys) * H + 2 * B * H * 64 * 4
     achieved = alg / (ms / 1e3) / 1e9
     traffic = recorded_traffic(wl.name)
-    return {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+    max_tiles = (ld + 63) // 64
+    grid = [-(-max_tiles // tiles_per_split), H, B]
+    return {"kernel": name, "grid": grid, "tiles_per_split": tiles_per_split, "bound": "hbm",
+            "achieved": round(achieved, 1), "peak": peak,
             "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)", "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": traffic, "algorithmic_bytes": alg,
             "launch_us": round(ms * 1e3, 2)}
@@ -368,11 +373,12 @@ def recorded_traffic(wl_name: str):
 
 # ---------------------------------------------------------------- CPU oracle
 
-def oracle_sample(wl: synth.Workload, seed: int, budget_s: float = 15.0):
+def oracle_sample(wl: synth.Workload, seed: int, budget_s: float = 15.0, cores: int = 0) -> dict:
     """Time the CPU oracle on a bounded sample of the workload: the first few streams
-    (at their own initial lengths), a few steps. Returns tokens/s and the sample."""
+    (at their own initial lengths), a few steps. Returns tokens/s and the sample. `cores`
+    is the BLAS thread count the caller set for this process (the oracle's arithmetic runs
+    in numpy's BLAS)."""
     import oracle
-    import torch
 
     cfg = wl.model
     W = synth.make_weights(cfg, seed)
@@ -401,31 +407,42 @@ def oracle_sample(wl: synth.Workload, seed: int, budget_s: float = 15.0):
                 st.n + 1 > wl.max_cache_len for st in states):
             break
     el = time.perf_counter() - t0
-    # the oracle's arithmetic runs in numpy's BLAS thread pool: report that pool's size, and a
-    # short single-thread continuation of the same streams beside the all-core figure
-    cores, single = torch.get_num_threads(), None
+    return {"value": n_streams * steps / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n_streams} of {wl.batch} streams at their seeded cache lengths, {steps} "
+                      f"decode steps, numpy f64 oracle ({el:.1f} s)"}
+
+
+BLAS_ENV = ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS", "BLIS_NUM_THREADS")
+
+
+def host_cores() -> int:
     try:
-        from threadpoolctl import threadpool_info, threadpool_limits
-        pools = [p.get("num_threads", 0) for p in threadpool_info() if p.get("user_api") == "blas"]
-        if pools:
-            cores = max(pools)
-        with threadpool_limits(limits=1):
-            t1, steps1 = time.perf_counter(), 0
-            while steps1 < max(1, steps // 2) and time.perf_counter() - t1 < max(2.0, budget_s / 3) and all(
-                    st.n + 1 <= wl.max_cache_len for st in states):
-                _, lg = ref.step(states, toks, [st.n for st in states])
-                toks = [int(np.argmax(r)) for r in lg]
-                steps1 += 1
-            if steps1:
-                single = n_streams * steps1 / (time.perf_counter() - t1)
-    except ImportError:
-        pass
-    out = {"value": n_streams * steps / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-           "sample": f"{n_streams} of {wl.batch} streams at their seeded cache lengths, {steps} "
-                     f"decode steps, numpy f64 oracle ({el:.1f} s)"}
-    if single is not None:
-        out["single_thread_value"] = single
-    return out
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_leg(config_key: str, budget_s: float, threads: int, extra: list = ()) -> dict:
+    """Run oracle_sample in a child process whose BLAS pools are set to `threads`."""
+    env = dict(os.environ)
+    for k in BLAS_ENV:
+        env[k] = str(threads)
+    cmd = [sys.executable, os.path.abspath(__file__), "--oracle-leg", "--config", config_key,
+           "--oracle-budget", str(budget_s), "--oracle-threads", str(threads), *extra]
+    r = subprocess.run(cmd, env=env, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"oracle leg failed: {r.stderr[-2000:]}")
+    return json.loads(r.stdout.strip().splitlines()[-1])
+
+
+def cpu_baseline(config_key: str, budget_s: float, extra: list = ()) -> dict:
+    """The oracle on all host cores, and a single-thread run of the same sample beside it."""
+    cores = host_cores()
+    allc = oracle_leg(config_key, budget_s, cores, extra)
+    one = oracle_leg(config_key, max(3.0, budget_s / 3), 1, extra)
+    allc["single_thread_value"] = one["value"]
+    allc["single_thread_sample"] = one["sample"]
+    return allc
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -478,7 +495,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=32)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="c2", choices=sorted(CONFIGS))
+    ap.add_argument("--config", default="c4", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-range", action="store_true",
@@ -489,6 +506,9 @@ def main():
                     help="profiling only: fewer streams than the workload (same model and kernels)")
     ap.add_argument("--max-cache-len", type=int, default=0,
                     help="profiling only: shorter caches, for ncu captures with a small device footprint")
+    ap.add_argument("--oracle-leg", action="store_true", help=argparse.SUPPRESS)
+    ap.add_argument("--oracle-budget", type=float, default=15.0, help=argparse.SUPPRESS)
+    ap.add_argument("--oracle-threads", type=int, default=0, help=argparse.SUPPRESS)
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -501,17 +521,23 @@ def main():
                           max_cache_len=L, lens_lo=min(wl.lens_lo, hi), lens_hi=hi,
                           retire_at=min(wl.retire_at, L) if wl.retire_at else wl.retire_at)
     cfg = wl.model
+    if args.oracle_leg:
+        print(json.dumps(oracle_sample(wl, 0, budget_s=args.oracle_budget, cores=args.oracle_threads)))
+        return
+    extra = (["--batch", str(args.batch)] if args.batch else []) + \
+        (["--max-cache-len", str(args.max_cache_len)] if args.max_cache_len else [])
     config = {"workload": wl.name, "batch": wl.batch, "n_layers": cfg.n_layers, "d_model": cfg.d_model,
               "vocab": cfg.vocab, "proj": cfg.proj_fmt, "cache_init": wl.cache_init,
               "cache_lens": f"U[{wl.lens_lo},{wl.lens_hi}]", "l2": "inputs larger than L2 per step"
               if step_bytes(cfg, synth.cache_lens(wl))["total"] > L2_BYTES else "n/a",
               "parallelism": f"replicas x{args.gpus}",
-              "cache_setup": "seeded K/V rows (profiling)" if args.fast_setup else wl.cache_init}
+              "cache_setup": "seeded K/V rows (profiling)" if args.fast_setup else wl.cache_init,
+              "fast_setup": bool(args.fast_setup)}
     metric = "decode tokens/s (device-timed)"
     if args.impl == "reference":
         if rank != 0:
             return
-        cb = oracle_sample(wl, 0, budget_s=max(5.0, min(60.0, 8.0 * max(1, args.steps) / 8)))
+        cb = cpu_baseline(args.config, max(5.0, min(60.0, float(max(1, args.steps)))), extra)
         # one step = one token for each of the workload's streams, at the oracle's rate
         line = {"impl": "reference", "metric": metric, "value": cb["value"], "unit": "tokens/s",
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -526,7 +552,7 @@ def main():
     r = run_ours(args, wl, rank, world)
     if rank != 0:
         return
-    cb = None if args.no_cpu_baseline or world > 1 else oracle_sample(wl, 0)
+    cb = None if args.no_cpu_baseline or world > 1 else cpu_baseline(args.config, 15.0, extra)
     dtype = {"f32": "f32", "w8a8": "int8 weights+activations, int32 acc, f32 elsewhere",
              "w8a32": "int8 weights, f32 activations"}[cfg.proj_fmt]
     peak, kind = measured_peaks()

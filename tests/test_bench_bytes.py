@@ -40,7 +40,7 @@ def test_hand_computed_qwen2_w8a8_step_counts_scales_and_qkv_bias():
     assert b["cross"] == 0
 
 
-def test_whisper_tiny_block_matches_the_survey_figure():
+def test_whisper_tiny_block_moves_92_9_mb_per_step():
     wl = synth.workload("c1_whisper_tiny_block_b1")
     b = bench.step_bytes(wl.model, synth.cache_lens(wl))
     assert b["head"] == 51865 * 384 * 4
