@@ -104,39 +104,47 @@ def quantize_weight_rows(w: np.ndarray):
     return q, s
 
 
-def int8_dot_acc(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:
+def _as64(w: np.ndarray, w64: Optional[np.ndarray]) -> np.ndarray:
+    """The weights in f64: `w64` when the caller already holds that exact conversion
+    (the decoder keeps one per matrix so that it converts each matrix once), else a new one."""
+    return w.astype(F64) if w64 is None else w64
+
+
+def int8_dot_acc(xq: np.ndarray, wq: np.ndarray, w64: Optional[np.ndarray] = None) -> np.ndarray:
     """Exact integer dot products acc[m, n] = sum_k xq[m,k] * wq[n,k] (int64).
 
     The int32 accumulation of the int8 GEMV ([focr] `gemv_i8_bias_prequant`,
     "int8, int32 accumulate"). f64 matmul is exact here: every product is at
     most 127^2 and every sum below 2^53. Pinned: brute-force Python int loop.
     """
-    acc = np.atleast_2d(xq).astype(F64) @ np.atleast_2d(wq).astype(F64).T
+    acc = np.atleast_2d(xq).astype(F64) @ _as64(np.atleast_2d(wq), w64).T
     return np.rint(acc).astype(np.int64)
 
 
-def linear_f32(x: np.ndarray, w: np.ndarray, b: Optional[np.ndarray]) -> np.ndarray:
+def linear_f32(x: np.ndarray, w: np.ndarray, b: Optional[np.ndarray],
+               w64: Optional[np.ndarray] = None) -> np.ndarray:
     """y = x W^T (+ b), f32 weights and activations ([cera] `linear_proj`).
 
     Pinned: zero weights give the bias (the page's own worked case:
     W = 0, b = 1 gives y = 1); brute-force loop on tiny shapes.
     """
-    y = np.atleast_2d(x).astype(F64) @ w.astype(F64).T
+    y = np.atleast_2d(x).astype(F64) @ _as64(w, w64).T
     if b is not None:
         y = y + b.astype(F64)
     return y.astype(F32)
 
 
 def linear_w8a8(xq: np.ndarray, a: np.ndarray, wq: np.ndarray, s: np.ndarray,
-                b: Optional[np.ndarray]) -> np.ndarray:
+                b: Optional[np.ndarray], w64: Optional[np.ndarray] = None) -> np.ndarray:
     """int8 x int8 projection: y_n = acc_n * (a * s_n) + b_n.
 
     [focr] `linear_auto` / `add_bias`: the int8 path dequantises the int32
     accumulator per row and adds the f32 bias after dequant. Reading of the
     dequant: acc times activation scale times row scale, then bias.
-    Pinned: integer part by brute force; zero activation row gives the bias.
+    Pinned: integer part by brute force; zero activation row gives the bias;
+    per-row scales by a brute-force loop with non-uniform scales.
     """
-    acc = int8_dot_acc(xq, wq).astype(F64)
+    acc = int8_dot_acc(xq, wq, w64).astype(F64)
     y = acc * np.asarray(a, dtype=F32).astype(F64)[:, None] * s.astype(F64)[None, :]
     if b is not None:
         y = y + b.astype(F64)
@@ -144,14 +152,15 @@ def linear_w8a8(xq: np.ndarray, a: np.ndarray, wq: np.ndarray, s: np.ndarray,
 
 
 def linear_w8a32(x: np.ndarray, wq: np.ndarray, s: np.ndarray,
-                 b: Optional[np.ndarray]) -> np.ndarray:
+                 b: Optional[np.ndarray], w64: Optional[np.ndarray] = None) -> np.ndarray:
     """int8 weights with f32 activations: y_n = s_n * sum_k q_nk x_k + b_n.
 
     [q8] module doc: int8 per-row weights are dequantised to f32 and used
     against f32 activations (`matmul_bt_q8`). Same value as dequantise-then-
-    matmul up to rounding. Pinned: equals linear_f32 on the dequantised matrix.
+    matmul up to rounding. Pinned: equals linear_f32 on the dequantised matrix;
+    per-row scales by a brute-force loop with non-uniform scales.
     """
-    y = (np.atleast_2d(x).astype(F64) @ wq.astype(F64).T) * s.astype(F64)[None, :]
+    y = (np.atleast_2d(x).astype(F64) @ _as64(wq, w64).T) * s.astype(F64)[None, :]
     if b is not None:
         y = y + b.astype(F64)
     return y.astype(F32)
@@ -315,6 +324,17 @@ class OracleDecoder:
         # int8 quantisations of the last forward_rows call.
         self.last_margins: Optional[np.ndarray] = None
         self._margins: Optional[np.ndarray] = None
+        # Tie bookkeeping of layer_forward (off unless a test asks): quantisation sites are
+        # numbered in call order within one layer (qwen2: 0 the q|k|v input, 1 the o input,
+        # 2 the gate/up input, 3 the down input). `tie_log`, when a list, receives
+        # (site, row, col, distance) for every activation whose x * inv lies within
+        # `tie_eps` code units of a rounding boundary; `flips` maps site -> [(row, col)] of
+        # activations to round to the other neighbouring integer instead (a correct
+        # implementation whose value sat on the other side of the tie).
+        self.tie_log: Optional[list] = None
+        self.tie_eps = 0.0
+        self.flips: Optional[dict] = None
+        self._site = 0
 
     # -- helpers ------------------------------------------------------------
 
@@ -326,36 +346,42 @@ class OracleDecoder:
         return c
 
     def _proj(self, x: np.ndarray, p: dict, key) -> np.ndarray:
-        """Whisper projection in the model's format (f32 or int8 weights, f32 acts)."""
+        """Whisper projection in the model's format: f32 weights (linear_f32) or int8
+        weights with per-row scales and f32 activations (linear_w8a32)."""
         w64 = self._w64(key, p["w"])
-        y = np.atleast_2d(x).astype(F64) @ w64.T
-        if p["s"] is not None:
-            y = y * p["s"].astype(F64)[None, :]
-        if p["b"] is not None:
-            y = y + p["b"].astype(F64)
-        return y.astype(F32)
+        if p["s"] is None:
+            return linear_f32(x, p["w"], p["b"], w64=w64)
+        return linear_w8a32(x, p["w"], p["s"], p["b"], w64=w64)
 
-    def _proj_i8(self, x: np.ndarray, p: dict, key) -> np.ndarray:
-        """Qwen2 W8A8 projection: quantise each input row, exact int dot, dequant, bias."""
-        xq, a = self._quant(x)
-        w64 = self._w64(key, p["w"])
-        acc = xq.astype(F64) @ w64.T
-        y = acc * a.astype(F64)[:, None] * p["s"].astype(F64)[None, :]
-        if p["b"] is not None:
-            y = y + p["b"].astype(F64)
-        return y.astype(F32)
+    def _proj_i8(self, x: np.ndarray, p: dict, key, quantised=None) -> np.ndarray:
+        """Qwen2 W8A8 projection (linear_w8a8): each input row quantised, exact integer
+        dot, dequantised, bias. `quantised` = (codes, scales) of x when the caller already
+        quantised it (one quantisation shared by several projections of the same row)."""
+        xq, a = self._quant(x) if quantised is None else quantised
+        return linear_w8a8(xq, a, p["w"], p["s"], p["b"], w64=self._w64(key, p["w"]))
 
     def _quant(self, x):
         if self._jitter is not None:
             x64 = np.atleast_2d(np.asarray(x, F32)).astype(F64)
             x = (x64 * (1.0 + self._jitter.uniform(-1.0, 1.0, x64.shape) * 2.0 ** -22)).astype(F32)
         q, a = quantize_rows_i8_te(x)
-        if self._margins is not None:
+        site = self._site
+        self._site += 1
+        if self._margins is not None or self.tie_log is not None or self.flips:
             x32 = np.atleast_2d(np.asarray(x, F32))
             inv = np.where(a > 0, F32(127.0) / np.where(a > 0, np.max(np.abs(x32), axis=1), F32(1)), F32(0))
             prod = (x32 * inv.astype(F32)[:, None]).astype(np.float64)
-            m = np.abs(prod - np.floor(prod) - 0.5).min(axis=1)
-            self._margins = np.minimum(self._margins, m)
+            dist = np.abs(prod - np.floor(prod) - 0.5)
+            if self._margins is not None:
+                self._margins = np.minimum(self._margins, dist.min(axis=1))
+            if self.tie_log is not None:
+                for r, c in zip(*np.nonzero(dist < self.tie_eps)):
+                    self.tie_log.append((site, int(r), int(c), float(dist[r, c])))
+            if self.flips and site in self.flips:
+                q = q.copy()
+                for r, c in self.flips[site]:
+                    alt = int(q[r, c]) + (1 if prod[r, c] > q[r, c] else -1)
+                    q[r, c] = np.int8(min(127, max(-127, alt)))
         return q, a
 
     def _norm(self, x, w, b):
@@ -380,7 +406,8 @@ class OracleDecoder:
 
     # -- forward ------------------------------------------------------------
 
-    def _embed(self, tokens, positions) -> np.ndarray:
+    def embed(self, tokens, positions) -> np.ndarray:
+        """x = E[token] (+ P[position] for whisper), one row per token."""
         cfg = self.cfg
         E = self.W["tok_emb"]
         x = np.empty((len(tokens), cfg.d_model), dtype=F32)
@@ -395,6 +422,88 @@ class OracleDecoder:
                 x[r] = x[r] + self.W["pos_emb"][int(p)]
         return x
 
+    def _self_attention(self, l, q, row_states, row_slots):
+        """Per row: attend cache rows 0..row_slots[r] of its own stream (all heads)."""
+        cfg = self.cfg
+        H, dh = cfg.n_heads, cfg.head_dim
+        ctx = np.empty_like(q)
+        views = {}
+        for r in range(len(row_slots)):
+            st = row_states[r]
+            if id(st) not in views:
+                top = max(sl for s2, sl in zip(row_states, row_slots) if s2 is st) + 1
+                views[id(st)] = (
+                    np.ascontiguousarray(st.k[l][:top].astype(F64).reshape(top, H, dh).transpose(1, 0, 2)),
+                    np.ascontiguousarray(st.v[l][:top].astype(F64).reshape(top, H, dh).transpose(1, 0, 2)))
+            kh, vh = views[id(st)]
+            n = row_slots[r] + 1
+            ctx[r] = _attend_heads(q[r].reshape(H, dh).astype(F64), kh[:, :n], vh[:, :n]).astype(F32).reshape(-1)
+        return ctx
+
+    def layer_forward(self, l: int, x: np.ndarray, row_states: Sequence[StreamState],
+                      row_slots: Sequence[int], positions: Sequence[int]) -> np.ndarray:
+        """Layer l of the decoder on rows x [R, d] (the residual stream entering the layer);
+        writes each row's K/V at its cache row and returns the residual leaving the layer.
+        Row r attends cache rows 0..row_slots[r] of its own stream."""
+        cfg = self.cfg
+        H, dh = cfg.n_heads, cfg.head_dim
+        R = x.shape[0]
+        L = self.W["layers"][l]
+        self._site = 0
+        # ---- self-attention block ----
+        h = self._norm(x, L["norm1_w"], L["norm1_b"])
+        if cfg.is_whisper:
+            q = self._proj(h, L["q"], (l, "q"))
+            k = self._proj(h, L["k"], (l, "k"))
+            v = self._proj(h, L["v"], (l, "v"))
+        else:
+            # one quantisation of the normed row shared by q, k, v ([focr] fused q|k|v GEMV)
+            hq = self._quant(h)
+            q = self._proj_i8(h, L["q"], (l, "q"), hq)
+            k = self._proj_i8(h, L["k"], (l, "k"), hq)
+            v = self._proj_i8(h, L["v"], (l, "v"), hq)
+            for r in range(R):
+                c, s = rope_cos_sin(int(positions[r]), cfg.rope_theta, dh)
+                q[r] = apply_rope_neox(q[r].reshape(H, dh), c, s).reshape(-1)
+                k[r] = apply_rope_neox(k[r].reshape(H, dh), c, s).reshape(-1)
+        for r in range(R):
+            row_states[r].k[l][row_slots[r]] = k[r]
+            row_states[r].v[l][row_slots[r]] = v[r]
+        ctx = self._self_attention(l, q, row_states, row_slots)
+        if cfg.is_whisper:
+            x = x + self._proj(ctx, L["o"], (l, "o"))
+        else:
+            x = x + self._proj_i8(ctx, L["o"], (l, "o"))
+        # ---- cross-attention block (whisper) ----
+        if cfg.is_whisper:
+            h = self._norm(x, L["norm2_w"], L["norm2_b"])
+            qx = self._proj(h, L["xq"], (l, "xq"))
+            cx = np.empty_like(qx)
+            xviews = {}
+            ne = cfg.enc_len
+            for r in range(R):
+                st = row_states[r]
+                if id(st) not in xviews:
+                    xviews[id(st)] = (
+                        np.ascontiguousarray(st.xk[l].astype(F64).reshape(ne, H, dh).transpose(1, 0, 2)),
+                        np.ascontiguousarray(st.xv[l].astype(F64).reshape(ne, H, dh).transpose(1, 0, 2)))
+                kh, vh = xviews[id(st)]
+                cx[r] = _attend_heads(qx[r].reshape(H, dh).astype(F64), kh, vh).astype(F32).reshape(-1)
+            x = x + self._proj(cx, L["xo"], (l, "xo"))
+        # ---- feed-forward block ----
+        if cfg.is_whisper:
+            h = self._norm(x, L["norm3_w"], L["norm3_b"])
+            f = gelu_tanh(self._proj(h, L["fc1"], (l, "fc1")))
+            x = x + self._proj(f, L["fc2"], (l, "fc2"))
+        else:
+            h = self._norm(x, L["norm2_w"], L["norm2_b"])
+            hq = self._quant(h)  # shared by gate and up
+            g = self._proj_i8(h, L["gate"], (l, "gate"), hq)
+            u = self._proj_i8(h, L["up"], (l, "up"), hq)
+            m = (silu(g) * u).astype(F32)
+            x = x + self._proj_i8(m, L["down"], (l, "down"))
+        return x
+
     def forward_rows(self, row_states: Sequence[StreamState], row_slots: Sequence[int],
                      tokens: Sequence[int], positions: Sequence[int],
                      logits_rows: Optional[Sequence[int]] = None):
@@ -406,82 +515,14 @@ class OracleDecoder:
         Returns (final hidden before the final norm [R, d], logits [len(logits_rows), V]).
         """
         cfg = self.cfg
-        H, dh = cfg.n_heads, cfg.head_dim
         R = len(tokens)
         for st, sl in zip(row_states, row_slots):
             if not (0 <= sl < st.max_len):
                 raise ValueError(f"cache row {sl} outside [0, {st.max_len})")
-        x = self._embed(tokens, positions)
+        x = self.embed(tokens, positions)
         self._margins = np.full(R, np.inf)
-        for l, L in enumerate(self.W["layers"]):
-            # ---- self-attention block ----
-            h = self._norm(x, L["norm1_w"], L["norm1_b"])
-            if cfg.is_whisper:
-                q = self._proj(h, L["q"], (l, "q"))
-                k = self._proj(h, L["k"], (l, "k"))
-                v = self._proj(h, L["v"], (l, "v"))
-            else:
-                # one quantisation of the normed row shared by q, k, v ([focr] fused q|k|v GEMV)
-                q = self._proj_i8(h, L["q"], (l, "q"))
-                k = self._proj_i8(h, L["k"], (l, "k"))
-                v = self._proj_i8(h, L["v"], (l, "v"))
-                for r in range(R):
-                    c, s = rope_cos_sin(int(positions[r]), cfg.rope_theta, dh)
-                    q[r] = apply_rope_neox(q[r].reshape(H, dh), c, s).reshape(-1)
-                    k[r] = apply_rope_neox(k[r].reshape(H, dh), c, s).reshape(-1)
-            for r in range(R):
-                row_states[r].k[l][row_slots[r]] = k[r]
-                row_states[r].v[l][row_slots[r]] = v[r]
-            ctx = np.empty_like(q)
-            views = {}
-            for r in range(R):
-                st = row_states[r]
-                if id(st) not in views:
-                    top = max(sl for s2, sl in zip(row_states, row_slots) if s2 is st) + 1
-                    views[id(st)] = (
-                        np.ascontiguousarray(st.k[l][:top].astype(F64).reshape(top, H, dh).transpose(1, 0, 2)),
-                        np.ascontiguousarray(st.v[l][:top].astype(F64).reshape(top, H, dh).transpose(1, 0, 2)))
-                kh, vh = views[id(st)]
-                n = row_slots[r] + 1
-                ctx[r] = _attend_heads(q[r].reshape(H, dh).astype(F64), kh[:, :n], vh[:, :n]
-                                       ).astype(F32).reshape(-1)
-            if cfg.is_whisper:
-                x = x + self._proj(ctx, L["o"], (l, "o"))
-            else:
-                x = x + self._proj_i8(ctx, L["o"], (l, "o"))
-            # ---- cross-attention block (whisper) ----
-            if cfg.is_whisper:
-                h = self._norm(x, L["norm2_w"], L["norm2_b"])
-                qx = self._proj(h, L["xq"], (l, "xq"))
-                cx = np.empty_like(qx)
-                xviews = {}
-                ne = cfg.enc_len
-                for r in range(R):
-                    st = row_states[r]
-                    if id(st) not in xviews:
-                        xviews[id(st)] = (
-                            np.ascontiguousarray(st.xk[l].astype(F64).reshape(ne, H, dh).transpose(1, 0, 2)),
-                            np.ascontiguousarray(st.xv[l].astype(F64).reshape(ne, H, dh).transpose(1, 0, 2)))
-                    kh, vh = xviews[id(st)]
-                    cx[r] = _attend_heads(qx[r].reshape(H, dh).astype(F64), kh, vh
-                                          ).astype(F32).reshape(-1)
-                x = x + self._proj(cx, L["xo"], (l, "xo"))
-            # ---- feed-forward block ----
-            if cfg.is_whisper:
-                h = self._norm(x, L["norm3_w"], L["norm3_b"])
-                f = gelu_tanh(self._proj(h, L["fc1"], (l, "fc1")))
-                x = x + self._proj(f, L["fc2"], (l, "fc2"))
-            else:
-                h = self._norm(x, L["norm2_w"], L["norm2_b"])
-                hq, a = self._quant(h)  # shared by gate and up
-                def lin(p, key):
-                    w64 = self._w64(key, p["w"])
-                    y = (hq.astype(F64) @ w64.T) * a.astype(F64)[:, None] * p["s"].astype(F64)[None, :]
-                    return y.astype(F32)
-                g = lin(L["gate"], (l, "gate"))
-                u = lin(L["up"], (l, "up"))
-                m = (silu(g) * u).astype(F32)
-                x = x + self._proj_i8(m, L["down"], (l, "down"))
+        for l in range(cfg.n_layers):
+            x = self.layer_forward(l, x, row_states, row_slots, positions)
         hidden = x
         self.last_margins, self._margins = self._margins, None
         if logits_rows is None:

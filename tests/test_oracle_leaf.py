@@ -302,3 +302,33 @@ def test_argmax_golden_first_max():
     for case in g["cases"]:
         row = np.array([float(v) for v in case["row"]], F32)
         assert oracle.argmax_first(row) == case["argmax"]
+
+
+def test_w8a32_brute_force_with_distinct_row_scales():
+    """y_n = s_n * sum_k q_nk x_k + b_n with a different scale on every output row: a
+    scale taken from the wrong row or applied along the input axis fails."""
+    r = rng(12)
+    q = r.integers(-127, 128, size=(5, 11)).astype(np.int8)
+    s = (r.random(5) + 0.5).astype(F32) * F32(0.01)
+    b = r.standard_normal(5).astype(F32)
+    x = r.standard_normal((3, 11)).astype(F32)
+    y = oracle.linear_w8a32(x, q, s, b)
+    for m in range(3):
+        for n in range(5):
+            ref = float(s[n]) * math.fsum(int(q[n, k]) * float(x[m, k]) for k in range(11)) + float(b[n])
+            assert abs(float(y[m, n]) - ref) <= 1e-6 * max(1.0, abs(ref))
+
+
+def test_linear_with_cached_f64_weights_is_the_same_function():
+    """The decoder passes each matrix's f64 copy (converted once); the result is the same bits."""
+    r = rng(13)
+    w = r.standard_normal((7, 19)).astype(F32)
+    q = r.integers(-127, 128, size=(7, 19)).astype(np.int8)
+    s = r.random(7).astype(F32)
+    b = r.standard_normal(7).astype(F32)
+    x = r.standard_normal((2, 19)).astype(F32)
+    xq, a = oracle.quantize_rows_i8_te(x)
+    assert np.array_equal(oracle.linear_f32(x, w, b), oracle.linear_f32(x, w, b, w64=w.astype(np.float64)))
+    assert np.array_equal(oracle.linear_w8a32(x, q, s, b), oracle.linear_w8a32(x, q, s, b, w64=q.astype(np.float64)))
+    assert np.array_equal(oracle.linear_w8a8(xq, a, q, s, b), oracle.linear_w8a8(xq, a, q, s, b, w64=q.astype(np.float64)))
+    assert np.array_equal(oracle.int8_dot_acc(xq, q), oracle.int8_dot_acc(xq, q, w64=q.astype(np.float64)))

@@ -286,3 +286,105 @@ def test_quant_jitter_is_small_and_off_by_default():
     sa, sc = a.new_state(None), c.new_state(None)
     la, lc = a.prefill(sa, toks), c.prefill(sc, toks)
     assert np.abs(la - lc).max() < 0.05
+
+
+def _scaled_permutation(rng_, n_out, n_in, perm, c):
+    """int8 codes 127 at (n, perm[n]) for n < len(perm), zero elsewhere, with row scales c / 127:
+    the projection computes y_n = c_n x_{perm[n]} exactly in real arithmetic."""
+    w = np.zeros((n_out, n_in), np.int8)
+    for n, k in enumerate(perm):
+        w[n, k] = 127
+    return w, (c.astype(np.float64) / 127.0).astype(F32)
+
+
+def test_permutation_structured_whisper_w8a32_closed_form():
+    """One W8A32 Whisper layer at position 0 whose v, o, xv, xo, fc1, fc2 are scaled
+    permutations with a different scale on every row (q, k, xq, xk zero). With y = c * x[perm]
+    for each of them and the encoder mean m_enc:
+      x1 = x0 + c_o (c_v LN1(x0)[p_v] + b_v)[p_o] + b_o          (one cached row: weight 1)
+      x2 = x1 + c_xo (c_xv m_enc[p_xv] + b_xv)[p_xo] + b_xo        (equal keys: uniform weights)
+      x3 = x2 + c_2 gelu(c_1 LN3(x2)[p_1] + b_1)[p_2] + b_2
+    Built from torch routines only. A row scale applied on the wrong axis or to the wrong row
+    fails, since every permutation here moves every index."""
+    cfg = synth.dataclasses.replace(synth.MODELS["tiny_whisper_w8a32"], n_layers=1)
+    W = synth.make_weights(cfg, 5)
+    W = _zero_projections(W)
+    d, f = cfg.d_model, cfg.d_ff
+    L = W["layers"][0]
+    r = np.random.default_rng(9)
+    perms, scales = {}, {}
+    for key, (n_out, n_in) in {"v": (d, d), "o": (d, d), "xv": (d, d), "xo": (d, d), "fc1": (f, d),
+                               "fc2": (d, f)}.items():
+        m = min(n_out, n_in)
+        perm = np.roll(np.arange(m), 1 + int(r.integers(0, m - 1)))   # a cyclic shift: no fixed point
+        c = (0.5 + r.random(n_out)).astype(F32)
+        L[key]["w"], L[key]["s"] = _scaled_permutation(r, n_out, n_in, perm[: min(n_out, m)], c)
+        perms[key], scales[key] = perm, L[key]["s"].astype(np.float64) * 127.0
+    dec = oracle.OracleDecoder(W, 16)
+    enc = synth.encoder_hidden(cfg, 0, 5)
+    st = dec.new_state(enc)
+    tok = 31
+    hidden, logits = dec.step([st], [tok], [0])
+    T = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))
+    ln = lambda x, g, b: torch.nn.functional.layer_norm(x, (d,), T(g), T(b), eps=float(F32(1e-5)))
+
+    def P(key, x, n_out):
+        y = torch.zeros(n_out, dtype=torch.float64)
+        m = len(perms[key])
+        y[:m] = T(scales[key][:m]) * x[torch.from_numpy(perms[key][:m])]
+        return y
+
+    x0 = T(W["tok_emb"][tok]) + T(W["pos_emb"][0])
+    x1 = x0 + P("o", P("v", ln(x0, L["norm1_w"], L["norm1_b"]), d) + T(L["v"]["b"]), d) + T(L["o"]["b"])
+    x2 = x1 + P("xo", P("xv", T(enc).mean(0), d) + T(L["xv"]["b"]), d) + T(L["xo"]["b"])
+    g = torch.nn.functional.gelu(P("fc1", ln(x2, L["norm3_w"], L["norm3_b"]), f) + T(L["fc1"]["b"]),
+                                 approximate="tanh")
+    x3 = x2 + P("fc2", g, d) + T(L["fc2"]["b"])
+    np.testing.assert_allclose(hidden[0], x3.numpy(), rtol=1e-5, atol=2e-6)
+    ref = T(W["tok_emb"]) @ ln(x3, W["final_w"], W["final_b"])
+    np.testing.assert_allclose(logits[0], ref.numpy(), rtol=1e-4, atol=1e-5)
+
+
+def test_permutation_structured_qwen2_w8a8_closed_form():
+    """One W8A8 Qwen2 layer at position 0 with q, k, v weights zero (every V row is b_v) and
+    o, gate, up, down scaled permutations with a different scale on every row. With the
+    pinned quantiser (q, a) = quant(.) and dequantised products acc * a * s:
+      x1 = x0 + c_o dq(quant(b_v))[p_o]
+      g = c_g dq(quant(h))[p_g], u = c_u dq(quant(h))[p_u] with h = RMS2(x1)
+      x2 = x1 + c_d dq(quant(silu(g) u))[p_d]
+    so each row scale, each permutation and the per-row activation scale are checked."""
+    cfg = synth.dataclasses.replace(synth.MODELS["tiny_qwen2"], n_layers=1)
+    W = synth.make_weights(cfg, 6)
+    W = _zero_projections(W)
+    d, f = cfg.d_model, cfg.d_ff
+    L = W["layers"][0]
+    r = np.random.default_rng(10)
+    perms, cs = {}, {}
+    for key, (n_out, n_in) in {"o": (d, d), "gate": (f, d), "up": (f, d), "down": (d, f)}.items():
+        m = min(n_out, n_in)
+        perm = np.roll(np.arange(m), 1 + int(r.integers(0, m - 1)))
+        c = (0.5 + r.random(n_out)).astype(F32)
+        L[key]["w"], L[key]["s"] = _scaled_permutation(r, n_out, n_in, perm, c)
+        perms[key], cs[key] = perm, L[key]["s"]
+    dec = oracle.OracleDecoder(W, 16)
+    st = dec.new_state(None)
+    tok = 5
+    hidden, _ = dec.step([st], [tok], [0])
+
+    def proj(key, x_row, n_out):
+        """acc * a * s exactly as dequantised: acc_n = 127 q[perm[n]] (zero past the permutation)."""
+        q, a = oracle.quantize_rows_i8_te(x_row[None, :])
+        y = np.zeros(n_out, np.float64)
+        m = len(perms[key])
+        y[:m] = 127.0 * q[0, perms[key]].astype(np.float64) * float(a[0]) * cs[key][:m].astype(np.float64)
+        return y.astype(F32)
+
+    x0 = W["tok_emb"][tok]
+    x1 = (x0 + proj("o", L["v"]["b"], d)).astype(F32)
+    h = torch.nn.functional.rms_norm(torch.from_numpy(x1).double(), (d,), torch.from_numpy(L["norm2_w"]).double(),
+                                     eps=float(F32(1e-6))).numpy().astype(F32)
+    g = proj("gate", h, f)
+    u = proj("up", h, f)
+    m = (torch.nn.functional.silu(torch.from_numpy(g).double()).numpy().astype(F32) * u).astype(F32)
+    x2 = (x1 + proj("down", m, d)).astype(F32)
+    np.testing.assert_allclose(hidden[0], x2, rtol=1e-6, atol=1e-7)
