@@ -96,6 +96,23 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t phase,
     }
 }
 
+// ---- launch attributes --------------------------------------------------------------
+
+// Every kernel of the step prefers the largest shared-memory carveout, so that consecutive
+// kernels never need the SM's L1 / shared-memory split changed between them: a change
+// drains the SM first, which stops a dependent kernel's CTAs from starting early under
+// programmatic dependent launch. Applied once per kernel and device (`attr_dev` is the
+// caller's per-kernel record of the device it was last applied on).
+template <typename K>
+inline cudaError_t prefer_max_shared_once(K kern, int& attr_dev) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || attr_dev == dev) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess) attr_dev = dev;
+    return e;
+}
+
 // ---- programmatic dependent launch -----------------------------------------------
 
 __device__ __forceinline__ void pdl_wait() {

@@ -529,6 +529,9 @@ cudaError_t rowprep_digits_launch(const float* x, int x_ld, const float* gw, con
                                   int rows, long long plane_stride, int8_t* out, float* scale, bool pdl,
                                   cudaStream_t st) {
     if (K % 4 != 0 || rows <= 0) return cudaErrorInvalidValue;
+    thread_local int attr_dev = -1;
+    const cudaError_t e = prefer_max_shared_once(k_rowprep_digits<PRO>, attr_dev);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((rows + 3) / 4);
     cfg.blockDim = dim3(128);
@@ -552,6 +555,9 @@ cudaError_t head_tc_launch_bt(int num_sms, HeadArgs a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     if (attr_dev != dev) {
         e = cudaFuncSetAttribute(k_head_tc<BT, XPRO>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024 - 1024);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(k_head_tc<BT, XPRO>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         attr_dev = dev;
     }

@@ -95,6 +95,9 @@ cudaError_t rowprep_i8_launch(const GemvArgs& g, int8_t* xq, float* xs, cudaStre
 template <int PRO>
 cudaError_t rowprep_i8_launch(const GemvArgs& g, int8_t* xq, float* xs, cudaStream_t st) {
     if (g.K % 16 != 0) return cudaErrorNotSupported;
+    thread_local int attr_dev = -1;
+    const cudaError_t e = prefer_max_shared_once(k_rowprep_i8<PRO>, attr_dev);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((g.B + 3) / 4);
     cfg.blockDim = dim3(128);
