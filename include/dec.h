@@ -221,6 +221,45 @@ dec_status dec_step_host(dec_handle* h, int32_t batch, const int32_t* slots,
                          const int32_t* cache_lens, float* logits_host, int32_t* argmax_host,
                          void* stream);
 
+/*
+ * Each listed slot's greedy continuation token (the argmax of its most recent
+ * dec_prefill last row or dec_step row) into host `tokens` [n]. Synchronises
+ * `stream`; DEC_ESTATE for a slot with no continuation yet, DEC_ETIMEOUT (and
+ * the handle becomes failed) when a bounded device wait gave up.
+ */
+dec_status dec_next_tokens(dec_handle* h, int32_t n, const int32_t* slots, int32_t* tokens, void* stream);
+
+/* The configuration the handle was created with. */
+dec_status dec_get_config(const dec_handle* h, dec_config* out);
+
+/*
+ * Greedy generation for many requests with continuous batching ([focr]
+ * `BatchScheduler::run`, `generate_greedy_batched`). Requests are admitted in
+ * order whenever one of min(max_active, max_slots, DEC_MAX_BATCH) slots is
+ * free: the prompt is prefilled and its last row's argmax is the first token.
+ * Every iteration then advances all admitted streams by one token with one
+ * dec_step. A stream retires after emitting `eos` (which is kept in its
+ * output) or `max_new` tokens, or when its next row would overflow the cache
+ * or the position range; its slot is refilled from the queue before the next
+ * step. A stream's tokens are those it would get alone (the step's per-stream
+ * arithmetic does not depend on the batch).
+ *   reqs        host [n_reqs]; prompt host int32 [n_prompt] (n_prompt >= 1);
+ *               enc_hidden device f32 [enc_len, d] for whisper, NULL for qwen2
+ *   tokens_out  host int32 [n_reqs, stride]: request r's tokens in row r
+ *   n_out       host int32 [n_reqs]: tokens written per request
+ * Synchronises `stream` once per step. Uses (and overwrites) slots
+ * 0..min(max_active, max_slots) - 1 of the handle.
+ */
+typedef struct dec_request {
+    const int32_t* prompt;
+    int32_t n_prompt;
+    int32_t max_new;
+    int32_t eos;               /* stop token, or -1 for none */
+    const float* enc_hidden;
+} dec_request;
+dec_status dec_generate(dec_handle* h, const dec_request* reqs, int32_t n_reqs, int32_t max_active,
+                        int32_t* tokens_out, int32_t stride, int32_t* n_out, void* stream);
+
 /* Current length (cached rows) of `slot` as tracked by the handle. */
 dec_status dec_slot_len(const dec_handle* h, int32_t slot, int32_t* len);
 
@@ -236,9 +275,57 @@ dec_status dec_kv_read(dec_handle* h, int32_t slot, int32_t layer, int32_t start
  * (before the final norm), f32 [batch, d_model], into device `out`. */
 dec_status dec_hidden(dec_handle* h, float* out, int32_t batch, void* stream);
 
-/* Synchronise `stream` and report device-side failures (DEC_ETIMEOUT when a
- * bounded wait inside a kernel gave up). Clears the device status word. */
+/*
+ * Parity bisection ([wa-dec] `forward_traced`: per-layer hidden states for
+ * comparison against a reference). While `buf` is not NULL, every dec_step /
+ * dec_step_host also copies the residual stream leaving each layer (after its
+ * FFN residual add, before the next layer's norm) into device `buf` as f32
+ * [n_layers, batch, d_model] for that step's batch; `buf` must hold
+ * n_layers * batch * d_model floats for every later step's batch (the caller
+ * owns it; it must stay valid while set). NULL turns tracing off. Traced steps
+ * run as their own captured graphs (one extra device-to-device copy per layer).
+ */
+dec_status dec_set_layer_trace(dec_handle* h, float* buf);
+
+/*
+ * Synchronise `stream` and report device-side failures: DEC_ETIMEOUT when a
+ * bounded wait inside one of the handle's kernels gave up (a copy that never
+ * landed; lattice-inference-style fail-closed reporting instead of a hang). The
+ * kernel that gave up returned early, so that step's results are not valid.
+ * From then on the handle is failed: dec_step, dec_step_host, dec_prefill and
+ * dec_kv_append return DEC_ETIMEOUT without queueing work until dec_reset.
+ * dec_step_host checks the status word itself (it synchronises anyway).
+ */
 dec_status dec_sync(dec_handle* h, void* stream);
+
+/*
+ * Recover a failed handle: synchronise the device, clear the status word and
+ * every arrival counter and argmax key the kernels share across launches, and
+ * empty every slot (its cache contents are no longer trusted; prefill or
+ * dec_kv_append it again). The wait limit and the weights are kept.
+ */
+dec_status dec_reset(dec_handle* h);
+
+/*
+ * Limit of every bounded device wait of this handle's kernels, in nanoseconds
+ * (0: the default of one second). Synchronous (writes the handle's status block).
+ */
+dec_status dec_set_wait_limit(dec_handle* h, uint64_t ns);
+
+/*
+ * Test hooks for the failure path; no fault is ever raised on the device.
+ *   dec_debug_inject(h, DEC_INJECT_DROP_ATTN_COPY, 1): in every later step the
+ *     first self-attention CTA of layer 0 announces its first K/V tile on its
+ *     mbarrier but issues no copy, so its bounded wait runs out (after the
+ *     handle's wait limit) and the step reports DEC_ETIMEOUT; such steps run
+ *     without CUDA-graph capture. Value 0 switches it off.
+ *   dec_debug_fail_alloc(n): the n-th device or pinned-host allocation made by
+ *     the next dec_create on the calling thread fails, which must return
+ *     DEC_ENOMEM with everything already allocated freed; 0 switches it off.
+ */
+enum { DEC_INJECT_DROP_ATTN_COPY = 1 };
+dec_status dec_debug_inject(dec_handle* h, int32_t what, int32_t value);
+void dec_debug_fail_alloc(int32_t nth);
 
 /* Number of kernels one step of the most recent dec_step / dec_step_host call
  * launches (the kernel nodes of its captured CUDA graph), or -1 when that step's

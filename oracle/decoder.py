@@ -328,7 +328,8 @@ class OracleDecoder:
         # numbered in call order within one layer (qwen2: 0 the q|k|v input, 1 the o input,
         # 2 the gate/up input, 3 the down input). `tie_log`, when a list, receives
         # (site, row, col, distance) for every activation whose x * inv lies within
-        # `tie_eps` code units of a rounding boundary; `flips` maps site -> [(row, col)] of
+        # `tie_eps` code units (a number, or a dict site -> number) of a rounding
+        # boundary; `flips` maps site -> [(row, col)] of
         # activations to round to the other neighbouring integer instead (a correct
         # implementation whose value sat on the other side of the tie).
         self.tie_log: Optional[list] = None
@@ -375,7 +376,8 @@ class OracleDecoder:
             if self._margins is not None:
                 self._margins = np.minimum(self._margins, dist.min(axis=1))
             if self.tie_log is not None:
-                for r, c in zip(*np.nonzero(dist < self.tie_eps)):
+                eps = self.tie_eps.get(site, 0.0) if isinstance(self.tie_eps, dict) else self.tie_eps
+                for r, c in zip(*np.nonzero(dist < eps)):
                     self.tie_log.append((site, int(r), int(c), float(dist[r, c])))
             if self.flips and site in self.flips:
                 q = q.copy()

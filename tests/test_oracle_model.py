@@ -388,3 +388,24 @@ def test_permutation_structured_qwen2_w8a8_closed_form():
     m = (torch.nn.functional.silu(torch.from_numpy(g).double()).numpy().astype(F32) * u).astype(F32)
     x2 = (x1 + proj("down", m, d)).astype(F32)
     np.testing.assert_allclose(hidden[0], x2, rtol=1e-6, atol=1e-7)
+
+
+def test_tie_log_and_flips():
+    """The quantiser's tie bookkeeping: an activation within tie_eps of a rounding boundary is
+    logged with its site, row, column and distance, and a flip rounds exactly that activation
+    to the other neighbouring integer and changes nothing else."""
+    cfg, W = _model("tiny_qwen2")
+    dec = oracle.OracleDecoder(W, 8)
+    x = np.array([[127.0, 2.5, 1.0, -3.4999], [127.0, 2.25, 1.0, 0.0]], F32)
+    dec.tie_log, dec.tie_eps = [], {0: 1e-3}
+    dec._site = 0
+    q0, a0 = dec._quant(x)
+    assert [(s, r, c) for s, r, c, _ in dec.tie_log] == [(0, 0, 1), (0, 0, 3)]
+    dec.tie_log, dec.flips = None, {1: [(0, 1), (0, 3)]}
+    dec._site = 1
+    q1, a1 = dec._quant(x)
+    assert np.array_equal(a0, a1)
+    assert int(q1[0, 1]) == 3 and int(q0[0, 1]) == 2     # 2.5 rounds to even 2; flipped to 3
+    assert int(q1[0, 3]) == -4 and int(q0[0, 3]) == -3   # -3.4999 rounds to -3; flipped to -4
+    diff = q1.astype(int) != q0.astype(int)
+    assert int(diff.sum()) == 2

@@ -24,10 +24,13 @@ PROJ = {"f32": 0, "w8a8": 1, "w8a32": 2}
 
 # Every symbol include/dec.h declares.
 EXPORTS = ["dec_create", "dec_destroy", "dec_last_error", "dec_prefill", "dec_kv_append", "dec_step",
-           "dec_step_host", "dec_slot_len", "dec_kv_read", "dec_hidden", "dec_sync", "dec_step_kernels",
+           "dec_step_host", "dec_slot_len", "dec_kv_read", "dec_hidden", "dec_set_layer_trace", "dec_sync",
+           "dec_reset", "dec_set_wait_limit", "dec_debug_inject", "dec_debug_fail_alloc", "dec_step_kernels",
+           "dec_next_tokens", "dec_get_config", "dec_generate",
            "dec_attention_workspace_size", "dec_attention", "dec_attention_plan", "dec_attention_noalloc",
            "dec_i8_dot"]
 I8_PATH = {"dp4a": 0, "tcgen05": 1}
+DEC_INJECT_DROP_ATTN_COPY = 1
 
 
 class DecError(RuntimeError):
@@ -59,6 +62,11 @@ class DecLayerWeights(C.Structure):
                 ("gate", DecProj), ("up", DecProj), ("down", DecProj)]
 
 
+class DecRequest(C.Structure):
+    _fields_ = [("prompt", C.POINTER(C.c_int32)), ("n_prompt", C.c_int32), ("max_new", C.c_int32),
+                ("eos", C.c_int32), ("enc_hidden", C.c_void_p)]
+
+
 class DecWeights(C.Structure):
     _fields_ = [("tok_emb", C.c_void_p), ("pos_emb", C.c_void_p), ("final_w", C.c_void_p),
                 ("final_b", C.c_void_p), ("layers", C.POINTER(DecLayerWeights))]
@@ -81,7 +89,15 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
         "dec_slot_len": (C.c_int, [vp, i32, pi32]),
         "dec_kv_read": (C.c_int, [vp, i32, i32, i32, i32, vp, vp, vp]),
         "dec_hidden": (C.c_int, [vp, vp, i32, vp]),
+        "dec_set_layer_trace": (C.c_int, [vp, vp]),
         "dec_sync": (C.c_int, [vp, vp]),
+        "dec_reset": (C.c_int, [vp]),
+        "dec_next_tokens": (C.c_int, [vp, i32, pi32, pi32, vp]),
+        "dec_get_config": (C.c_int, [vp, C.POINTER(DecConfig)]),
+        "dec_generate": (C.c_int, [vp, C.POINTER(DecRequest), i32, i32, pi32, i32, pi32, vp]),
+        "dec_set_wait_limit": (C.c_int, [vp, C.c_uint64]),
+        "dec_debug_inject": (C.c_int, [vp, i32, i32]),
+        "dec_debug_fail_alloc": (None, [i32]),
         "dec_step_kernels": (C.c_int, [vp, pi32]),
         "dec_attention_workspace_size": (C.c_size_t, [i32, i32, i32]),
         "dec_attention": (C.c_int, [vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, C.c_size_t, vp]),
@@ -218,6 +234,11 @@ class Decoder:
     def hidden(self, out, batch: int, stream: int = 0):
         self._check(self._lib.dec_hidden(self._h, _ptr(out), batch, stream))
 
+    def set_layer_trace(self, buf):
+        """Device buffer f32 [n_layers, batch, d_model] for the residual leaving each layer
+        of every later step (None turns tracing off)."""
+        self._check(self._lib.dec_set_layer_trace(self._h, _ptr(buf)))
+
     def sync(self, stream: int = 0):
         self._check(self._lib.dec_sync(self._h, stream))
 
@@ -227,11 +248,49 @@ class Decoder:
         self._check(self._lib.dec_attention_plan(self._h, 1 if cross else 0, C.byref(n)))
         return int(n.value)
 
+    def next_tokens(self, slots, stream: int = 0):
+        """Each slot's greedy continuation token (host list)."""
+        out = (C.c_int32 * len(slots))()
+        self._check(self._lib.dec_next_tokens(self._h, len(slots), _i32arr(slots), out, stream))
+        return list(out)
+
+    def generate(self, requests, max_active: int, stream: int = 0):
+        """Greedy generation with continuous batching. requests: list of dicts with
+        'prompt' (token ids), 'max_new', optional 'eos' (-1) and 'enc_hidden' (device
+        tensor, whisper). Returns one list of token ids per request."""
+        n = len(requests)
+        keep = []
+        arr = (DecRequest * max(1, n))()
+        stride = max([int(r["max_new"]) for r in requests] + [1])
+        for i, r in enumerate(requests):
+            p = _i32arr(r["prompt"])
+            keep.append(p)
+            arr[i] = DecRequest(C.cast(p, C.POINTER(C.c_int32)), len(r["prompt"]), int(r["max_new"]),
+                                int(r.get("eos", -1)), _ptr(r.get("enc_hidden")))
+        toks = (C.c_int32 * (max(1, n) * stride))()
+        lens = (C.c_int32 * max(1, n))()
+        self._check(self._lib.dec_generate(self._h, arr, n, max_active, toks, stride, lens, stream))
+        return [list(toks[i * stride: i * stride + lens[i]]) for i in range(n)]
+
+    def reset(self):
+        self._check(self._lib.dec_reset(self._h))
+
+    def set_wait_limit(self, ns: int):
+        self._check(self._lib.dec_set_wait_limit(self._h, int(ns)))
+
+    def debug_inject(self, what: int, value: int):
+        self._check(self._lib.dec_debug_inject(self._h, what, value))
+
     def step_kernels(self) -> int:
         """Kernels launched by one step of the most recent step call (-1: not captured)."""
         n = C.c_int32(0)
         self._check(self._lib.dec_step_kernels(self._h, C.byref(n)))
         return int(n.value)
+
+
+def debug_fail_alloc(nth: int):
+    """The nth allocation of the next Decoder created on this thread fails (0: off)."""
+    lib().dec_debug_fail_alloc(int(nth))
 
 
 def _raise_thread_error(st: int):

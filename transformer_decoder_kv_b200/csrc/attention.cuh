@@ -51,13 +51,17 @@ struct AttnArgs {
     int tps;               // 64-key tiles per split; 0: ceil(tiles / S) per row
     int stages;            // shared-memory pipeline stages (1..3); 0: 3
     int* err;              // device status word
+    int drop_first_copy;   // test hook: CTA (0, 0, 0) never issues its first tile's copies
 };
 
+// `drop`: announce the bytes but issue no copy, so that the tile's wait can only run out
+// (the host-side fault injection of the failure-path tests; no memory is touched).
 __device__ __forceinline__ void attn_issue(float* sK, float* sV, uint64_t* bar, const float* Kb,
-                                           const float* Vb, int tile, int n) {
+                                           const float* Vb, int tile, int n, bool drop = false) {
     const int rows = min(kAttnTile, n - tile * kAttnTile);
     const uint32_t bytes = static_cast<uint32_t>(rows) * kHeadDim * sizeof(float);
     mbar_arrive_expect_tx(bar, 2 * bytes);
+    if (drop) return;
     bulk_g2s(sK, Kb + static_cast<long long>(tile) * kAttnTile * kHeadDim, bytes, bar);
     bulk_g2s(sV, Vb + static_cast<long long>(tile) * kAttnTile * kHeadDim, bytes, bar);
 }
@@ -113,12 +117,13 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
     // before the dependency wait
     const int first_new_tile = (a.mode == ATTN_SELF) ? (n - 1) / kAttnTile : ntiles;
     int pre = 0;
+    const bool drop = a.drop_first_copy && s == 0 && h == 0 && b == 0;
     if (tid == 0) {
         for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
         for (; pre < NS && t0 + pre < t1 && t0 + pre < first_new_tile; ++pre)
             attn_issue(sK + pre * kAttnTile * kHeadDim, sV + pre * kAttnTile * kHeadDim, &bars[pre], Kb,
-                       Vb, t0 + pre, n);
+                       Vb, t0 + pre, n, drop && pre == 0);
     }
     pdl_launch_dependents();
     if (a.mode != ATTN_OP) pdl_wait();
@@ -126,7 +131,7 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
     if (tid == 0) {
         for (int i = pre; i < NS && t0 + i < t1; ++i)
             attn_issue(sK + i * kAttnTile * kHeadDim, sV + i * kAttnTile * kHeadDim, &bars[i], Kb,
-                       Vb, t0 + i, n);
+                       Vb, t0 + i, n, drop && i == 0);
     }
     __syncthreads();
 

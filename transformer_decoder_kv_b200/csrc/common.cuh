@@ -82,14 +82,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
     return ok != 0;
 }
 
-// Wait for phase `phase` of `bar`, giving up after kWaitLimitNs. On give-up the
-// device status word gets DEC_DEVERR_TIMEOUT and false is returned.
+// Device status block of a handle: word 0 is the status (DEC_DEVERR_* bits), words 2-3 the
+// wait limit in nanoseconds as an unsigned 64-bit value (0: kWaitLimitNs).
+constexpr int kStatusWords = 4;
+
+__device__ __forceinline__ unsigned long long wait_limit_ns(const int* err) {
+    if (err == nullptr) return kWaitLimitNs;
+    const unsigned long long v = *reinterpret_cast<const volatile unsigned long long*>(err + 2);
+    return v ? v : kWaitLimitNs;
+}
+
+// Wait for phase `phase` of `bar`, giving up after the status block's wait limit (kWaitLimitNs
+// without one). On give-up the status word gets DEC_DEVERR_TIMEOUT and false is returned.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t phase, int* err) {
     if (mbar_try_wait(bar, phase)) return true;
     const unsigned long long t0 = global_ns();
+    const unsigned long long limit = wait_limit_ns(err);
     while (true) {
         if (mbar_try_wait(bar, phase)) return true;
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > limit) {
             if (err) atomicOr(err, DEC_DEVERR_TIMEOUT);
             return false;
         }

@@ -36,6 +36,10 @@ constexpr int kMetaRing = 8;
 constexpr int kMaxSplits = kAttnMaxSplits;
 
 thread_local std::string g_create_error;
+// Allocation-failure injection for tests (dec_debug_fail_alloc): the n-th allocation of the
+// next dec_create on this thread fails; 0 disables.
+thread_local int g_fail_alloc_at = 0;
+thread_local int g_alloc_count = 0;
 
 }  // namespace
 
@@ -108,6 +112,11 @@ struct dec_handle {
     int* head_counter = nullptr;
     int* last_tok = nullptr;
     int* dev_err = nullptr;
+    int* host_status = nullptr;     // pinned copy of the status word after dec_step_host
+    int* host_tok = nullptr;        // pinned copy of every slot's greedy continuation token
+    bool failed = false;            // a bounded device wait gave up; dec_reset required
+    int inject_drop = 0;            // test hook: drop one attention tile copy per step
+    int mma_cnt_bytes = 0;
     StepMeta* dmeta = nullptr;
     StepMeta* hmeta[kMetaRing] = {};
     cudaEvent_t hev[kMetaRing] = {};
@@ -123,7 +132,8 @@ struct dec_handle {
         cudaGraphExec_t exec;
         int kernels;   // kernel launches in one step of this key (-1: not captured)
     };
-    std::map<std::array<long long, 4>, StepGraph> graphs;
+    std::map<std::array<long long, 5>, StepGraph> graphs;
+    float* trace = nullptr;          // per-layer residual copies [L, B, d], or null
     int last_step_kernels = -1;
     cudaStream_t cap_stream = nullptr;
     float* stage_logits = nullptr;   // dec_step_host result staging
@@ -151,10 +161,15 @@ dec_status cuda_fail(dec_handle* h, cudaError_t e, const char* what) {
         if (e_ != cudaSuccess) return cuda_fail((h), e_, #call); \
     } while (0)
 
+// The allocation-failure hook: true when this allocation is the one asked to fail.
+bool injected_alloc_failure() { return g_fail_alloc_at > 0 && ++g_alloc_count == g_fail_alloc_at; }
+
 template <typename T>
 dec_status dalloc(dec_handle* h, T** p, size_t bytes) {
     void* q = nullptr;
     if (bytes == 0) bytes = 16;
+    if (injected_alloc_failure())
+        return fail(h, DEC_ENOMEM, "cudaMalloc of " + std::to_string(bytes) + " bytes failed (injected)");
     cudaError_t e = cudaMalloc(&q, bytes);
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -525,7 +540,9 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
         at.part = h->part;
         at.counters = h->counters;
         at.err = h->dev_err;
+        at.drop_first_copy = (l == 0) ? h->inject_drop : 0;
         DEC_TRY(attention(h, at, B, max_len_plus1, h->tps_self, st));
+        at.drop_first_copy = 0;
         // ---- output projection + residual ----
         g = base_args(h, B);
         g.x = h->ctx;
@@ -627,6 +644,9 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             g.out_ld = d;
             DEC_TRY((gemv_qwen<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, L.m_2, st)));
         }
+        if (h->trace)
+            DEC_CUDA(h, cudaMemcpyAsync(h->trace + static_cast<size_t>(l) * B * d, h->x, size_t(B) * d * 4,
+                                        cudaMemcpyDeviceToDevice, st));
     }
     // ---- final norm + tied head + greedy argmax ----
     GemvArgs g = base_args(h, B);
@@ -659,6 +679,13 @@ dec_status upload_meta(dec_handle* h, const StepMeta& m, cudaStream_t st) {
     std::memcpy(h->hmeta[i], &m, sizeof(StepMeta));
     DEC_CUDA(h, cudaMemcpyAsync(h->dmeta, h->hmeta[i], sizeof(StepMeta), cudaMemcpyHostToDevice, st));
     DEC_CUDA(h, cudaEventRecord(h->hev[i], st));
+    return DEC_OK;
+}
+
+// Entry points that queue work refuse it after a bounded device wait gave up, until dec_reset.
+dec_status check_not_failed(dec_handle* h) {
+    if (h->failed)
+        return fail(h, DEC_ETIMEOUT, "a bounded device wait gave up in an earlier call; call dec_reset first");
     return DEC_OK;
 }
 
@@ -711,7 +738,7 @@ dec_status validate_step(dec_handle* h, int B, const int32_t* slots, const int32
 
 // Record the step's launch sequence into a graph for later identical steps. Capture
 // problems are not errors: the key is marked and such steps keep running eagerly.
-void capture_step(dec_handle* h, const std::array<long long, 4>& key, int B, int max_len, float* logits,
+void capture_step(dec_handle* h, const std::array<long long, 5>& key, int B, int max_len, float* logits,
                   int* argmax) {
     if (h->graphs.size() >= 256) {
         for (auto& kv : h->graphs)
@@ -749,16 +776,22 @@ void capture_step(dec_handle* h, const std::array<long long, 4>& key, int B, int
 dec_status step_validated(dec_handle* h, const StepMeta& m, int max_len, float* logits, int* argmax,
                           cudaStream_t st) {
     DEC_TRY(upload_meta(h, m, st));
-    const std::array<long long, 4> key = {m.B, (max_len + kAttnTile - 1) / kAttnTile,
-                                          reinterpret_cast<long long>(logits), reinterpret_cast<long long>(argmax)};
+    const std::array<long long, 5> key = {m.B, (max_len + kAttnTile - 1) / kAttnTile,
+                                          reinterpret_cast<long long>(logits), reinterpret_cast<long long>(argmax),
+                                          reinterpret_cast<long long>(h->trace)};
     auto it = h->graphs.find(key);
-    if (it != h->graphs.end() && it->second.exec != nullptr) {
+    if (h->inject_drop) {
+        // fault-injection steps run eagerly and are never captured
+        DEC_TRY(run_step(h, m.B, max_len, logits, argmax, st));
+        h->last_step_kernels = -1;
+    } else if (it != h->graphs.end() && it->second.exec != nullptr) {
         DEC_CUDA(h, cudaGraphLaunch(it->second.exec, st));
+        h->last_step_kernels = it->second.kernels;
     } else {
         DEC_TRY(run_step(h, m.B, max_len, logits, argmax, st));
         if (it == h->graphs.end()) capture_step(h, key, m.B, max_len, logits, argmax);
+        h->last_step_kernels = h->graphs[key].kernels;
     }
-    h->last_step_kernels = h->graphs[key].kernels;
     for (int b = 0; b < m.B; ++b) {
         h->slot_len[m.slot[b]] += 1;
         h->has_tok[m.slot[b]] = 1;
@@ -956,6 +989,7 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
         h->mma_part_bytes = pb;
         DEC_TRY(dalloc(h, &h->mma_cnt, size_t(cl) * 4));
         DEC_CUDA(h, cudaMemset(h->mma_cnt, 0, size_t(cl) * 4));
+        h->mma_cnt_bytes = cl * 4;
         h->mma_cnt_len = cl;
     }
     DEC_TRY(dalloc(h, &h->keys, size_t(MB) * 8));
@@ -964,20 +998,33 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
     DEC_CUDA(h, cudaMemset(h->head_counter, 0, 16));
     DEC_TRY(dalloc(h, &h->last_tok, size_t(c.max_slots) * 4));
     DEC_CUDA(h, cudaMemset(h->last_tok, 0, size_t(c.max_slots) * 4));
-    DEC_TRY(dalloc(h, &h->dev_err, 16));
-    DEC_CUDA(h, cudaMemset(h->dev_err, 0, 16));
+    DEC_TRY(dalloc(h, &h->dev_err, kStatusWords * 4));
+    DEC_CUDA(h, cudaMemset(h->dev_err, 0, kStatusWords * 4));
     DEC_TRY(dalloc(h, &h->dmeta, sizeof(StepMeta)));
     DEC_TRY(dalloc(h, &h->stage_logits, size_t(MB) * c.vocab * 4));
     DEC_TRY(dalloc(h, &h->stage_argmax, size_t(MB) * 4));
-    for (int i = 0; i < kMetaRing; ++i) {
-        void* p = nullptr;
-        if (cudaMallocHost(&p, sizeof(StepMeta)) != cudaSuccess) {
+    auto halloc = [&](void** p, size_t bytes) {
+        if (injected_alloc_failure()) return fail(h, DEC_ENOMEM, "cudaMallocHost failed (injected)");
+        if (cudaMallocHost(p, bytes) != cudaSuccess) {
             cudaGetLastError();
             return fail(h, DEC_ENOMEM, "cudaMallocHost failed");
         }
-        h->hallocs.push_back(p);
+        h->hallocs.push_back(*p);
+        return DEC_OK;
+    };
+    for (int i = 0; i < kMetaRing; ++i) {
+        void* p = nullptr;
+        DEC_TRY(halloc(&p, sizeof(StepMeta)));
         h->hmeta[i] = static_cast<StepMeta*>(p);
         DEC_CUDA(h, cudaEventCreateWithFlags(&h->hev[i], cudaEventDisableTiming));
+    }
+    {
+        void* p = nullptr;
+        DEC_TRY(halloc(&p, 16));
+        h->host_status = static_cast<int*>(p);
+        *h->host_status = 0;
+        DEC_TRY(halloc(&p, size_t(c.max_slots) * 4));
+        h->host_tok = static_cast<int*>(p);
     }
     DEC_CUDA(h, cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking));
     h->slot_len.assign(c.max_slots, 0);
@@ -996,7 +1043,9 @@ dec_status dec_create(const dec_config* cfg, const dec_weights* w, dec_handle** 
     if (st != DEC_OK) return st;
     dec_handle* h = new dec_handle();
     h->cfg = *cfg;
+    g_alloc_count = 0;
     st = create_impl(h, cfg, w);
+    g_fail_alloc_at = 0;   // the hook covers one dec_create
     if (st != DEC_OK) {
         g_create_error = h->err;
         dec_destroy(h);
@@ -1009,6 +1058,7 @@ dec_status dec_create(const dec_config* cfg, const dec_weights* w, dec_handle** 
 dec_status dec_prefill(dec_handle* h, int32_t slot, const int32_t* tokens, int32_t n_tokens,
                        const float* enc_hidden, float* last_logits, void* stream) {
     if (!h) return DEC_EINVAL;
+    DEC_TRY(check_not_failed(h));
     const dec_config& c = h->cfg;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (slot < 0 || slot >= c.max_slots) return fail(h, DEC_EINVAL, "slot out of range");
@@ -1059,6 +1109,7 @@ dec_status dec_prefill(dec_handle* h, int32_t slot, const int32_t* tokens, int32
 dec_status dec_kv_append(dec_handle* h, int32_t slot, int32_t start_pos, int32_t n_rows, const float* k,
                          const float* v, void* stream) {
     if (!h) return DEC_EINVAL;
+    DEC_TRY(check_not_failed(h));
     const dec_config& c = h->cfg;
     if (slot < 0 || slot >= c.max_slots) return fail(h, DEC_EINVAL, "slot out of range");
     if (n_rows < 0 || (n_rows > 0 && (!k || !v))) return fail(h, DEC_EINVAL, "bad rows");
@@ -1104,6 +1155,7 @@ dec_status dec_step(dec_handle* h, int32_t batch, const int32_t* slots, const in
                     const int32_t* positions, const int32_t* cache_lens, float* logits, int32_t* argmax,
                     void* stream) {
     if (!h) return DEC_EINVAL;
+    DEC_TRY(check_not_failed(h));
     StepMeta m{};
     int max_len = 0;
     DEC_TRY(validate_step(h, batch, slots, tokens, positions, cache_lens, m, max_len));
@@ -1115,6 +1167,7 @@ dec_status dec_step_host(dec_handle* h, int32_t batch, const int32_t* slots, con
                          const int32_t* positions, const int32_t* cache_lens, float* logits_host,
                          int32_t* argmax_host, void* stream) {
     if (!h) return DEC_EINVAL;
+    DEC_TRY(check_not_failed(h));
     StepMeta m{};
     int max_len = 0;
     DEC_TRY(validate_step(h, batch, slots, tokens, positions, cache_lens, m, max_len));
@@ -1127,7 +1180,12 @@ dec_status dec_step_host(dec_handle* h, int32_t batch, const int32_t* slots, con
                                     cudaMemcpyDeviceToHost, st));
     if (argmax_host)
         DEC_CUDA(h, cudaMemcpyAsync(argmax_host, h->stage_argmax, size_t(batch) * 4, cudaMemcpyDeviceToHost, st));
+    DEC_CUDA(h, cudaMemcpyAsync(h->host_status, h->dev_err, 4, cudaMemcpyDeviceToHost, st));
     DEC_CUDA(h, cudaStreamSynchronize(st));
+    if (*h->host_status) {
+        h->failed = true;
+        return fail(h, DEC_ETIMEOUT, "a bounded device wait gave up during this step; its results are not valid");
+    }
     return DEC_OK;
 }
 
@@ -1137,11 +1195,45 @@ dec_status dec_slot_len(const dec_handle* h, int32_t slot, int32_t* len) {
     return DEC_OK;
 }
 
+dec_status dec_next_tokens(dec_handle* h, int32_t n, const int32_t* slots, int32_t* tokens, void* stream) {
+    if (!h) return fail(nullptr, DEC_EINVAL, "dec_next_tokens: null handle");
+    if (n < 0 || (n > 0 && (!slots || !tokens))) return fail(h, DEC_EINVAL, "dec_next_tokens: bad arguments");
+    for (int i = 0; i < n; ++i) {
+        if (slots[i] < 0 || slots[i] >= h->cfg.max_slots) return fail(h, DEC_EINVAL, "dec_next_tokens: slot out of range");
+        if (!h->has_tok[slots[i]])
+            return fail(h, DEC_ESTATE, "slot " + std::to_string(slots[i]) + " has no greedy continuation yet");
+    }
+    DEC_TRY(check_device(h));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    DEC_CUDA(h, cudaMemcpyAsync(h->host_tok, h->last_tok, size_t(h->cfg.max_slots) * 4, cudaMemcpyDeviceToHost, st));
+    DEC_CUDA(h, cudaMemcpyAsync(h->host_status, h->dev_err, 4, cudaMemcpyDeviceToHost, st));
+    DEC_CUDA(h, cudaStreamSynchronize(st));
+    if (*h->host_status) {
+        h->failed = true;
+        return fail(h, DEC_ETIMEOUT, "a bounded device wait gave up; the tokens are not valid");
+    }
+    for (int i = 0; i < n; ++i) tokens[i] = h->host_tok[slots[i]];
+    return DEC_OK;
+}
+
+dec_status dec_get_config(const dec_handle* h, dec_config* out) {
+    if (!h || !out) return fail(nullptr, DEC_EINVAL, "dec_get_config: null pointer");
+    *out = h->cfg;
+    return DEC_OK;
+}
+
 dec_status dec_hidden(dec_handle* h, float* out, int32_t batch, void* stream) {
     if (!h) return DEC_EINVAL;
     if (!out || batch < 1 || batch > h->last_batch) return fail(h, DEC_EINVAL, "bad output or batch");
     DEC_CUDA(h, cudaMemcpyAsync(out, h->x, size_t(batch) * h->cfg.d_model * 4, cudaMemcpyDeviceToDevice,
                                 static_cast<cudaStream_t>(stream)));
+    return DEC_OK;
+}
+
+dec_status dec_set_layer_trace(dec_handle* h, float* buf) {
+    if (!h) return fail(nullptr, DEC_EINVAL, "dec_set_layer_trace: null handle");
+    if (buf && (reinterpret_cast<uintptr_t>(buf) & 3)) return fail(h, DEC_EINVAL, "trace buffer must be 4-byte aligned");
+    h->trace = buf;
     return DEC_OK;
 }
 
@@ -1157,11 +1249,48 @@ dec_status dec_sync(dec_handle* h, void* stream) {
     DEC_CUDA(h, cudaStreamSynchronize(st));
     int e = 0;
     DEC_CUDA(h, cudaMemcpy(&e, h->dev_err, 4, cudaMemcpyDeviceToHost));
-    if (e) {
-        DEC_CUDA(h, cudaMemset(h->dev_err, 0, 4));
-        return fail(h, DEC_ETIMEOUT, "a bounded device wait gave up");
-    }
+    if (e) h->failed = true;
+    if (h->failed) return fail(h, DEC_ETIMEOUT, "a bounded device wait gave up; call dec_reset before more work");
     return DEC_OK;
+}
+
+dec_status dec_reset(dec_handle* h) {
+    if (!h) return fail(nullptr, DEC_EINVAL, "dec_reset: null handle");
+    DEC_TRY(check_device(h));
+    // every kernel of the handle has ended before the counters are cleared
+    DEC_CUDA(h, cudaDeviceSynchronize());
+    const int MB = h->max_batch, H = h->cfg.n_heads;
+    DEC_CUDA(h, cudaMemset(h->counters, 0, size_t(MB) * H * 4));
+    if (h->mma_cnt) DEC_CUDA(h, cudaMemset(h->mma_cnt, 0, size_t(h->mma_cnt_bytes)));
+    DEC_CUDA(h, cudaMemset(h->head_counter, 0, 16));
+    DEC_CUDA(h, cudaMemset(h->keys, 0, size_t(MB) * 8));
+    DEC_CUDA(h, cudaMemset(h->dev_err, 0, 4));   // the status word; the wait limit stays
+    DEC_CUDA(h, cudaDeviceSynchronize());
+    std::fill(h->slot_len.begin(), h->slot_len.end(), 0);
+    std::fill(h->has_tok.begin(), h->has_tok.end(), 0);
+    std::fill(h->has_cross.begin(), h->has_cross.end(), 0);
+    h->failed = false;
+    return DEC_OK;
+}
+
+dec_status dec_set_wait_limit(dec_handle* h, uint64_t ns) {
+    if (!h) return fail(nullptr, DEC_EINVAL, "dec_set_wait_limit: null handle");
+    DEC_TRY(check_device(h));
+    const unsigned long long v = ns;
+    DEC_CUDA(h, cudaMemcpy(h->dev_err + 2, &v, sizeof(v), cudaMemcpyHostToDevice));
+    return DEC_OK;
+}
+
+dec_status dec_debug_inject(dec_handle* h, int32_t what, int32_t value) {
+    if (!h) return fail(nullptr, DEC_EINVAL, "dec_debug_inject: null handle");
+    if (what != DEC_INJECT_DROP_ATTN_COPY) return fail(h, DEC_EINVAL, "dec_debug_inject: unknown injection");
+    h->inject_drop = value ? 1 : 0;
+    return DEC_OK;
+}
+
+void dec_debug_fail_alloc(int32_t nth) {
+    g_fail_alloc_at = nth > 0 ? nth : 0;
+    g_alloc_count = 0;
 }
 
 size_t dec_attention_workspace_size(int32_t batch, int32_t n_heads, int32_t ld) {
