@@ -166,8 +166,11 @@ const char* dec_last_error(const dec_handle* h);
 /*
  * Reset stream `slot` and run `n_tokens` tokens (host int32) at positions
  * 0..n_tokens-1 through the decoder, filling its self-attention cache
- * ([focr] `forward_prefill_seed` seeds the cache; here each row goes through
- * the m = 1 step). Whisper: `enc_hidden` (device f32 [enc_len, d]) is
+ * ([focr] `forward_prefill_seed`: the prompt in one forward that seeds the
+ * cache). The prompt runs in chunks of up to 128 rows (dec_set_prefill_chunk):
+ * each chunk is one step whose projections are m = chunk contractions on the
+ * tensor-core paths and whose attention is causal per row; only the last row
+ * goes through the head. Whisper: `enc_hidden` (device f32 [enc_len, d]) is
  * required; cross-attention K and V are computed from it once per layer
  * ([cera] `precompute_cross_attention`: K = enc Wk^T + bk, V = enc Wv^T + bv).
  * Qwen2: enc_hidden must be NULL. n_tokens may be 0 (cross K/V only).
@@ -176,6 +179,29 @@ const char* dec_last_error(const dec_handle* h);
  */
 dec_status dec_prefill(dec_handle* h, int32_t slot, const int32_t* tokens, int32_t n_tokens,
                        const float* enc_hidden, float* last_logits, void* stream);
+
+/*
+ * Per-phase device timing ([wa-dec] `forward_probed`: where a decode step's
+ * time goes). While enabled, every dec_step / dec_step_host runs uncaptured
+ * with a CUDA event after each phase; dec_phase_times then gives, for the most
+ * recent step, each phase's device time in ms with its layer (-1 outside the
+ * layers) and kind, in launch order. Programmatic dependent launch does not
+ * overlap kernels across the events, so the phases sum to more than a captured
+ * step. dec_phase_times synchronises on the step's last event; *n receives the
+ * phase count (entries beyond cap are not written).
+ */
+enum {
+    DEC_PHASE_EMBED = 1, DEC_PHASE_QKV = 2, DEC_PHASE_SELF_ATTN = 3, DEC_PHASE_O = 4,
+    DEC_PHASE_CROSS_Q = 5, DEC_PHASE_CROSS_ATTN = 6, DEC_PHASE_CROSS_O = 7,
+    DEC_PHASE_FFN_UP = 8, DEC_PHASE_FFN_DOWN = 9, DEC_PHASE_HEAD = 10
+};
+dec_status dec_set_phase_timing(dec_handle* h, int32_t enabled);
+dec_status dec_phase_times(dec_handle* h, int32_t cap, float* ms, int32_t* layer, int32_t* kind, int32_t* n);
+
+/* Prompt rows per prefill step, 1..128 (default 128). A W8A8 model gives the same
+ * bits for every chunk size; f32 / W8A32 projections switch to the split-TF32
+ * tensor-core path from 8 rows on. */
+dec_status dec_set_prefill_chunk(dec_handle* h, int32_t rows);
 
 /*
  * Write rows [start_pos, start_pos + n_rows) of every layer's self-attention
@@ -284,6 +310,7 @@ dec_status dec_hidden(dec_handle* h, float* out, int32_t batch, void* stream);
  * n_layers * batch * d_model floats for every later step's batch (the caller
  * owns it; it must stay valid while set). NULL turns tracing off. Traced steps
  * run as their own captured graphs (one extra device-to-device copy per layer).
+ * dec_prefill's prompt chunks are not traced.
  */
 dec_status dec_set_layer_trace(dec_handle* h, float* buf);
 

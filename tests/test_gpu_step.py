@@ -206,3 +206,68 @@ def test_head_digit_planes_made_in_kernel_or_by_row_kernel_give_same_bits():
     assert np.array_equal(l17[:9].view(np.uint32), l9.view(np.uint32))
     p17.gpu.close()
     p9.gpu.close()
+
+
+@pytest.mark.parametrize("name,n", [("mid_qwen2", 200), ("small_qwen2", 131), ("mid_whisper", 60),
+                                     ("tiny_whisper_w8a32", 50)])
+def test_chunked_prefill_equals_row_by_row_prefill(name, n):
+    """A prompt run as chunks of rows of one slot (causal attention per row, m = chunk
+    projections) fills the same cache and gives the same last logits as one row per step:
+    bit for bit for W8A8 (exact integer products, per-row split boundaries), within the
+    tolerance for f32 / W8A32 (the split-TF32 path from 8 rows on)."""
+    import torch
+    from transformer_decoder_kv_b200 import Decoder
+
+    cfg = synth.MODELS[name]
+    W = synth.make_weights(cfg, 0)
+    n = min(n, cfg.max_pos)
+    toks = synth.token_ids(cfg, 3, n)
+    enc = torch.from_numpy(synth.encoder_hidden(cfg, 0)).cuda() if cfg.is_whisper else None
+    outs = []
+    for chunk in (1, 128, 37):
+        dec = Decoder(cfg, W, max_slots=2, max_cache_len=256)
+        dec.set_prefill_chunk(chunk)
+        lg = torch.empty(cfg.vocab, device="cuda")
+        dec.prefill(1, toks, enc, lg)
+        k = torch.empty((cfg.n_layers, n, cfg.d_model), device="cuda")
+        v = torch.empty_like(k)
+        for l in range(cfg.n_layers):
+            dec.kv_read(1, l, 0, n, k[l], v[l])
+        nxt = dec.next_tokens([1])[0]
+        torch.cuda.synchronize()
+        outs.append((lg.cpu().numpy(), k.cpu().numpy(), v.cpu().numpy(), nxt))
+        assert dec.slot_len(1) == n
+        dec.close()
+    base = outs[0]
+    for o in outs[1:]:
+        if cfg.proj_fmt == "w8a8":
+            for a, b in zip(o[:3], base[:3]):
+                assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+        else:
+            for a, b in zip(o[:3], base[:3]):
+                close(a, b, what=name)
+        assert o[3] == int(np.argmax(o[0]))
+
+
+def test_phase_timing_lists_every_phase_and_matches_the_step():
+    """dec_phase_times: one entry per phase in launch order (embed, per layer q|k|v,
+    self-attention, o, [cross q, cross-attention, cross o,] FFN up, FFN down, then the head),
+    positive device times, and the timed step computes the same logits as an untimed one."""
+    import torch
+    for wl_name in ("tiny_whisper_b3", "tiny_qwen2_b3"):
+        wl = synth.workload(wl_name)
+        cfg = wl.model
+        a, b = build_pair(wl), build_pair(wl)
+        b.gpu.set_phase_timing(True)
+        toks = [4, 5, 6]
+        la = step_both(a, toks)[0]
+        lb = step_both(b, toks)[0]
+        assert np.array_equal(la.view(np.uint32), lb.view(np.uint32))
+        ph = b.gpu.phase_times()
+        per_layer = ["qkv", "self_attn", "o"] + (["cross_q", "cross_attn", "cross_o"] if cfg.is_whisper else []) + \
+            ["ffn_up", "ffn_down"]
+        want = [(-1, "embed")] + [(l, k) for l in range(cfg.n_layers) for k in per_layer] + [(-1, "head")]
+        assert [(l, k) for l, k, _ in ph] == want
+        assert all(ms > 0 for _, _, ms in ph)
+        a.gpu.close()
+        b.gpu.close()

@@ -26,11 +26,14 @@ PROJ = {"f32": 0, "w8a8": 1, "w8a32": 2}
 EXPORTS = ["dec_create", "dec_destroy", "dec_last_error", "dec_prefill", "dec_kv_append", "dec_step",
            "dec_step_host", "dec_slot_len", "dec_kv_read", "dec_hidden", "dec_set_layer_trace", "dec_sync",
            "dec_reset", "dec_set_wait_limit", "dec_debug_inject", "dec_debug_fail_alloc", "dec_step_kernels",
-           "dec_next_tokens", "dec_get_config", "dec_generate",
+           "dec_next_tokens", "dec_get_config", "dec_generate", "dec_set_prefill_chunk",
+           "dec_set_phase_timing", "dec_phase_times",
            "dec_attention_workspace_size", "dec_attention", "dec_attention_plan", "dec_attention_noalloc",
            "dec_i8_dot"]
 I8_PATH = {"dp4a": 0, "tcgen05": 1}
 DEC_INJECT_DROP_ATTN_COPY = 1
+PHASE_NAMES = {1: "embed", 2: "qkv", 3: "self_attn", 4: "o", 5: "cross_q", 6: "cross_attn", 7: "cross_o",
+               8: "ffn_up", 9: "ffn_down", 10: "head"}
 
 
 class DecError(RuntimeError):
@@ -92,6 +95,9 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
         "dec_set_layer_trace": (C.c_int, [vp, vp]),
         "dec_sync": (C.c_int, [vp, vp]),
         "dec_reset": (C.c_int, [vp]),
+        "dec_set_prefill_chunk": (C.c_int, [vp, i32]),
+        "dec_set_phase_timing": (C.c_int, [vp, i32]),
+        "dec_phase_times": (C.c_int, [vp, i32, C.POINTER(C.c_float), pi32, pi32, pi32]),
         "dec_next_tokens": (C.c_int, [vp, i32, pi32, pi32, vp]),
         "dec_get_config": (C.c_int, [vp, C.POINTER(DecConfig)]),
         "dec_generate": (C.c_int, [vp, C.POINTER(DecRequest), i32, i32, pi32, i32, pi32, vp]),
@@ -271,6 +277,23 @@ class Decoder:
         lens = (C.c_int32 * max(1, n))()
         self._check(self._lib.dec_generate(self._h, arr, n, max_active, toks, stride, lens, stream))
         return [list(toks[i * stride: i * stride + lens[i]]) for i in range(n)]
+
+    def set_phase_timing(self, enabled: bool):
+        self._check(self._lib.dec_set_phase_timing(self._h, 1 if enabled else 0))
+
+    def phase_times(self):
+        """[(layer, phase name, ms)] of the most recent phase-timed step."""
+        cap = 4096
+        ms = (C.c_float * cap)()
+        layer = (C.c_int32 * cap)()
+        kind = (C.c_int32 * cap)()
+        n = C.c_int32(0)
+        self._check(self._lib.dec_phase_times(self._h, cap, ms, layer, kind, C.byref(n)))
+        return [(int(layer[i]), PHASE_NAMES.get(int(kind[i]), str(kind[i])), float(ms[i]))
+                for i in range(min(n.value, cap))]
+
+    def set_prefill_chunk(self, rows: int):
+        self._check(self._lib.dec_set_prefill_chunk(self._h, rows))
 
     def reset(self):
         self._check(self._lib.dec_reset(self._h))

@@ -113,9 +113,9 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
     const float* Kb = a.k + slot * a.slot_stride + static_cast<long long>(h) * a.ld * kHeadDim;
     const float* Vb = a.v + slot * a.slot_stride + static_cast<long long>(h) * a.ld * kHeadDim;
 
-    // tiles before the first one holding the row this step appends can be fetched
-    // before the dependency wait
-    const int first_new_tile = (a.mode == ATTN_SELF) ? (n - 1) / kAttnTile : ntiles;
+    // tiles before the first one holding a row this step writes can be fetched before the
+    // dependency wait (a prompt chunk writes rows fresh..len of its slot in one step)
+    const int first_new_tile = (a.mode == ATTN_SELF) ? a.meta->fresh[b] / kAttnTile : ntiles;
     int pre = 0;
     const bool drop = a.drop_first_copy && s == 0 && h == 0 && b == 0;
     if (tid == 0) {

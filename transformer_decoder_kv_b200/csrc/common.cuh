@@ -23,6 +23,8 @@ struct StepMeta {
     int tok[kMaxBatch];    // input token, or -1 for the slot's previous greedy pick
     int pos[kMaxBatch];    // learned-position row / RoPE position
     int len[kMaxBatch];    // cached rows before this step; the new row goes here
+    int fresh[kMaxBatch];  // first cache row of the row's slot that this step writes (len, or the
+                           // chunk's first row when several rows of one slot run together)
 };
 
 __device__ __forceinline__ unsigned long long global_ns() {

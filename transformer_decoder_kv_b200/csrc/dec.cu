@@ -33,6 +33,8 @@ using namespace dec;
 namespace {
 
 constexpr int kMetaRing = 8;
+// Prompt tokens of one slot that dec_prefill runs together as one step's rows.
+constexpr int kPrefillChunk = DEC_MAX_BATCH;
 constexpr int kMaxSplits = kAttnMaxSplits;
 
 thread_local std::string g_create_error;
@@ -94,6 +96,8 @@ struct dec_handle {
     float *kc = nullptr, *vc = nullptr, *xkc = nullptr, *xvc = nullptr;
     long long self_slot_stride = 0, self_layer_stride = 0, cross_slot_stride = 0, cross_layer_stride = 0;
     int max_batch = 0;
+    int max_rows = 0;                  // rows of the per-step workspaces: max(max_batch, prompt chunk)
+    int prefill_chunk = kPrefillChunk; // prompt rows per prefill step
     int tps_self = 1, tps_cross = 1;   // attention tiles per split (handle constants)
     // workspace
     float *x = nullptr, *q = nullptr, *ctx = nullptr, *ffn = nullptr, *xq = nullptr;
@@ -134,6 +138,11 @@ struct dec_handle {
     };
     std::map<std::array<long long, 5>, StepGraph> graphs;
     float* trace = nullptr;          // per-layer residual copies [L, B, d], or null
+    // per-phase device timing: an event after each phase of the most recent timed step
+    bool phase_timing = false;
+    std::vector<cudaEvent_t> phase_ev;
+    std::vector<std::array<int, 2>> phase_tag;   // (layer, DEC_PHASE_*) of each event after the first
+    size_t phase_n = 0;
     int last_step_kernels = -1;
     cudaStream_t cap_stream = nullptr;
     float* stage_logits = nullptr;   // dec_step_host result staging
@@ -486,16 +495,38 @@ GemvArgs base_args(dec_handle* h, int B) {
     return g;
 }
 
+// Per-phase timing: an event recorded after the phase (only while timing is on).
+dec_status phase_mark(dec_handle* h, cudaStream_t st, int layer, int kind) {
+    if (!h->phase_timing) return DEC_OK;
+    if (h->phase_n == h->phase_ev.size()) {
+        cudaEvent_t e;
+        DEC_CUDA(h, cudaEventCreate(&e));
+        h->phase_ev.push_back(e);
+        h->phase_tag.push_back({0, 0});
+    }
+    DEC_CUDA(h, cudaEventRecord(h->phase_ev[h->phase_n], st));
+    h->phase_tag[h->phase_n] = {layer, kind};
+    ++h->phase_n;
+    return DEC_OK;
+}
+
 // One step for the batch described in h->dmeta (already uploaded).
-dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int* argmax, cudaStream_t st) {
+// head_row0 / head_rows: the rows whose logits the head computes (all by default; a prompt
+// chunk needs its last row only, or none). trace: copy each layer's residual (decode steps).
+dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int* argmax, cudaStream_t st,
+                    int head_row0 = 0, int head_rows = -1, bool trace = true) {
+    if (head_rows < 0) head_rows = B;
     const dec_config& c = h->cfg;
     const int d = c.d_model, F = c.d_ff, H = c.n_heads;
     {
         thread_local int attr_dev = -1;
         DEC_CUDA(h, prefer_max_shared_once(k_embed, attr_dev));
     }
+    h->phase_n = 0;
+    DEC_TRY(phase_mark(h, st, -1, 0));
     DEC_CUDA(h, launch(k_embed, dim3(B), dim3(128), 0, st, (const float*)h->tok_emb, (const float*)h->pos_emb,
                        (const StepMeta*)h->dmeta, (const int*)h->last_tok, h->x, d));
+    DEC_TRY(phase_mark(h, st, -1, DEC_PHASE_EMBED));
     for (int l = 0; l < c.n_layers; ++l) {
         const LayerDev& L = h->layers[l];
         float* kc = h->kc + l * h->self_layer_stride;
@@ -524,6 +555,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             g.rope = h->rope;
             DEC_TRY((gemv_qwen<PRO_RMS, EPI_QKV, MAP_ROPE>(h, g, L.m_qkv, st)));
         }
+        DEC_TRY(phase_mark(h, st, l, DEC_PHASE_QKV));
         // ---- self-attention over rows 0..len ----
         AttnArgs at{};
         at.q = h->q;
@@ -542,6 +574,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
         at.err = h->dev_err;
         at.drop_first_copy = (l == 0) ? h->inject_drop : 0;
         DEC_TRY(attention(h, at, B, max_len_plus1, h->tps_self, st));
+        DEC_TRY(phase_mark(h, st, l, DEC_PHASE_SELF_ATTN));
         at.drop_first_copy = 0;
         // ---- output projection + residual ----
         g = base_args(h, B);
@@ -559,6 +592,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
         } else {
             DEC_TRY((gemv_qwen<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, L.m_o, st)));
         }
+        DEC_TRY(phase_mark(h, st, l, DEC_PHASE_O));
         if (c.family == DEC_FAMILY_WHISPER) {
             // ---- cross-attention block ----
             g = base_args(h, B);
@@ -574,6 +608,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             g.out = h->xq;
             g.out_ld = d;
             DEC_TRY((gemv_whisper<PRO_LN, EPI_STORE, MAP_ADJ>(h, g, st, &L.m_xq)));
+            DEC_TRY(phase_mark(h, st, l, DEC_PHASE_CROSS_Q));
             at.q = h->xq;
             at.k = h->xkc + l * h->cross_layer_stride;
             at.v = h->xvc + l * h->cross_layer_stride;
@@ -582,6 +617,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             at.mode = ATTN_CROSS;
             at.n_fixed = c.enc_len;
             DEC_TRY(attention(h, at, B, c.enc_len, h->tps_cross, st));
+            DEC_TRY(phase_mark(h, st, l, DEC_PHASE_CROSS_ATTN));
             g = base_args(h, B);
             g.x = h->ctx;
             g.x_ld = d;
@@ -593,6 +629,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             g.out = h->x;
             g.out_ld = d;
             DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st, &L.m_xo)));
+            DEC_TRY(phase_mark(h, st, l, DEC_PHASE_CROSS_O));
             // ---- GELU FFN ----
             g = base_args(h, B);
             g.x = h->x;
@@ -607,6 +644,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             g.out = h->ffn;
             g.out_ld = F;
             DEC_TRY((gemv_whisper<PRO_LN, EPI_GELU, MAP_ADJ>(h, g, st, &L.m_1)));
+            DEC_TRY(phase_mark(h, st, l, DEC_PHASE_FFN_UP));
             g = base_args(h, B);
             g.x = h->ffn;
             g.x_ld = F;
@@ -618,6 +656,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             g.out = h->x;
             g.out_ld = d;
             DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st, &L.m_2)));
+            DEC_TRY(phase_mark(h, st, l, DEC_PHASE_FFN_DOWN));
         } else {
             // ---- SwiGLU MLP ----
             g = base_args(h, B);
@@ -633,6 +672,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             g.out = h->ffn;
             g.out_ld = F;
             DEC_TRY((gemv_qwen<PRO_RMS, EPI_SWIGLU, MAP_DUAL>(h, g, L.m_1, st)));
+            DEC_TRY(phase_mark(h, st, l, DEC_PHASE_FFN_UP));
             g = base_args(h, B);
             g.x = h->ffn;
             g.x_ld = F;
@@ -643,14 +683,16 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             g.out = h->x;
             g.out_ld = d;
             DEC_TRY((gemv_qwen<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, L.m_2, st)));
+            DEC_TRY(phase_mark(h, st, l, DEC_PHASE_FFN_DOWN));
         }
-        if (h->trace)
+        if (trace && h->trace)
             DEC_CUDA(h, cudaMemcpyAsync(h->trace + static_cast<size_t>(l) * B * d, h->x, size_t(B) * d * 4,
                                         cudaMemcpyDeviceToDevice, st));
     }
     // ---- final norm + tied head + greedy argmax ----
-    GemvArgs g = base_args(h, B);
-    g.x = h->x;
+    if (head_rows == 0) return DEC_OK;
+    GemvArgs g = base_args(h, head_rows);
+    g.x = h->x + static_cast<size_t>(head_row0) * d;
     g.x_ld = d;
     g.norm_w = h->final_w;
     g.norm_b = h->final_b;
@@ -668,6 +710,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
     } else {
         DEC_TRY(head<PRO_RMS>(h, g, st));
     }
+    DEC_TRY(phase_mark(h, st, -1, DEC_PHASE_HEAD));
     return DEC_OK;
 }
 
@@ -731,6 +774,7 @@ dec_status validate_step(dec_handle* h, int B, const int32_t* slots, const int32
         m.tok[b] = tokens ? tokens[b] : -1;
         m.pos[b] = positions[b];
         m.len[b] = cache_lens[b];
+        m.fresh[b] = cache_lens[b];
         max_len = std::max(max_len, cache_lens[b] + 1);
     }
     return DEC_OK;
@@ -780,8 +824,8 @@ dec_status step_validated(dec_handle* h, const StepMeta& m, int max_len, float* 
                                           reinterpret_cast<long long>(logits), reinterpret_cast<long long>(argmax),
                                           reinterpret_cast<long long>(h->trace)};
     auto it = h->graphs.find(key);
-    if (h->inject_drop) {
-        // fault-injection steps run eagerly and are never captured
+    if (h->inject_drop || h->phase_timing) {
+        // fault-injection and phase-timed steps run eagerly and are never captured
         DEC_TRY(run_step(h, m.B, max_len, logits, argmax, st));
         h->last_step_kernels = -1;
     } else if (it != h->graphs.end() && it->second.exec != nullptr) {
@@ -813,6 +857,7 @@ dec_status dec_destroy(dec_handle* h) {
     cudaDeviceSynchronize();
     for (auto& kv : h->graphs)
         if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
+    for (cudaEvent_t e : h->phase_ev) cudaEventDestroy(e);
     if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
     for (void* p : h->dallocs) cudaFree(p);
     for (void* p : h->hallocs) cudaFreeHost(p);
@@ -938,7 +983,9 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
     h->max_batch = std::min(c.max_slots, DEC_MAX_BATCH);
     h->tps_self = tiles_per_split(h, c.max_cache_len);
     h->tps_cross = wh ? tiles_per_split(h, c.enc_len) : 1;
-    const int MB = h->max_batch;
+    // per-step workspaces hold a decode batch or a prompt chunk, whichever is larger
+    h->max_rows = std::max(h->max_batch, kPrefillChunk);
+    const int MB = h->max_rows;
     DEC_TRY(dalloc(h, &h->x, size_t(MB) * d * 4));
     DEC_TRY(dalloc(h, &h->q, size_t(MB) * d * 4));
     DEC_TRY(dalloc(h, &h->ctx, size_t(MB) * d * 4));
@@ -1001,8 +1048,8 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
     DEC_TRY(dalloc(h, &h->dev_err, kStatusWords * 4));
     DEC_CUDA(h, cudaMemset(h->dev_err, 0, kStatusWords * 4));
     DEC_TRY(dalloc(h, &h->dmeta, sizeof(StepMeta)));
-    DEC_TRY(dalloc(h, &h->stage_logits, size_t(MB) * c.vocab * 4));
-    DEC_TRY(dalloc(h, &h->stage_argmax, size_t(MB) * 4));
+    DEC_TRY(dalloc(h, &h->stage_logits, size_t(h->max_batch) * c.vocab * 4));
+    DEC_TRY(dalloc(h, &h->stage_argmax, size_t(h->max_batch) * 4));
     auto halloc = [&](void** p, size_t bytes) {
         if (injected_alloc_failure()) return fail(h, DEC_ENOMEM, "cudaMallocHost failed (injected)");
         if (cudaMallocHost(p, bytes) != cudaSuccess) {
@@ -1093,16 +1140,36 @@ dec_status dec_prefill(dec_handle* h, int32_t slot, const int32_t* tokens, int32
     }
     h->slot_len[slot] = 0;
     h->has_tok[slot] = 0;
-    for (int i = 0; i < n_tokens; ++i) {
+    // The prompt runs in chunks of up to prefill_chunk rows of this one slot at consecutive
+    // positions ([focr] `forward_prefill_seed`: the whole prompt in one forward): each
+    // chunk is one step whose projections are m = chunk contractions and whose attention is
+    // causal per row (row i attends cache rows 0..i, the chunk's earlier rows included).
+    // Only the prompt's last row goes through the head. Chunks run uncaptured.
+    for (int i0 = 0; i0 < n_tokens; i0 += h->prefill_chunk) {
+        const int B = std::min(h->prefill_chunk, n_tokens - i0);
         StepMeta m{};
-        m.B = 1;
-        m.slot[0] = slot;
-        m.tok[0] = tokens[i];
-        m.pos[0] = i;
-        m.len[0] = i;
-        float* lg = (i == n_tokens - 1) ? last_logits : nullptr;
-        DEC_TRY(step_validated(h, m, i + 1, lg, nullptr, st));
+        m.B = B;
+        for (int b = 0; b < B; ++b) {
+            m.slot[b] = slot;
+            m.tok[b] = tokens[i0 + b];
+            m.pos[b] = i0 + b;
+            m.len[b] = i0 + b;
+            m.fresh[b] = i0;
+        }
+        const bool last = i0 + B == n_tokens;
+        DEC_TRY(upload_meta(h, m, st));
+        const bool timing = h->phase_timing;   // prompt chunks are not phase-timed
+        h->phase_timing = false;
+        struct Restore {
+            dec_handle* h;
+            bool v;
+            ~Restore() { h->phase_timing = v; }
+        } restore{h, timing};
+        DEC_TRY(run_step(h, B, i0 + B, last ? last_logits : nullptr, nullptr, st, B - 1, last ? 1 : 0, false));
+        h->slot_len[slot] = i0 + B;
     }
+    if (n_tokens > 0) h->has_tok[slot] = 1;
+    h->last_batch = 0;
     return DEC_OK;
 }
 
@@ -1230,6 +1297,35 @@ dec_status dec_hidden(dec_handle* h, float* out, int32_t batch, void* stream) {
     return DEC_OK;
 }
 
+dec_status dec_set_phase_timing(dec_handle* h, int32_t enabled) {
+    if (!h) return fail(nullptr, DEC_EINVAL, "dec_set_phase_timing: null handle");
+    h->phase_timing = enabled != 0;
+    h->phase_n = 0;
+    return DEC_OK;
+}
+
+dec_status dec_phase_times(dec_handle* h, int32_t cap, float* ms, int32_t* layer, int32_t* kind, int32_t* n) {
+    if (!h || !n || (cap > 0 && (!ms || !layer || !kind))) return fail(h, DEC_EINVAL, "dec_phase_times: bad arguments");
+    const int phases = h->phase_n > 0 ? static_cast<int>(h->phase_n) - 1 : 0;
+    *n = phases;
+    if (phases == 0) return DEC_OK;
+    DEC_CUDA(h, cudaEventSynchronize(h->phase_ev[h->phase_n - 1]));
+    for (int i = 0; i < phases && i < cap; ++i) {
+        DEC_CUDA(h, cudaEventElapsedTime(&ms[i], h->phase_ev[i], h->phase_ev[i + 1]));
+        layer[i] = h->phase_tag[i + 1][0];
+        kind[i] = h->phase_tag[i + 1][1];
+    }
+    return DEC_OK;
+}
+
+dec_status dec_set_prefill_chunk(dec_handle* h, int32_t rows) {
+    if (!h) return fail(nullptr, DEC_EINVAL, "dec_set_prefill_chunk: null handle");
+    if (rows < 1 || rows > kPrefillChunk)
+        return fail(h, DEC_EINVAL, "prefill chunk must be in [1, " + std::to_string(kPrefillChunk) + "]");
+    h->prefill_chunk = rows;
+    return DEC_OK;
+}
+
 dec_status dec_set_layer_trace(dec_handle* h, float* buf) {
     if (!h) return fail(nullptr, DEC_EINVAL, "dec_set_layer_trace: null handle");
     if (buf && (reinterpret_cast<uintptr_t>(buf) & 3)) return fail(h, DEC_EINVAL, "trace buffer must be 4-byte aligned");
@@ -1259,7 +1355,7 @@ dec_status dec_reset(dec_handle* h) {
     DEC_TRY(check_device(h));
     // every kernel of the handle has ended before the counters are cleared
     DEC_CUDA(h, cudaDeviceSynchronize());
-    const int MB = h->max_batch, H = h->cfg.n_heads;
+    const int MB = h->max_rows, H = h->cfg.n_heads;
     DEC_CUDA(h, cudaMemset(h->counters, 0, size_t(MB) * H * 4));
     if (h->mma_cnt) DEC_CUDA(h, cudaMemset(h->mma_cnt, 0, size_t(h->mma_cnt_bytes)));
     DEC_CUDA(h, cudaMemset(h->head_counter, 0, 16));
