@@ -53,8 +53,10 @@ def measured_peaks():
 
 # ---------------------------------------------------------------- algorithmic bytes
 
-def step_bytes(cfg: synth.ModelConfig, lens) -> dict:
-    """Bytes one decode step must move (each weight once, caches read, rows written)."""
+def step_bytes(cfg: synth.ModelConfig, lens, head: str = "exact") -> dict:
+    """Bytes one decode step must move (each weight once, caches read, rows written). The
+    head is the f32 embedding (V d 4 bytes), or for the int8 head its int8 rows and row
+    scales (V d + 4 V bytes; the candidates' exact re-score is a few rows)."""
     d, F, L, V = cfg.d_model, cfg.d_ff, cfg.n_layers, cfg.vocab
     B = len(lens)
     wb = 4 if cfg.proj_fmt == "f32" else 1
@@ -69,7 +71,7 @@ def step_bytes(cfg: synth.ModelConfig, lens) -> dict:
     weights = nW * wb + (rows * 4 if wb == 1 else 0) + rows * 4 * (1 if cfg.is_whisper else 0) + small
     if not cfg.is_whisper:
         weights += L * 3 * d * 4                            # q/k/v biases
-    head = V * d * 4
+    head = V * d * 4 if head == "exact" else V * d + V * 4
     self_kv = sum(L * (int(n) + 1) * d * 2 * 4 for n in lens)
     kv_write = B * L * d * 2 * 4
     cross = B * L * cfg.enc_len * d * 2 * 4 if cfg.is_whisper else 0
@@ -150,7 +152,7 @@ def clocks_rejected(clocks: dict) -> bool:
 class GpuWorkload:
     """The workload's decoder with its streams brought to their initial cache state."""
 
-    def __init__(self, wl: synth.Workload, seed: int, fast_setup: bool = False):
+    def __init__(self, wl: synth.Workload, seed: int, fast_setup: bool = False, head: str = "exact"):
         import torch
         from transformer_decoder_kv_b200 import Decoder
 
@@ -158,7 +160,7 @@ class GpuWorkload:
         cfg = wl.model
         self.cfg = cfg
         W = synth.make_weights(cfg, seed)
-        self.dec = Decoder(cfg, W, max_slots=wl.batch, max_cache_len=wl.max_cache_len)
+        self.dec = Decoder(cfg, W, max_slots=wl.batch, max_cache_len=wl.max_cache_len, head=head)
         del W
         self.lens0 = synth.cache_lens(wl, seed).astype(np.int64)
         B = wl.batch
@@ -223,7 +225,7 @@ def run_ours(args, wl: synth.Workload, rank: int, world: int) -> dict:
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
     seed = rank
     cfg = wl.model
-    gw = GpuWorkload(wl, seed, fast_setup=args.fast_setup)
+    gw = GpuWorkload(wl, seed, fast_setup=args.fast_setup, head=args.head)
     stream = torch.cuda.Stream()
     sh = stream.cuda_stream
     with torch.cuda.stream(stream):
@@ -260,7 +262,7 @@ def run_ours(args, wl: synth.Workload, rank: int, world: int) -> dict:
     value, ms_max, tokens_all = combine_ranks(ms, tokens, world)
 
     # bytes actually moved per step at the lengths seen
-    per_step_bytes = [step_bytes(cfg, p)["total"] for p in lens_seen]
+    per_step_bytes = [step_bytes(cfg, p, args.head)["total"] for p in lens_seen]
     achieved_gbs = sum(per_step_bytes) / (ms / 1e3) / 1e9
 
     # ---- e2e through host buffers ----
@@ -502,6 +504,8 @@ def main():
                     help="bracket the timed steps with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
     ap.add_argument("--fast-setup", action="store_true",
                     help="seed caches with N(0,1) K/V instead of prefilling tokens (profiling runs)")
+    ap.add_argument("--head", default="exact", choices=["exact", "int8"],
+                    help="LM head: exact three-digit split, or int8 with exact re-scoring of the candidates")
     ap.add_argument("--batch", type=int, default=0,
                     help="profiling only: fewer streams than the workload (same model and kernels)")
     ap.add_argument("--max-cache-len", type=int, default=0,
@@ -532,7 +536,8 @@ def main():
               if step_bytes(cfg, synth.cache_lens(wl))["total"] > L2_BYTES else "n/a",
               "parallelism": f"replicas x{args.gpus}",
               "cache_setup": "seeded K/V rows (profiling)" if args.fast_setup else wl.cache_init,
-              "fast_setup": bool(args.fast_setup)}
+              "fast_setup": bool(args.fast_setup),
+              "head": "exact three-digit" if args.head == "exact" else "int8 + exact re-score of candidates"}
     metric = "decode tokens/s (device-timed)"
     if args.impl == "reference":
         if rank != 0:

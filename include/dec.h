@@ -70,7 +70,17 @@ enum { DEC_PROJ_F32 = 0, DEC_PROJ_W8A8 = 1, DEC_PROJ_W8A32 = 2 };
  *   rope_theta  RoPE base (qwen2), e.g. 1e6.
  *   max_slots   number of independent streams the handle holds caches for.
  *   max_cache_len  rows per stream and layer in the self-attention cache.
+ *   head_fmt    DEC_HEAD_EXACT: the tied head on the f32 embedding (three-digit
+ *               exact-integer split, 3 bytes per weight). DEC_HEAD_INT8_REFINE
+ *               ([focr] `LmHead` int8 arm, `got_lm_head`: int8 per-row head, then an
+ *               exact re-score of the best candidates): coarse logits from the
+ *               embedding's per-row int8 quantisation (1 byte per weight), then every
+ *               token whose coarse logit is within a proven error bound of the row's
+ *               best is re-scored with the exact head's arithmetic. The greedy pick
+ *               equals the exact head's pick; the returned logits are exact for those
+ *               candidates and coarse (within the bound) elsewhere.
  */
+enum { DEC_HEAD_EXACT = 0, DEC_HEAD_INT8_REFINE = 1 };
 typedef struct dec_config {
     int32_t family;
     int32_t n_layers;
@@ -86,6 +96,7 @@ typedef struct dec_config {
     float rope_theta;
     int32_t max_slots;
     int32_t max_cache_len;
+    int32_t head_fmt;
 } dec_config;
 
 /*

@@ -113,3 +113,70 @@ def test_dropping_a_kept_product_is_detected():
     exact = float(np.dot(w.astype(np.float64), x.astype(np.float64)))
     good = float(head_logit(w, x))
     assert abs(bad - exact) > 20 * abs(good - exact) + 1e-9
+
+
+def coarse_logit(w: np.ndarray, x: np.ndarray) -> np.float32:
+    """The int8 head's coarse logit: only the embedding row's first digit (its per-row int8
+    quantisation) against the hidden row's three digits, combined like head_logit."""
+    D1, _, _, sw = digits3(w)
+    E1, E2, E3, sx = digits3(x)
+    a0, a1, a2 = int(np.dot(D1, E1)), int(np.dot(D1, E2)), int(np.dot(D1, E3))
+    u = F(F(a1) + F(F(a2) * F(1.0 / 254.0)))
+    t = F(F(a0) + F(u * F(1.0 / 254.0)))
+    return F(F(sw * sx) * t)
+
+
+def int8_head_bound(w, x, coarse, c1=0.502, c2=0.002):
+    """The kernel's bound on |exact head - coarse|: s_n s_b (c1 S1 + c2 S2) * 1.001 plus a few
+    ulps of the coarse logit, with S1 = sum |E1|, S2 = sum |E2| of the hidden row's digits."""
+    _, _, _, sw = digits3(w)
+    E1, E2, _, sx = digits3(x)
+    b = float(F(sw * sx)) * (c1 * float(np.abs(E1).sum()) + c2 * float(np.abs(E2).sum()))
+    return b * 1.001 + 4e-6 * abs(float(coarse)) + 1e-30
+
+
+@pytest.mark.parametrize("kind", ["normal", "outlier"])
+def test_int8_head_bound_holds(kind):
+    """Every exact-head logit lies within the bound of its coarse logit, so the candidates
+    (coarse + bound >= the row's largest coarse - bound) contain the exact argmax."""
+    rng = np.random.default_rng([13, len(kind)])
+    worst = 0.0
+    for k in (384, 1024, 1280):
+        for _ in range(40):
+            w = (_rows(rng, k, kind) * F(0.02)).astype(F)
+            x = _rows(rng, k, "normal")
+            c = coarse_logit(w, x)
+            e = head_logit(w, x)
+            bnd = int8_head_bound(w, x, c)
+            assert abs(float(e) - float(c)) <= bnd, (kind, k, e, c, bnd)
+            worst = max(worst, abs(float(e) - float(c)) / bnd)
+    assert worst > 0.01   # the bound is not vacuous by orders of magnitude
+
+
+def test_int8_head_bound_with_a_halved_coefficient_fails():
+    """Mutation: a bound with half the first coefficient is violated on ordinary rows."""
+    rng = np.random.default_rng(17)
+    misses = 0
+    for _ in range(200):
+        w = (rng.standard_normal(64) * 0.02).astype(F)
+        w[0] = F(0.08)   # a large element: coarse digits round away much of the small ones
+        x = rng.standard_normal(64).astype(F)
+        c = coarse_logit(w, x)
+        if abs(float(head_logit(w, x)) - float(c)) > int8_head_bound(w, x, c, c1=0.0, c2=0.0):
+            misses += 1
+    assert misses > 0
+
+
+def test_int8_head_candidates_contain_the_argmax():
+    """On a small vocabulary, the candidate rule keeps the exact head's argmax and few others."""
+    rng = np.random.default_rng(19)
+    V, k = 2000, 256
+    E = (rng.standard_normal((V, k)) * 0.02).astype(F)
+    x = rng.standard_normal(k).astype(F)
+    exact = np.array([head_logit(E[n], x) for n in range(V)], np.float64)
+    coarse = np.array([coarse_logit(E[n], x) for n in range(V)], np.float64)
+    bound = np.array([int8_head_bound(E[n], x, coarse[n]) for n in range(V)])
+    thr = np.max(coarse - bound)
+    cand = np.nonzero(coarse + bound >= thr)[0]
+    assert int(np.argmax(exact)) in set(cand.tolist())
+    assert len(cand) < V // 10

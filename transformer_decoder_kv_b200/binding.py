@@ -20,6 +20,7 @@ DEC_OK, DEC_EINVAL, DEC_ERANGE, DEC_EOVERFLOW, DEC_ESTATE, DEC_ENOMEM, DEC_ECUDA
 STATUS_NAMES = ["DEC_OK", "DEC_EINVAL", "DEC_ERANGE", "DEC_EOVERFLOW", "DEC_ESTATE", "DEC_ENOMEM",
                 "DEC_ECUDA", "DEC_ETIMEOUT"]
 FAMILY = {"whisper": 0, "qwen2": 1}
+HEAD = {"exact": 0, "int8": 1}
 PROJ = {"f32": 0, "w8a8": 1, "w8a32": 2}
 
 # Every symbol include/dec.h declares.
@@ -48,7 +49,7 @@ class DecConfig(C.Structure):
                 ("n_heads", C.c_int32), ("head_dim", C.c_int32), ("d_ff", C.c_int32),
                 ("vocab", C.c_int32), ("max_pos", C.c_int32), ("enc_len", C.c_int32),
                 ("proj_fmt", C.c_int32), ("norm_eps", C.c_float), ("rope_theta", C.c_float),
-                ("max_slots", C.c_int32), ("max_cache_len", C.c_int32)]
+                ("max_slots", C.c_int32), ("max_cache_len", C.c_int32), ("head_fmt", C.c_int32)]
 
 
 class DecProj(C.Structure):
@@ -147,11 +148,11 @@ def _ptr(a) -> Optional[int]:
 class Decoder:
     """One handle of the CUDA decoder (dec_create ... dec_destroy)."""
 
-    def __init__(self, cfg, weights: dict, max_slots: int, max_cache_len: int):
+    def __init__(self, cfg, weights: dict, max_slots: int, max_cache_len: int, head: str = "exact"):
         self._lib = lib()
         c = DecConfig(FAMILY[cfg.family], cfg.n_layers, cfg.d_model, cfg.n_heads, cfg.head_dim,
                       cfg.d_ff, cfg.vocab, cfg.max_pos, cfg.enc_len, PROJ[cfg.proj_fmt],
-                      float(cfg.norm_eps), float(cfg.rope_theta), max_slots, max_cache_len)
+                      float(cfg.norm_eps), float(cfg.rope_theta), max_slots, max_cache_len, HEAD[head])
         self.cfg = cfg
         self.max_slots = max_slots
         self.max_cache_len = max_cache_len

@@ -89,6 +89,10 @@ struct dec_handle {
     // tcgen05 head: embedding and hidden rows as three int8 digit planes with row scales
     int8_t *wdig = nullptr, *xdig = nullptr;
     float *wsc = nullptr, *xsc = nullptr;
+    int* xsum = nullptr;            // per hidden row: sum |D1|, sum |D2| (int8 head bound)
+    float* head_thr = nullptr;      // int8 head: per-row candidate threshold
+    int* head_cand = nullptr;       // int8 head: candidate list (max_batch * vocab)
+    float* head_logits = nullptr;   // int8 head: coarse logits when the caller passes none
     int xdig_rows = 0;             // rows per hidden digit plane (>= max batch, >= 32)
     CUtensorMap m_wdig, m_xdig16, m_xdig32;
     bool head_tc_ok = false;
@@ -253,6 +257,10 @@ dec_status validate_config(const dec_config& c) {
     if (c.max_slots < 1) return bad("max_slots must be >= 1");
     if (c.max_cache_len < 1) return bad("max_cache_len must be >= 1");
     if (!(c.norm_eps > 0.0f)) return bad("norm_eps must be > 0");
+    if (c.head_fmt != DEC_HEAD_EXACT && c.head_fmt != DEC_HEAD_INT8_REFINE) return bad("unknown head_fmt");
+    if (c.head_fmt == DEC_HEAD_INT8_REFINE &&
+        (c.d_model > 4096 || static_cast<long long>(c.vocab) * DEC_MAX_BATCH >= (1LL << 31)))
+        return bad("the int8 head needs d_model <= 4096 and vocab * 128 < 2^31");
     if (c.family == DEC_FAMILY_WHISPER) {
         if (c.enc_len < 1) return bad("whisper needs enc_len >= 1");
         if (c.proj_fmt != DEC_PROJ_F32 && c.proj_fmt != DEC_PROJ_W8A32)
@@ -395,13 +403,16 @@ template <int PRO>
 dec_status head(dec_handle* h, const GemvArgs& a, cudaStream_t st) {
     if (h->head_tc_ok) {
         const int d = h->cfg.d_model;
-        // batches above 16: the hidden rows' digit planes come from their own kernel;
-        // smaller batches make them inside the head kernel (same arithmetic)
-        const bool own = head_tc_makes_planes(a.B);
+        const bool int8_head = h->cfg.head_fmt == DEC_HEAD_INT8_REFINE;
+        // batches above 16 (and the int8 head, whose refine kernel reads them): the hidden
+        // rows' digit planes come from their own kernel; smaller batches of the exact head make
+        // them inside the head kernel (same arithmetic)
+        const bool own = !int8_head && head_tc_makes_planes(a.B);
         cudaError_t e = cudaSuccess;
         if (!own) {
             e = rowprep_digits_launch<PRO>(a.x, a.x_ld, a.norm_w, a.norm_b, a.eps, d, a.B,
-                                           static_cast<long long>(h->xdig_rows) * d, h->xdig, h->xsc, true, st);
+                                           static_cast<long long>(h->xdig_rows) * d, h->xdig, h->xsc, h->xsum, true,
+                                           st);
             if (e != cudaSuccess) return cuda_fail(h, e, "head row split launch");
         }
         HeadArgs ha;
@@ -427,6 +438,16 @@ dec_status head(dec_handle* h, const GemvArgs& a, cudaStream_t st) {
         ha.last_tok = a.last_tok;
         ha.meta = a.meta;
         ha.err = a.err;
+        ha.xsum = h->xsum;
+        ha.thr = h->head_thr;
+        if (int8_head) {
+            // coarse logits go to the caller's buffer, or to the handle's when there is none
+            if (ha.logits == nullptr) ha.logits = h->head_logits;
+            e = head_int8_launch(h->num_sms, ha, h->wdig, h->xdig, h->head_cand, h->head_counter + 2,
+                                 h->head_counter + 1, st);
+            if (e != cudaSuccess) return cuda_fail(h, e, "int8 head launch");
+            return DEC_OK;
+        }
         e = head_tc_launch(h->num_sms, ha, own ? PRO : kHeadXExternal, st);
         if (e != cudaSuccess) return cuda_fail(h, e, "tensor-core head launch");
         return DEC_OK;
@@ -950,18 +971,28 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
         DEC_TRY(dalloc(h, &h->wdig, size_t(3) * V * d));
         DEC_TRY(dalloc(h, &h->wsc, size_t(V) * 4));
         DEC_CUDA(h, rowprep_digits_launch<PRO_NONE>(h->tok_emb, d, nullptr, nullptr, 0.0f, d, c.vocab, V * d, h->wdig,
-                                                   h->wsc, false, 0));
+                                                   h->wsc, nullptr, false, 0));
         h->xdig_rows = std::max(std::min(c.max_slots, DEC_MAX_BATCH), 32);
         const size_t xb = size_t(3) * h->xdig_rows * d;
         DEC_TRY(dalloc(h, &h->xdig, xb));
         DEC_CUDA(h, cudaMemset(h->xdig, 0, xb));
         DEC_TRY(dalloc(h, &h->xsc, size_t(h->xdig_rows) * 4));
         DEC_CUDA(h, cudaMemset(h->xsc, 0, size_t(h->xdig_rows) * 4));
+        DEC_TRY(dalloc(h, &h->xsum, size_t(h->xdig_rows) * 8));
+        DEC_CUDA(h, cudaMemset(h->xsum, 0, size_t(h->xdig_rows) * 8));
+        if (c.head_fmt == DEC_HEAD_INT8_REFINE) {
+            const size_t mb = size_t(std::min(c.max_slots, DEC_MAX_BATCH));
+            DEC_TRY(dalloc(h, &h->head_thr, mb * 4));
+            DEC_TRY(dalloc(h, &h->head_cand, mb * size_t(c.vocab) * 4));
+            DEC_TRY(dalloc(h, &h->head_logits, mb * size_t(c.vocab) * 4));
+        }
         dec_status ts = make_wmap(h, &h->m_wdig, h->wdig, int(3 * V), d, false);
         if (ts == DEC_OK) ts = make_wmap(h, &h->m_xdig16, h->xdig, 3 * h->xdig_rows, d, false, 16);
         if (ts == DEC_OK) ts = make_wmap(h, &h->m_xdig32, h->xdig, 3 * h->xdig_rows, d, false, 32);
         h->head_tc_ok = (ts == DEC_OK);
         if (!h->head_tc_ok) h->err.clear();
+        if (!h->head_tc_ok && c.head_fmt == DEC_HEAD_INT8_REFINE)
+            return fail(h, DEC_EINVAL, "the int8 head needs the tensor-core head (TMA descriptors unavailable)");
         DEC_CUDA(h, cudaDeviceSynchronize());
     }
     // caches

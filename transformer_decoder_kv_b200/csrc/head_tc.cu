@@ -7,9 +7,9 @@
 
 namespace dec {
 template cudaError_t rowprep_digits_launch<PRO_NONE>(const float*, int, const float*, const float*, float, int, int,
-                                                     long long, int8_t*, float*, bool, cudaStream_t);
+                                                     long long, int8_t*, float*, int*, bool, cudaStream_t);
 template cudaError_t rowprep_digits_launch<PRO_LN>(const float*, int, const float*, const float*, float, int, int,
-                                                   long long, int8_t*, float*, bool, cudaStream_t);
+                                                   long long, int8_t*, float*, int*, bool, cudaStream_t);
 template cudaError_t rowprep_digits_launch<PRO_RMS>(const float*, int, const float*, const float*, float, int, int,
-                                                    long long, int8_t*, float*, bool, cudaStream_t);
+                                                    long long, int8_t*, float*, int*, bool, cudaStream_t);
 }  // namespace dec

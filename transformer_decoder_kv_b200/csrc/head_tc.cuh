@@ -42,7 +42,8 @@ constexpr int kHeadRows = 128;                      // embedding rows per block 
 constexpr int kHeadKC = 128;                        // K per stage (one 128-byte box per plane)
 constexpr int kHeadPlaneBox = kHeadRows * kHeadKC;  // 16 KB
 constexpr int kHeadStageBytes = 3 * kHeadPlaneBox;  // 48 KB
-constexpr int kHeadMaxStages = 4;
+constexpr int kHeadMaxStages = 4;      // three-digit stages (48 KB)
+constexpr int kHeadMaxStagesW1 = 8;    // one-digit stages (16 KB)
 constexpr int kHeadMaxK = 4096;
 
 struct HeadArgs {
@@ -65,6 +66,10 @@ struct HeadArgs {
     int* last_tok;             // [slots]
     const StepMeta* meta;
     int* err;
+    // int8 head (one embedding digit): per hidden row S1 = sum |D1|, S2 = sum |D2| [MB, 2], and
+    // the per-row threshold max_n (coarse_n - bound_n) written by the last CTA [B]
+    const int* xsum;
+    float* thr;
 };
 
 // Three base-254 digits of v / s with inv = 1 / s (|v| <= amax, so |v inv| <= 127).
@@ -87,7 +92,7 @@ __device__ __forceinline__ void digits3(float v, float inv, int& d1, int& d2, in
 template <int PRO, class Sink>
 __device__ __forceinline__ float row_digits_warp(const float* __restrict__ x, const float* __restrict__ gw,
                                                  const float* __restrict__ gb, float eps, int K, int lane,
-                                                 Sink sink) {
+                                                 Sink sink, int* s12 = nullptr) {
     const float4* xr = reinterpret_cast<const float4*>(x);
     const int K4 = K >> 2;
     float mu = 0.0f, rstd = 1.0f;
@@ -139,6 +144,7 @@ __device__ __forceinline__ float row_digits_warp(const float* __restrict__ x, co
     }
     amax = warp_max(amax);
     const float inv = amax > 0.0f ? 127.0f / amax : 0.0f;
+    int sum1 = 0, sum2 = 0;
     for (int k = lane; k < K4; k += 32) {
         const float4 v = normed(k);
         const float e[4] = {v.x, v.y, v.z, v.w};
@@ -147,13 +153,51 @@ __device__ __forceinline__ float row_digits_warp(const float* __restrict__ x, co
         for (int j = 0; j < 4; ++j) {
             int a, b, c;
             digits3(e[j], inv, a, b, c);
+            sum1 += abs(a);
+            sum2 += abs(b);
             p1 |= (static_cast<uint32_t>(a) & 0xffu) << (8 * j);
             p2 |= (static_cast<uint32_t>(b) & 0xffu) << (8 * j);
             p3 |= (static_cast<uint32_t>(c) & 0xffu) << (8 * j);
         }
         sink(k, p1, p2, p3);
     }
+    if (s12) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            sum1 += __shfl_xor_sync(0xffffffffu, sum1, o);
+            sum2 += __shfl_xor_sync(0xffffffffu, sum2, o);
+        }
+        s12[0] = sum1;
+        s12[1] = sum2;
+    }
     return amax / 127.0f;
+}
+
+// One logit from the three exact digit-product sums: s_n s_b (A0 + (A1 + A2 / 254) / 254), every
+// f32 operation rounded on its own (no contraction), so that the head and the refine kernel of
+// the int8 head give the same bits for the same sums.
+__device__ __forceinline__ float digit_logit(int a0, int a1, int a2, float sn, float sb) {
+    const float u = __fadd_rn(static_cast<float>(a1), __fmul_rn(static_cast<float>(a2), 1.0f / 254.0f));
+    const float w = __fadd_rn(static_cast<float>(a0), __fmul_rn(u, 1.0f / 254.0f));
+    return __fmul_rn(__fmul_rn(sn, sb), w);
+}
+
+// Bound on |exact - coarse| of the int8 head, where coarse uses only the embedding row's first
+// digit: the dropped terms are s_n s_b (D1.E2 / 254 + (D1.E3 + D2.E2) / 254^2) with every
+// embedding digit in [-127, 127], so their magnitude is at most
+// s_n s_b (127 / 254 (1 + 1 / 254) S1 + 127 / 254^2 S2), S1 = sum |D1|, S2 = sum |D2| of the
+// hidden row; 0.502 and 0.002 cover the two coefficients (0.50197, 0.00197), and the last term
+// covers the f32 rounding of both logits (a few ulps each).
+__device__ __forceinline__ float int8_head_bound(float sn, float sb, int s1, int s2, float coarse) {
+    const float b = sn * sb * (0.502f * static_cast<float>(s1) + 0.002f * static_cast<float>(s2));
+    return b * 1.001f + 4.0e-6f * fabsf(coarse) + 1.0e-30f;
+}
+
+// Value of an argmax key (the inverse of argmax_key's order-preserving transform).
+__device__ __forceinline__ float argmax_key_value(unsigned long long k) {
+    uint32_t u = static_cast<uint32_t>(k >> 32);
+    u = (u & 0x80000000u) ? (u & 0x7fffffffu) : ~u;
+    return __uint_as_float(u);
 }
 
 // Digit planes of rows of a row-major f32 matrix: out[p][r][k], scale[r]. One warp per
@@ -162,7 +206,8 @@ template <int PRO>
 __global__ void __launch_bounds__(128) k_rowprep_digits(const float* __restrict__ x, int x_ld,
                                                         const float* __restrict__ gw, const float* __restrict__ gb,
                                                         float eps, int K, int rows, long long plane_stride,
-                                                        int8_t* __restrict__ out, float* __restrict__ scale) {
+                                                        int8_t* __restrict__ out, float* __restrict__ scale,
+                                                        int* __restrict__ sums) {
     pdl_launch_dependents();
     pdl_wait();
     const int lane = threadIdx.x & 31;
@@ -171,13 +216,21 @@ __global__ void __launch_bounds__(128) k_rowprep_digits(const float* __restrict_
     uint32_t* o1 = reinterpret_cast<uint32_t*>(out + static_cast<long long>(r) * K);
     uint32_t* o2 = reinterpret_cast<uint32_t*>(out + plane_stride + static_cast<long long>(r) * K);
     uint32_t* o3 = reinterpret_cast<uint32_t*>(out + 2 * plane_stride + static_cast<long long>(r) * K);
+    int s12[2];
     const float sc = row_digits_warp<PRO>(x + static_cast<long long>(r) * x_ld, gw, gb, eps, K, lane,
                                           [&](int k4, uint32_t p1, uint32_t p2, uint32_t p3) {
                                               o1[k4] = p1;
                                               o2[k4] = p2;
                                               o3[k4] = p3;
-                                          });
-    if (lane == 0) scale[r] = sc;
+                                          },
+                                          s12);
+    if (lane == 0) {
+        scale[r] = sc;
+        if (sums) {
+            sums[2 * r] = s12[0];
+            sums[2 * r + 1] = s12[1];
+        }
+    }
 }
 
 // ---- tcgen05 / TMEM primitives ----------------------------------------------------
@@ -260,9 +313,15 @@ __device__ __forceinline__ void tmem_ld_wait() {
 // final norm (PRO_LN / PRO_RMS) with which this kernel makes them itself.
 constexpr int kHeadXExternal = -1;
 
-template <int BT, int XPRO>
+// WD: embedding digits streamed and multiplied, 3 (the exact head) or 1 (the int8 head: coarse
+// logits from the first digit, the per-row int8 quantisation of the embedding, plus the bound
+// that selects the candidates k_head_refine recomputes exactly).
+template <int BT, int XPRO, int WD>
 __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_constant__ HeadArgs A, int NS) {
     static_assert(BT == 16 || BT == 32, "batch tile");
+    static_assert(WD == 1 || WD == 3, "embedding digits");
+    static_assert(WD == 3 || XPRO == kHeadXExternal, "the int8 head reads the hidden planes k_rowprep_digits made");
+    constexpr int kStage = WD * kHeadPlaneBox;
     constexpr int ACC = 3 * BT;                           // TMEM columns of one accumulator set
     constexpr uint32_t TCOLS = BT == 16 ? 128 : 256;      // two sets, power of two
     constexpr uint32_t IDESC = idesc_i8(BT);
@@ -272,13 +331,14 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
     extern __shared__ unsigned char head_smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(head_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    unsigned char* ring = smem;                                             // NS x 48 KB
-    unsigned char* sx = smem + static_cast<size_t>(NS) * kHeadStageBytes;   // 3 x xplane
+    unsigned char* ring = smem;                                             // NS stages
+    unsigned char* sx = smem + static_cast<size_t>(NS) * kStage;            // 3 x xplane
     __shared__ __align__(8) uint64_t full[kHeadMaxStages], empty[kHeadMaxStages];
     __shared__ __align__(8) uint64_t tfull[2], tempty[2], bar_x, bar_done;
     __shared__ uint32_t s_tmem;
     __shared__ unsigned long long s_key[BT];
     __shared__ float s_xs[BT];
+    __shared__ int s_sum1[BT], s_sum2[BT];
     __shared__ int s_fail, s_last;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -319,10 +379,10 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
     auto issue = [&](int it) {
         const int jb = c0 + (it / nch) * cps;
         const int c = it % nch;
-        unsigned char* dst = ring + static_cast<size_t>(it % NS) * kHeadStageBytes;
-        mbar_arrive_expect_tx(&full[it % NS], kHeadStageBytes);
+        unsigned char* dst = ring + static_cast<size_t>(it % NS) * kStage;
+        mbar_arrive_expect_tx(&full[it % NS], kStage);
 #pragma unroll
-        for (int p = 0; p < 3; ++p)
+        for (int p = 0; p < WD; ++p)
             tma_load_2d(dst + p * kHeadPlaneBox, &A.wmap, c * kHeadKC, p * A.V + jb * kHeadRows, &full[it % NS]);
     };
     int n_issued = 0;
@@ -332,7 +392,13 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
     pdl_wait();
 
     if (XPRO == kHeadXExternal) {
-        if (tid < BT) s_xs[tid] = tid < nb ? A.xscale[b0 + tid] : 0.0f;
+        if (tid < BT) {
+            s_xs[tid] = tid < nb ? A.xscale[b0 + tid] : 0.0f;
+            if (WD == 1) {
+                s_sum1[tid] = tid < nb ? A.xsum[2 * (b0 + tid)] : 0;
+                s_sum2[tid] = tid < nb ? A.xsum[2 * (b0 + tid) + 1] : 0;
+            }
+        }
     } else {
         // the hidden planes in the swizzled K-major layout the MMA reads: zero first (rows past
         // the batch, columns past K), then one warp per row writes its digits
@@ -394,22 +460,30 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
                     break;
                 }
                 tc_fence_after();
-                const unsigned char* st = ring + static_cast<size_t>(stage) * kHeadStageBytes;
+                const unsigned char* st = ring + static_cast<size_t>(stage) * kStage;
 #pragma unroll
                 for (int s = 0; s < kHeadKC / 32; ++s) {
-                    // six digit products, grouped by weight into three accumulators
-                    const uint64_t w1 = smem_desc_sw128(st) + 2 * s, w2 = smem_desc_sw128(st + kHeadPlaneBox) + 2 * s,
-                                   w3 = smem_desc_sw128(st + 2 * kHeadPlaneBox) + 2 * s;
+                    const uint64_t w1 = smem_desc_sw128(st) + 2 * s;
                     const unsigned char* xc = sx + c * BT * 128;
                     const uint64_t x1 = smem_desc_sw128(xc) + 2 * s, x2 = smem_desc_sw128(xc + xplane) + 2 * s,
                                    x3 = smem_desc_sw128(xc + 2 * xplane) + 2 * s;
                     const uint32_t first = (c == 0 && s == 0) ? 0u : 1u;
-                    umma_i8(dacc, w1, x1, IDESC, first);
-                    umma_i8(dacc + BT, w1, x2, IDESC, first);
-                    umma_i8(dacc + BT, w2, x1, IDESC, 1u);
-                    umma_i8(dacc + 2 * BT, w1, x3, IDESC, first);
-                    umma_i8(dacc + 2 * BT, w2, x2, IDESC, 1u);
-                    umma_i8(dacc + 2 * BT, w3, x1, IDESC, 1u);
+                    if (WD == 3) {
+                        // six digit products, grouped by weight into three accumulators
+                        const uint64_t w2 = smem_desc_sw128(st + kHeadPlaneBox) + 2 * s,
+                                       w3 = smem_desc_sw128(st + 2 * kHeadPlaneBox) + 2 * s;
+                        umma_i8(dacc, w1, x1, IDESC, first);
+                        umma_i8(dacc + BT, w1, x2, IDESC, first);
+                        umma_i8(dacc + BT, w2, x1, IDESC, 1u);
+                        umma_i8(dacc + 2 * BT, w1, x3, IDESC, first);
+                        umma_i8(dacc + 2 * BT, w2, x2, IDESC, 1u);
+                        umma_i8(dacc + 2 * BT, w3, x1, IDESC, 1u);
+                    } else {
+                        // the embedding's first digit against the hidden row's three
+                        umma_i8(dacc, w1, x1, IDESC, first);
+                        umma_i8(dacc + BT, w1, x2, IDESC, first);
+                        umma_i8(dacc + 2 * BT, w1, x3, IDESC, first);
+                    }
                 }
                 umma_commit(&empty[stage]);   // stage free once these MMAs have read it
             }
@@ -449,11 +523,12 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
 #pragma unroll
                 for (int b = 0; b < BT; ++b) {
                     if (b >= nb) break;
-                    const float u = static_cast<float>(a1[b]) + static_cast<float>(a2[b]) * (1.0f / 254.0f);
-                    const float w = static_cast<float>(a0[b]) + u * (1.0f / 254.0f);
-                    const float y = __fmul_rn(sn * s_xs[b], w);
+                    const float y = digit_logit(a0[b], a1[b], a2[b], sn, s_xs[b]);
                     if (A.logits) A.logits[static_cast<long long>(b0 + b) * A.V + n] = y;
-                    const unsigned long long key = argmax_key(y, n);
+                    // the exact head ranks the logits; the int8 head ranks each logit's lower
+                    // bound, whose maximum is the candidates' threshold
+                    const float r = WD == 3 ? y : y - int8_head_bound(sn, s_xs[b], s_sum1[b], s_sum2[b], y);
+                    const unsigned long long key = argmax_key(r, n);
                     best[b] = key > best[b] ? key : best[b];
                 }
             }
@@ -491,6 +566,10 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
         __threadfence();
         for (int b = tid; b < A.B; b += kHeadThreads) {
             const unsigned long long k = atomicExch(&A.keys[b], 0ull);
+            if (WD == 1) {
+                A.thr[b] = (k == 0ull) ? -INFINITY : argmax_key_value(k);
+                continue;
+            }
             const int idx = (k == 0ull) ? 0 : argmax_key_index(k);
             if (A.argmax_out) A.argmax_out[b] = idx;
             if (A.last_tok) A.last_tok[A.meta->slot[b]] = idx;
@@ -501,32 +580,147 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
 
 // ---------------------------------------------------------------- host side
 
-inline size_t head_tc_smem(int K, int bt, int ns) {
+inline size_t head_tc_smem(int K, int bt, int ns, int wd = 3) {
     const int nch = (K + kHeadKC - 1) / kHeadKC;
-    return 1024 + size_t(ns) * kHeadStageBytes + size_t(3) * nch * bt * 128;
+    return 1024 + size_t(ns) * wd * kHeadPlaneBox + size_t(3) * nch * bt * 128;
 }
 // stages that fit next to the hidden planes (0: the head does not fit)
-inline int head_tc_stages(int K, int bt) {
+inline int head_tc_stages(int K, int bt, int wd = 3) {
     if (K % 16 != 0 || K > kHeadMaxK) return 0;
-    for (int ns = kHeadMaxStages; ns >= 2; --ns)
-        if (head_tc_smem(K, bt, ns) <= size_t(227 * 1024 - 1024)) return ns;   // room for static smem
+    for (int ns = wd == 1 ? kHeadMaxStagesW1 : kHeadMaxStages; ns >= 2; --ns)
+        if (head_tc_smem(K, bt, ns, wd) <= size_t(227 * 1024 - 1024)) return ns;   // room for static smem
     return 0;
 }
 
 template <int PRO>
 cudaError_t rowprep_digits_launch(const float* x, int x_ld, const float* gw, const float* gb, float eps, int K,
-                                  int rows, long long plane_stride, int8_t* out, float* scale, bool pdl,
+                                  int rows, long long plane_stride, int8_t* out, float* scale, int* sums, bool pdl,
                                   cudaStream_t st);
 // pro: the final norm when the head kernel makes the hidden planes itself (batches up to
 // 16), kHeadXExternal when k_rowprep_digits made them
 cudaError_t head_tc_launch(int num_sms, const HeadArgs& a, int pro, cudaStream_t st);
+// The int8 head: coarse logits and thresholds (k_head_tc with one embedding digit, hidden
+// planes from k_rowprep_digits), candidate selection, exact refine and the greedy pick.
+// cand holds B * V ints; ncand and counter are zero between launches.
+cudaError_t head_int8_launch(int num_sms, const HeadArgs& a, const int8_t* wdig, const int8_t* xdig, int* cand,
+                             int* ncand, int* refine_counter, cudaStream_t st);
 inline bool head_tc_makes_planes(int B) { return B <= 16; }
 
 #ifdef DEC_HEAD_TC_DEFINE
 
+// ---- int8 head: candidates and their exact logits ----------------------------------
+
+// Candidates of the int8 head: every n whose coarse logit plus its bound reaches the row's
+// threshold (the largest lower bound). The exact logit of every n is within the bound of its
+// coarse one, so every n that can hold the exact maximum (ties included) is a candidate.
+// Appended as b * V + n to `cand` (capacity B * V), counted in *ncand.
+__global__ void __launch_bounds__(256) k_head_select(const float* __restrict__ logits, const float* __restrict__ wscale,
+                                                     const float* __restrict__ xscale, const int* __restrict__ xsum,
+                                                     const float* __restrict__ thr, int V, int* __restrict__ cand,
+                                                     int* __restrict__ ncand) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int b = blockIdx.y;
+    const float sb = xscale[b], t = thr[b];
+    const int s1 = xsum[2 * b], s2 = xsum[2 * b + 1];
+    const int lane = threadIdx.x & 31;
+    for (int n0 = blockIdx.x * blockDim.x; n0 < V; n0 += gridDim.x * blockDim.x) {
+        const int n = n0 + threadIdx.x;
+        bool hit = false;
+        if (n < V) {
+            const float y = logits[static_cast<long long>(b) * V + n];
+            hit = y + int8_head_bound(__ldg(wscale + n), sb, s1, s2, y) >= t;
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, hit);
+        if (m == 0u) continue;
+        int base = 0;
+        if (lane == 0) base = atomicAdd(ncand, __popc(m));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (hit) cand[base + __popc(m & ((1u << lane) - 1u))] = b * V + n;
+    }
+}
+
+// Exact logits of the candidates (one warp each, the exact head's digit products summed with
+// dp4a and combined by digit_logit: the same bits as the three-digit head), written over the
+// coarse ones, then the greedy pick among them; the last CTA writes the picks and resets.
+__global__ void __launch_bounds__(256) k_head_refine(const int8_t* __restrict__ wdig, const float* __restrict__ wscale,
+                                                     const int8_t* __restrict__ xdig, const float* __restrict__ xscale,
+                                                     long long wplane, long long xplane, int V, int K, int B,
+                                                     const int* __restrict__ cand, int* __restrict__ ncand,
+                                                     float* __restrict__ logits, unsigned long long* __restrict__ keys,
+                                                     int* __restrict__ counter, int* __restrict__ argmax_out,
+                                                     int* __restrict__ last_tok, const StepMeta* __restrict__ meta) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nw = (gridDim.x * blockDim.x) >> 5;
+    const int total = *ncand;
+    for (int c = gw; c < total; c += nw) {
+        const int code = cand[c];
+        const int b = code / V, n = code - b * V;
+        const int8_t* e1 = wdig + static_cast<long long>(n) * K;
+        const int8_t* h1 = xdig + static_cast<long long>(b) * K;
+        int a0 = 0, a1 = 0, a2 = 0;
+        for (int k = lane * 16; k < K; k += 32 * 16) {
+            const int4 E1 = *reinterpret_cast<const int4*>(e1 + k);
+            const int4 E2 = *reinterpret_cast<const int4*>(e1 + wplane + k);
+            const int4 E3 = *reinterpret_cast<const int4*>(e1 + 2 * wplane + k);
+            const int4 D1 = *reinterpret_cast<const int4*>(h1 + k);
+            const int4 D2 = *reinterpret_cast<const int4*>(h1 + xplane + k);
+            const int4 D3 = *reinterpret_cast<const int4*>(h1 + 2 * xplane + k);
+            const int e1v[4] = {E1.x, E1.y, E1.z, E1.w}, e2v[4] = {E2.x, E2.y, E2.z, E2.w},
+                      e3v[4] = {E3.x, E3.y, E3.z, E3.w};
+            const int d1v[4] = {D1.x, D1.y, D1.z, D1.w}, d2v[4] = {D2.x, D2.y, D2.z, D2.w},
+                      d3v[4] = {D3.x, D3.y, D3.z, D3.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                a0 = __dp4a(e1v[j], d1v[j], a0);
+                a1 = __dp4a(e1v[j], d2v[j], a1);
+                a1 = __dp4a(e2v[j], d1v[j], a1);
+                a2 = __dp4a(e1v[j], d3v[j], a2);
+                a2 = __dp4a(e2v[j], d2v[j], a2);
+                a2 = __dp4a(e3v[j], d1v[j], a2);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+            a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+            a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+        }
+        if (lane == 0) {
+            const float y = digit_logit(a0, a1, a2, __ldg(wscale + n), xscale[b]);
+            logits[static_cast<long long>(b) * V + n] = y;
+            atomicMax(&keys[b], argmax_key(y, n));
+        }
+    }
+    __shared__ int s_last;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        s_last = (atomicAdd(counter, 1) == static_cast<int>(gridDim.x) - 1);
+    }
+    __syncthreads();
+    if (s_last) {
+        __threadfence();
+        for (int b = threadIdx.x; b < B; b += blockDim.x) {
+            const unsigned long long k = atomicExch(&keys[b], 0ull);
+            const int idx = (k == 0ull) ? 0 : argmax_key_index(k);
+            if (argmax_out) argmax_out[b] = idx;
+            if (last_tok) last_tok[meta->slot[b]] = idx;
+        }
+        if (threadIdx.x == 0) {
+            *counter = 0;
+            *ncand = 0;
+        }
+    }
+}
+
+
 template <int PRO>
 cudaError_t rowprep_digits_launch(const float* x, int x_ld, const float* gw, const float* gb, float eps, int K,
-                                  int rows, long long plane_stride, int8_t* out, float* scale, bool pdl,
+                                  int rows, long long plane_stride, int8_t* out, float* scale, int* sums, bool pdl,
                                   cudaStream_t st) {
     if (K % 4 != 0 || rows <= 0) return cudaErrorInvalidValue;
     thread_local int attr_dev = -1;
@@ -541,22 +735,24 @@ cudaError_t rowprep_digits_launch(const float* x, int x_ld, const float* gw, con
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, k_rowprep_digits<PRO>, x, x_ld, gw, gb, eps, K, rows, plane_stride, out, scale);
+    return cudaLaunchKernelEx(&cfg, k_rowprep_digits<PRO>, x, x_ld, gw, gb, eps, K, rows, plane_stride, out, scale,
+                              sums);
 }
 
-template <int BT, int XPRO>
+template <int BT, int XPRO, int WD = 3>
 cudaError_t head_tc_launch_bt(int num_sms, HeadArgs a, cudaStream_t st) {
-    const int ns = head_tc_stages(a.K, BT);
+    const int ns = head_tc_stages(a.K, BT, WD);
     if (ns == 0) return cudaErrorNotSupported;
-    const size_t smem = head_tc_smem(a.K, BT, ns);
+    const size_t smem = head_tc_smem(a.K, BT, ns, WD);
     thread_local int attr_dev = -1;   // attributes are per device; set again when it changes
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (attr_dev != dev) {
-        e = cudaFuncSetAttribute(k_head_tc<BT, XPRO>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024 - 1024);
+        e = cudaFuncSetAttribute(k_head_tc<BT, XPRO, WD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 227 * 1024 - 1024);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(k_head_tc<BT, XPRO>, cudaFuncAttributePreferredSharedMemoryCarveout,
+        e = cudaFuncSetAttribute(k_head_tc<BT, XPRO, WD>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         attr_dev = dev;
@@ -575,7 +771,7 @@ cudaError_t head_tc_launch_bt(int num_sms, HeadArgs a, cudaStream_t st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_head_tc<BT, XPRO>, a, ns);
+    return cudaLaunchKernelEx(&cfg, k_head_tc<BT, XPRO, WD>, a, ns);
 }
 
 cudaError_t head_tc_launch(int num_sms, const HeadArgs& a, int pro, cudaStream_t st) {
@@ -587,6 +783,37 @@ cudaError_t head_tc_launch(int num_sms, const HeadArgs& a, int pro, cudaStream_t
     }
     if (pro != kHeadXExternal) return cudaErrorInvalidValue;
     return head_tc_launch_bt<32, kHeadXExternal>(num_sms, a, st);
+}
+
+template <typename K, typename... Args>
+cudaError_t head_pdl_launch(K kern, dim3 grid, dim3 block, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+cudaError_t head_int8_launch(int num_sms, const HeadArgs& a, const int8_t* wdig, const int8_t* xdig, int* cand,
+                             int* ncand, int* refine_counter, cudaStream_t st) {
+    if (a.B < 1 || a.B > a.MB || a.logits == nullptr || a.thr == nullptr || a.xsum == nullptr || a.K % 16 != 0)
+        return cudaErrorInvalidValue;
+    cudaError_t e = a.B <= 16 ? head_tc_launch_bt<16, kHeadXExternal, 1>(num_sms, a, st)
+                              : head_tc_launch_bt<32, kHeadXExternal, 1>(num_sms, a, st);
+    if (e != cudaSuccess) return e;
+    const int chunks = std::max(1, std::min((a.V + 255) / 256, (2 * num_sms + a.B - 1) / a.B));
+    e = head_pdl_launch(k_head_select, dim3(chunks, a.B), dim3(256), st, static_cast<const float*>(a.logits),
+                        a.wscale, a.xscale, a.xsum, static_cast<const float*>(a.thr), a.V, cand, ncand);
+    if (e != cudaSuccess) return e;
+    return head_pdl_launch(k_head_refine, dim3(num_sms), dim3(256), st, wdig, a.wscale, xdig, a.xscale,
+                           static_cast<long long>(a.V) * a.K, static_cast<long long>(a.MB) * a.K, a.V, a.K, a.B,
+                           static_cast<const int*>(cand), ncand, a.logits, a.keys, refine_counter, a.argmax_out,
+                           a.last_tok, a.meta);
 }
 
 #endif  // DEC_HEAD_TC_DEFINE
