@@ -65,15 +65,16 @@ def step_bytes(cfg: synth.ModelConfig, lens, head: str = "exact") -> dict:
         rows = L * (6 * d + F + d)
         small = L * (3 * 2 * d) * 4                         # three LayerNorms
     else:
-        nW = L * (4 * d * d + 3 * d * F)
-        rows = L * (4 * d + 2 * F + d)
+        nW = L * (2 * d * d + 2 * cfg.kv_dim * d + 3 * d * F)
+        rows = L * (2 * d + 2 * cfg.kv_dim + 2 * F + d)
         small = L * (2 * d) * 4
     weights = nW * wb + (rows * 4 if wb == 1 else 0) + rows * 4 * (1 if cfg.is_whisper else 0) + small
     if not cfg.is_whisper:
-        weights += L * 3 * d * 4                            # q/k/v biases
+        weights += L * (d + 2 * cfg.kv_dim) * 4             # q/k/v biases
     head = V * d * 4 if head == "exact" else V * d + V * 4
-    self_kv = sum(L * (int(n) + 1) * d * 2 * 4 for n in lens)
-    kv_write = B * L * d * 2 * 4
+    kvd = cfg.kv_dim
+    self_kv = sum(L * (int(n) + 1) * kvd * 2 * 4 for n in lens)
+    kv_write = B * L * kvd * 2 * 4
     cross = B * L * cfg.enc_len * d * 2 * 4 if cfg.is_whisper else 0
     logits = B * V * 4
     emb = B * d * 4 * (2 if cfg.is_whisper else 1)
@@ -178,8 +179,8 @@ class GpuWorkload:
                     enc = torch.from_numpy(synth.encoder_hidden(cfg, s, seed)).cuda()
                     self.dec.prefill(s, [], enc)
                 g.manual_seed(seed * 100003 + s)
-                k = torch.randn((cfg.n_layers, n, cfg.d_model), device="cuda", generator=g)
-                v = torch.randn((cfg.n_layers, n, cfg.d_model), device="cuda", generator=g)
+                k = torch.randn((cfg.n_layers, n, cfg.kv_dim), device="cuda", generator=g)
+                v = torch.randn((cfg.n_layers, n, cfg.kv_dim), device="cuda", generator=g)
                 self.dec.kv_append(s, 0, n, k, v)
                 del k, v
         # the first step feeds one seeded token per stream; later steps continue greedily

@@ -70,6 +70,11 @@ enum { DEC_PROJ_F32 = 0, DEC_PROJ_W8A8 = 1, DEC_PROJ_W8A32 = 2 };
  *   rope_theta  RoPE base (qwen2), e.g. 1e6.
  *   max_slots   number of independent streams the handle holds caches for.
  *   max_cache_len  rows per stream and layer in the self-attention cache.
+ *   n_kv_heads  K/V heads (grouped-query attention, qwen2 only; [focr] native kv-lane
+ *               mapping: query head h reads K/V head h / (n_heads / n_kv_heads));
+ *               must divide n_heads; 0 means one K/V head per query head. The K and
+ *               V projections are [n_kv_heads * 64, d] and the caches hold n_kv_heads
+ *               heads.
  *   head_fmt    DEC_HEAD_EXACT: the tied head on the f32 embedding (three-digit
  *               exact-integer split, 3 bytes per weight). DEC_HEAD_INT8_REFINE
  *               ([focr] `LmHead` int8 arm, `got_lm_head`: int8 per-row head, then an
@@ -97,6 +102,7 @@ typedef struct dec_config {
     int32_t max_slots;
     int32_t max_cache_len;
     int32_t head_fmt;
+    int32_t n_kv_heads;
 } dec_config;
 
 /*
@@ -218,7 +224,7 @@ dec_status dec_set_prefill_chunk(dec_handle* h, int32_t rows);
  * Write rows [start_pos, start_pos + n_rows) of every layer's self-attention
  * K and V for `slot` and set the slot length to start_pos + n_rows
  * ([focr] `Qwen2KvCache::seed`). k and v are device f32 [n_layers, n_rows,
- * n_heads * 64], token-major (already rotated K for qwen2). Requires
+ * kv heads * 64], token-major (already rotated K for qwen2). Requires
  * start_pos <= the slot's current length (no holes). Rows are copied bit for bit.
  * Whisper slots still need dec_prefill (n_tokens may be 0) for cross K/V.
  */
@@ -302,7 +308,7 @@ dec_status dec_slot_len(const dec_handle* h, int32_t slot, int32_t* len);
 
 /*
  * Copy rows [start, start + n) of layer `layer`'s self-attention K and V of
- * `slot` into device buffers k_out, v_out (f32 [n, n_heads * 64], token-major).
+ * `slot` into device buffers k_out, v_out (f32 [n, kv heads * 64], token-major).
  * Rows at or beyond the slot length hold whatever was last written there.
  */
 dec_status dec_kv_read(dec_handle* h, int32_t slot, int32_t layer, int32_t start, int32_t n,

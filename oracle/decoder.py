@@ -282,17 +282,17 @@ def argmax_first(logits: np.ndarray) -> int:
 class StreamState:
     """One stream's decode state: per-layer self K/V rows and static cross K/V.
 
-    Self caches are token-major [max_len, H*dh] f32 per layer, holding post-RoPE
+    Self caches are token-major [max_len, kv heads * dh] f32 per layer, holding post-RoPE
     K (qwen2) and V ([focr] `Qwen2KvCache`; [cera] `WhisperDecoderKVCache`).
     Cross K/V [enc_len, d] f32 per layer are computed once from the encoder
     hidden states ([cera] `precompute_cross_attention`).
     """
 
-    def __init__(self, n_layers: int, d: int, max_len: int):
+    def __init__(self, n_layers: int, kv_dim: int, max_len: int):
         self.n = 0
         self.max_len = max_len
-        self.k = [np.zeros((max_len, d), dtype=F32) for _ in range(n_layers)]
-        self.v = [np.zeros((max_len, d), dtype=F32) for _ in range(n_layers)]
+        self.k = [np.zeros((max_len, kv_dim), dtype=F32) for _ in range(n_layers)]
+        self.v = [np.zeros((max_len, kv_dim), dtype=F32) for _ in range(n_layers)]
         self.xk: Optional[List[np.ndarray]] = None
         self.xv: Optional[List[np.ndarray]] = None
 
@@ -393,7 +393,7 @@ class OracleDecoder:
 
     def new_state(self, enc_hidden: Optional[np.ndarray] = None) -> StreamState:
         cfg = self.cfg
-        st = StreamState(cfg.n_layers, cfg.d_model, self.max_len)
+        st = StreamState(cfg.n_layers, cfg.kv_dim, self.max_len)
         if cfg.is_whisper:
             if enc_hidden is None:
                 raise ValueError("whisper stream needs encoder hidden states")
@@ -425,18 +425,22 @@ class OracleDecoder:
         return x
 
     def _self_attention(self, l, q, row_states, row_slots):
-        """Per row: attend cache rows 0..row_slots[r] of its own stream (all heads)."""
+        """Per row: attend cache rows 0..row_slots[r] of its own stream (all heads). With
+        grouped K/V heads, query head h attends K/V head h // (H / H_kv) ([focr] native
+        kv-lane mapping of grouped-query attention)."""
         cfg = self.cfg
-        H, dh = cfg.n_heads, cfg.head_dim
+        H, dh, Hkv = cfg.n_heads, cfg.head_dim, cfg.kv_heads
+        group = H // Hkv
         ctx = np.empty_like(q)
         views = {}
         for r in range(len(row_slots)):
             st = row_states[r]
             if id(st) not in views:
                 top = max(sl for s2, sl in zip(row_states, row_slots) if s2 is st) + 1
-                views[id(st)] = (
-                    np.ascontiguousarray(st.k[l][:top].astype(F64).reshape(top, H, dh).transpose(1, 0, 2)),
-                    np.ascontiguousarray(st.v[l][:top].astype(F64).reshape(top, H, dh).transpose(1, 0, 2)))
+                kh = st.k[l][:top].astype(F64).reshape(top, Hkv, dh).transpose(1, 0, 2)
+                vh = st.v[l][:top].astype(F64).reshape(top, Hkv, dh).transpose(1, 0, 2)
+                views[id(st)] = (np.ascontiguousarray(np.repeat(kh, group, axis=0)),
+                                 np.ascontiguousarray(np.repeat(vh, group, axis=0)))
             kh, vh = views[id(st)]
             n = row_slots[r] + 1
             ctx[r] = _attend_heads(q[r].reshape(H, dh).astype(F64), kh[:, :n], vh[:, :n]).astype(F32).reshape(-1)
@@ -467,7 +471,7 @@ class OracleDecoder:
             for r in range(R):
                 c, s = rope_cos_sin(int(positions[r]), cfg.rope_theta, dh)
                 q[r] = apply_rope_neox(q[r].reshape(H, dh), c, s).reshape(-1)
-                k[r] = apply_rope_neox(k[r].reshape(H, dh), c, s).reshape(-1)
+                k[r] = apply_rope_neox(k[r].reshape(cfg.kv_heads, dh), c, s).reshape(-1)
         for r in range(R):
             row_states[r].k[l][row_slots[r]] = k[r]
             row_states[r].v[l][row_slots[r]] = v[r]

@@ -71,10 +71,19 @@ class ModelConfig:
     proj_fmt: str         # PROJ_F32 | PROJ_W8A8 | PROJ_W8A32
     norm_eps: float
     rope_theta: float = 0.0
+    n_kv_heads: int = 0   # grouped-query attention: K/V heads (0: one per query head)
 
     @property
     def is_whisper(self) -> bool:
         return self.family == "whisper"
+
+    @property
+    def kv_heads(self) -> int:
+        return self.n_kv_heads or self.n_heads
+
+    @property
+    def kv_dim(self) -> int:
+        return self.kv_heads * self.head_dim
 
     @property
     def qkv_bias(self) -> bool:
@@ -149,6 +158,14 @@ MODELS: Dict[str, ModelConfig] = {
     "mid_qwen2": _m(name="mid_qwen2", family="qwen2", n_layers=2, d_model=896, n_heads=14,
                     head_dim=64, d_ff=2432, vocab=1009, max_pos=32768, enc_len=0,
                     proj_fmt=PROJ_W8A8, norm_eps=1e-6, rope_theta=1e6),
+    # Grouped-query attention (two query heads per K/V head, and seven as in Qwen2-0.5B's
+    # 14 query / 2 K/V heads at d 896).
+    "tiny_qwen2_gqa": _m(name="tiny_qwen2_gqa", family="qwen2", n_layers=2, d_model=256, n_heads=4,
+                         head_dim=64, d_ff=352, vocab=1009, max_pos=32768, enc_len=0,
+                         proj_fmt=PROJ_W8A8, norm_eps=1e-6, rope_theta=1e6, n_kv_heads=2),
+    "mid_qwen2_gqa": _m(name="mid_qwen2_gqa", family="qwen2", n_layers=2, d_model=896, n_heads=14,
+                        head_dim=64, d_ff=2432, vocab=1009, max_pos=32768, enc_len=0,
+                        proj_fmt=PROJ_W8A8, norm_eps=1e-6, rope_theta=1e6, n_kv_heads=2),
 }
 
 WORKLOADS: Dict[str, Workload] = {
@@ -197,6 +214,10 @@ WORKLOADS: Dict[str, Workload] = {
                                cache_init="prefill", lens_lo=1, lens_hi=10, steps=3),
     "mid_qwen2_b9": Workload("mid_qwen2_b9", MODELS["mid_qwen2"], batch=9, max_cache_len=64,
                              cache_init="prefill", lens_lo=1, lens_hi=10, steps=3),
+    "tiny_qwen2_gqa_b3": Workload("tiny_qwen2_gqa_b3", MODELS["tiny_qwen2_gqa"], batch=3, max_cache_len=96,
+                                  cache_init="prefill", lens_lo=1, lens_hi=40, steps=4),
+    "mid_qwen2_gqa_b9": Workload("mid_qwen2_gqa_b9", MODELS["mid_qwen2_gqa"], batch=9, max_cache_len=200,
+                                 cache_init="kv_seed", lens_lo=1, lens_hi=150, steps=3),
     "small_qwen2_kv_b5": Workload("small_qwen2_kv_b5", MODELS["small_qwen2"], batch=5,
                                   max_cache_len=700, cache_init="kv_seed", lens_lo=1,
                                   lens_hi=600, steps=4),
@@ -247,8 +268,8 @@ _LAYER_TENSORS = {
 
 
 def _proj_shape(cfg: ModelConfig, name: str):
-    d, f = cfg.d_model, cfg.d_ff
-    return {"q": (d, d), "k": (d, d), "v": (d, d), "o": (d, d),
+    d, f, kv = cfg.d_model, cfg.d_ff, cfg.kv_dim
+    return {"q": (d, d), "k": (kv, d), "v": (kv, d), "o": (d, d),
             "xq": (d, d), "xk": (d, d), "xv": (d, d), "xo": (d, d),
             "fc1": (f, d), "fc2": (d, f),
             "gate": (f, d), "up": (f, d), "down": (d, f)}[name]
@@ -329,9 +350,9 @@ def cache_lens(wl: Workload, seed: int = 0) -> np.ndarray:
 
 
 def seed_kv(cfg: ModelConfig, stream: int, layer: int, n_rows: int, seed: int = 0):
-    """N(0,1) K and V rows [n_rows, H*head_dim] f32 for one stream and layer (token-major)."""
+    """N(0,1) K and V rows [n_rows, kv heads * head_dim] f32 for one stream and layer (token-major)."""
     g = _rng(seed, _TAG_KV, stream, layer)
-    dm = cfg.n_heads * cfg.head_dim
+    dm = cfg.kv_dim
     k = g.standard_normal((n_rows, dm), dtype=np.float32)
     v = g.standard_normal((n_rows, dm), dtype=np.float32)
     return k, v

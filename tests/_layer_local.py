@@ -111,8 +111,8 @@ class LayerLocal:
                     k, v = torch.from_numpy(np.stack(ks)).cuda(), torch.from_numpy(np.stack(vs)).cuda()
                 else:
                     g.manual_seed(1000 + s)
-                    k = torch.randn((cfg.n_layers, n, cfg.d_model), device="cuda", generator=g)
-                    v = torch.randn((cfg.n_layers, n, cfg.d_model), device="cuda", generator=g)
+                    k = torch.randn((cfg.n_layers, n, cfg.kv_dim), device="cuda", generator=g)
+                    v = torch.randn((cfg.n_layers, n, cfg.kv_dim), device="cuda", generator=g)
                 self.gpu.kv_append(s, 0, n, k, v)
                 del k, v
             if s in self.sample:
@@ -161,7 +161,7 @@ class LayerLocal:
         gk, gv = [], []
         for s in self.sample:
             n = int(self.lens[s])
-            k = torch.empty((cfg.n_layers, n + 1, cfg.d_model), device="cuda")
+            k = torch.empty((cfg.n_layers, n + 1, cfg.kv_dim), device="cuda")
             v = torch.empty_like(k)
             for l in range(cfg.n_layers):
                 self.gpu.kv_read(s, l, 0, n + 1, k[l], v[l])

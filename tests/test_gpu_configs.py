@@ -62,8 +62,8 @@ def _setup(wl, sample, seed=0):
                     sts[s] = st
             else:
                 g.manual_seed(1000 + s)
-                k = torch.randn((cfg.n_layers, n, cfg.d_model), device="cuda", generator=g)
-                v = torch.randn((cfg.n_layers, n, cfg.d_model), device="cuda", generator=g)
+                k = torch.randn((cfg.n_layers, n, cfg.kv_dim), device="cuda", generator=g)
+                v = torch.randn((cfg.n_layers, n, cfg.kv_dim), device="cuda", generator=g)
                 gpu.kv_append(s, 0, n, k, v)
                 del k, v
     torch.cuda.synchronize()

@@ -186,8 +186,8 @@ def test_c4_sampled_streams_32_greedy_steps_match_oracle():
             states[s] = st
         else:
             g.manual_seed(1000 + s)
-            dec.kv_append(s, 0, n, torch.randn((cfg.n_layers, n, cfg.d_model), device="cuda", generator=g),
-                          torch.randn((cfg.n_layers, n, cfg.d_model), device="cuda", generator=g))
+            dec.kv_append(s, 0, n, torch.randn((cfg.n_layers, n, cfg.kv_dim), device="cuda", generator=g),
+                          torch.randn((cfg.n_layers, n, cfg.kv_dim), device="cuda", generator=g))
     first = [int(t) for t in synth.token_ids(cfg, 4242, wl.batch, 0)]
     am = torch.empty(wl.batch, dtype=torch.int32, device="cuda")
     gpu_ids = {s: [] for s in sample}

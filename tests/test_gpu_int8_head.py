@@ -33,8 +33,8 @@ def _pair(wl, seed=0):
                 d.prefill(s, toks, enc)
         else:
             g.manual_seed(1000 + s)
-            k = torch.randn((cfg.n_layers, n, cfg.d_model), device="cuda", generator=g)
-            v = torch.randn((cfg.n_layers, n, cfg.d_model), device="cuda", generator=g)
+            k = torch.randn((cfg.n_layers, n, cfg.kv_dim), device="cuda", generator=g)
+            v = torch.randn((cfg.n_layers, n, cfg.kv_dim), device="cuda", generator=g)
             for d in decs:
                 if cfg.is_whisper:
                     d.prefill(s, [], enc)

@@ -29,7 +29,8 @@ def _check(rep, whisper):
 
 @pytest.mark.parametrize("wl_name,steps", [("small_qwen2_kv_b5", 3), ("mid_qwen2_b9", 2), ("tiny_qwen2_b9", 2),
                                            ("tiny_whisper_b3", 2), ("mid_whisper_b9", 2),
-                                           ("tiny_whisper_w8a32_b9", 2)])
+                                           ("tiny_whisper_w8a32_b9", 2), ("mid_qwen2_gqa_b9", 2),
+                                           ("tiny_qwen2_gqa_b3", 2)])
 def test_layer_local_small_models(wl_name, steps):
     wl = synth.workload(wl_name)
     rep = run_layer_local(wl_name, steps, sample=list(range(wl.batch)))

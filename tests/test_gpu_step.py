@@ -35,8 +35,8 @@ def _run(wl_name, steps=None, seed=0):
     for slot, st in enumerate(p.states):
         for l in range(cfg.n_layers):
             n = st.n
-            ko = torch.empty((n, cfg.d_model), device="cuda")
-            vo = torch.empty((n, cfg.d_model), device="cuda")
+            ko = torch.empty((n, cfg.kv_dim), device="cuda")
+            vo = torch.empty((n, cfg.kv_dim), device="cuda")
             p.gpu.kv_read(slot, l, 0, n, ko, vo)
             torch.cuda.synchronize()
             env_k = max([0.0] + [float(np.abs(sts[slot].k[l][:n] - st.k[l][:n]).max()) for _, sts in p.jrefs])
@@ -51,7 +51,8 @@ def _run(wl_name, steps=None, seed=0):
 
 @pytest.mark.parametrize("wl_name", ["tiny_whisper_b3", "tiny_qwen2_b3", "tiny_whisper_w8a32_b3",
                                      "small_qwen2_kv_b5", "tiny_whisper_b9", "tiny_whisper_w8a32_b9",
-                                     "tiny_qwen2_b9", "mid_whisper_b9", "mid_qwen2_b9"])
+                                     "tiny_qwen2_b9", "mid_whisper_b9", "mid_qwen2_b9", "tiny_qwen2_gqa_b3",
+                                     "mid_qwen2_gqa_b9"])
 def test_step_matches_oracle(wl_name):
     _run(wl_name)
 
@@ -229,7 +230,7 @@ def test_chunked_prefill_equals_row_by_row_prefill(name, n):
         dec.set_prefill_chunk(chunk)
         lg = torch.empty(cfg.vocab, device="cuda")
         dec.prefill(1, toks, enc, lg)
-        k = torch.empty((cfg.n_layers, n, cfg.d_model), device="cuda")
+        k = torch.empty((cfg.n_layers, n, cfg.kv_dim), device="cuda")
         v = torch.empty_like(k)
         for l in range(cfg.n_layers):
             dec.kv_read(1, l, 0, n, k[l], v[l])

@@ -409,3 +409,44 @@ def test_tie_log_and_flips():
     assert int(q1[0, 3]) == -4 and int(q0[0, 3]) == -3   # -3.4999 rounds to -3; flipped to -4
     diff = q1.astype(int) != q0.astype(int)
     assert int(diff.sum()) == 2
+
+
+@pytest.mark.parametrize("name", ["tiny_qwen2_gqa", "mid_qwen2_gqa"])
+def test_grouped_query_attention_equals_mha_with_repeated_kv_heads(name):
+    """Grouped-query attention (query head h reads K/V head h // group) is the multi-head
+    decoder whose K and V projections repeat each K/V head's rows `group` times: same codes,
+    scales and biases row for row, so every logit is the same bits. A wrong head mapping
+    (h % H_kv instead of h // group) breaks it."""
+    cfg_g, W = _model(name)
+    cfg_m = synth.dataclasses.replace(cfg_g, n_kv_heads=0, name=name + "_as_mha")
+    group = cfg_g.n_heads // cfg_g.kv_heads
+    Wm = copy.deepcopy(W)
+    Wm["config"] = cfg_m
+    idx = np.concatenate([np.arange(h * 64, (h + 1) * 64) for h in range(cfg_g.kv_heads) for _ in range(group)])
+    for L in Wm["layers"]:
+        for key in ("k", "v"):
+            p = L[key]
+            L[key] = {"w": p["w"][idx], "s": p["s"][idx] if p["s"] is not None else None,
+                      "b": p["b"][idx] if p["b"] is not None else None}
+    toks = list(synth.token_ids(cfg_g, 0, 7))
+    outs = []
+    for Wx in (W, Wm):
+        dec = oracle.OracleDecoder(Wx, 32)
+        st = dec.new_state(None)
+        lg = dec.prefill(st, toks)
+        _, lg2 = dec.step([st], [5], [st.n])
+        outs.append((lg, lg2))
+    np.testing.assert_array_equal(outs[0][0], outs[1][0])
+    np.testing.assert_array_equal(outs[0][1], outs[1][1])
+    # the mapping matters: interleaved repetition (head h reads K/V head h % H_kv) differs
+    idx_bad = np.concatenate([np.arange((h % cfg_g.kv_heads) * 64, (h % cfg_g.kv_heads + 1) * 64)
+                              for h in range(cfg_g.n_heads)])
+    Wb = copy.deepcopy(W)
+    Wb["config"] = cfg_m
+    for L, L0 in zip(Wb["layers"], W["layers"]):
+        for key in ("k", "v"):
+            p = L0[key]
+            L[key] = {"w": p["w"][idx_bad], "s": p["s"][idx_bad], "b": p["b"][idx_bad]}
+    dec = oracle.OracleDecoder(Wb, 32)
+    st = dec.new_state(None)
+    assert not np.array_equal(dec.prefill(st, toks), outs[0][0])

@@ -49,7 +49,8 @@ class DecConfig(C.Structure):
                 ("n_heads", C.c_int32), ("head_dim", C.c_int32), ("d_ff", C.c_int32),
                 ("vocab", C.c_int32), ("max_pos", C.c_int32), ("enc_len", C.c_int32),
                 ("proj_fmt", C.c_int32), ("norm_eps", C.c_float), ("rope_theta", C.c_float),
-                ("max_slots", C.c_int32), ("max_cache_len", C.c_int32), ("head_fmt", C.c_int32)]
+                ("max_slots", C.c_int32), ("max_cache_len", C.c_int32), ("head_fmt", C.c_int32),
+                ("n_kv_heads", C.c_int32)]
 
 
 class DecProj(C.Structure):
@@ -152,7 +153,8 @@ class Decoder:
         self._lib = lib()
         c = DecConfig(FAMILY[cfg.family], cfg.n_layers, cfg.d_model, cfg.n_heads, cfg.head_dim,
                       cfg.d_ff, cfg.vocab, cfg.max_pos, cfg.enc_len, PROJ[cfg.proj_fmt],
-                      float(cfg.norm_eps), float(cfg.rope_theta), max_slots, max_cache_len, HEAD[head])
+                      float(cfg.norm_eps), float(cfg.rope_theta), max_slots, max_cache_len, HEAD[head],
+                      int(getattr(cfg, "n_kv_heads", 0)))
         self.cfg = cfg
         self.max_slots = max_slots
         self.max_cache_len = max_cache_len

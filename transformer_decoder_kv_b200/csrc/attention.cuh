@@ -52,6 +52,7 @@ struct AttnArgs {
     int stages;            // shared-memory pipeline stages (1..3); 0: 3
     int* err;              // device status word
     int drop_first_copy;   // test hook: CTA (0, 0, 0) never issues its first tile's copies
+    int kv_group;          // query heads per K/V head (grouped-query attention); 0 or 1: one each
 };
 
 // `drop`: announce the bytes but issue no copy, so that the tile's wait can only run out
@@ -110,8 +111,10 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
     const int t1 = min(ntiles, t0 + tps);
     if (t0 >= t1) return;
 
-    const float* Kb = a.k + slot * a.slot_stride + static_cast<long long>(h) * a.ld * kHeadDim;
-    const float* Vb = a.v + slot * a.slot_stride + static_cast<long long>(h) * a.ld * kHeadDim;
+    // grouped-query attention: query head h reads the K/V of head h / kv_group
+    const int hk = a.kv_group > 1 ? h / a.kv_group : h;
+    const float* Kb = a.k + slot * a.slot_stride + static_cast<long long>(hk) * a.ld * kHeadDim;
+    const float* Vb = a.v + slot * a.slot_stride + static_cast<long long>(hk) * a.ld * kHeadDim;
 
     // tiles before the first one holding a row this step writes can be fetched before the
     // dependency wait (a prompt chunk writes rows fresh..len of its slot in one step)

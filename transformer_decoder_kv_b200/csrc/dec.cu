@@ -208,6 +208,9 @@ dec_status upload(dec_handle* h, T** dst, const void* src, size_t bytes) {
     } while (0)
 
 size_t wbytes(const dec_config& c) { return c.proj_fmt == DEC_PROJ_F32 ? 4 : 1; }
+// K/V heads (grouped-query attention) and the K/V width
+int kv_heads(const dec_config& c) { return c.n_kv_heads > 0 ? c.n_kv_heads : c.n_heads; }
+int kv_width(const dec_config& c) { return kv_heads(c) * 64; }
 
 // Upload a projection: weights [out, in], optional scales [out] and bias [out].
 dec_status upload_proj(dec_handle* h, const dec_proj& p, int out, int in, bool want_bias, void** w, float** s,
@@ -226,21 +229,26 @@ dec_status upload_proj(dec_handle* h, const dec_proj& p, int out, int in, bool w
 // Fused q|k|v panel [3d, d] with its scales and biases (franken_ocr decoder_qwen2.rs, `concat_qkv`).
 dec_status upload_qkv(dec_handle* h, const dec_layer_weights& L, LayerDev& D) {
     const dec_config& c = h->cfg;
-    const int d = c.d_model;
-    const size_t wb = wbytes(c), mat = size_t(d) * d * wb;
+    const int d = c.d_model, kvd = kv_width(c);
+    const size_t wb = wbytes(c);
     const dec_proj* ps[3] = {&L.q, &L.k, &L.v};
+    const int rows[3] = {d, kvd, kvd};        // q [d, d], k and v [kv width, d]
+    const int off[3] = {0, d, d + kvd};       // first row of each section in the panel
     for (int i = 0; i < 3; ++i) {
         if (!ps[i]->w) return fail(h, DEC_EINVAL, "missing q/k/v weights");
         if (c.proj_fmt != DEC_PROJ_F32 && !ps[i]->scale) return fail(h, DEC_EINVAL, "missing q/k/v scales");
         if (!ps[i]->bias) return fail(h, DEC_EINVAL, "missing q/k/v bias");
     }
-    DEC_TRY(dalloc(h, &D.wqkv, 3 * mat));
-    DEC_TRY(dalloc(h, &D.bqkv, size_t(3) * d * 4));
-    if (c.proj_fmt != DEC_PROJ_F32) DEC_TRY(dalloc(h, &D.sqkv, size_t(3) * d * 4));
+    const int n_rows = d + 2 * kvd;
+    DEC_TRY(dalloc(h, &D.wqkv, size_t(n_rows) * d * wb));
+    DEC_TRY(dalloc(h, &D.bqkv, size_t(n_rows) * 4));
+    if (c.proj_fmt != DEC_PROJ_F32) DEC_TRY(dalloc(h, &D.sqkv, size_t(n_rows) * 4));
     for (int i = 0; i < 3; ++i) {
-        DEC_CUDA(h, cudaMemcpy(static_cast<char*>(D.wqkv) + i * mat, ps[i]->w, mat, cudaMemcpyHostToDevice));
-        DEC_CUDA(h, cudaMemcpy(D.bqkv + i * d, ps[i]->bias, size_t(d) * 4, cudaMemcpyHostToDevice));
-        if (D.sqkv) DEC_CUDA(h, cudaMemcpy(D.sqkv + i * d, ps[i]->scale, size_t(d) * 4, cudaMemcpyHostToDevice));
+        DEC_CUDA(h, cudaMemcpy(static_cast<char*>(D.wqkv) + size_t(off[i]) * d * wb, ps[i]->w,
+                               size_t(rows[i]) * d * wb, cudaMemcpyHostToDevice));
+        DEC_CUDA(h, cudaMemcpy(D.bqkv + off[i], ps[i]->bias, size_t(rows[i]) * 4, cudaMemcpyHostToDevice));
+        if (D.sqkv)
+            DEC_CUDA(h, cudaMemcpy(D.sqkv + off[i], ps[i]->scale, size_t(rows[i]) * 4, cudaMemcpyHostToDevice));
     }
     return DEC_OK;
 }
@@ -250,6 +258,10 @@ dec_status validate_config(const dec_config& c) {
     if (c.family != DEC_FAMILY_WHISPER && c.family != DEC_FAMILY_QWEN2) return bad("unknown family");
     if (c.head_dim != 64) return bad("head_dim must be 64");
     if (c.n_heads < 1 || c.d_model != c.n_heads * 64) return bad("d_model must equal n_heads * 64");
+    if (c.n_kv_heads < 0 || (c.n_kv_heads > 0 && c.n_heads % c.n_kv_heads != 0))
+        return bad("n_kv_heads must divide n_heads (0: one K/V head per query head)");
+    if (c.family == DEC_FAMILY_WHISPER && c.n_kv_heads > 0 && c.n_kv_heads != c.n_heads)
+        return bad("grouped-query attention is a qwen2 option");
     if (c.n_layers < 1) return bad("n_layers must be >= 1");
     if (c.d_ff < 16 || c.d_ff % 16) return bad("d_ff must be a positive multiple of 16");
     if (c.vocab < 1) return bad("vocab must be >= 1");
@@ -559,7 +571,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
         g.norm_w = L.n1w;
         g.norm_b = L.n1b;
         g.K = d;
-        g.N = 3 * d;
+        g.N = d + 2 * kv_width(c);
         g.W = L.wqkv;
         g.scale = L.sqkv;
         g.bias = L.bqkv;
@@ -570,6 +582,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
         g.slot_stride = h->self_slot_stride;
         g.ld = c.max_cache_len;
         g.d = d;
+        g.kvd = kv_width(c);
         if (c.family == DEC_FAMILY_WHISPER) {
             DEC_TRY((gemv_whisper<PRO_LN, EPI_QKV, MAP_ADJ>(h, g, st, &L.m_qkv)));
         } else {
@@ -586,6 +599,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
         at.slot_stride = h->self_slot_stride;
         at.ld = c.max_cache_len;
         at.H = H;
+        at.kv_group = H / kv_heads(c);
         at.mode = ATTN_SELF;
         at.meta = h->dmeta;
         at.out = h->ctx;
@@ -636,6 +650,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             at.slot_stride = h->cross_slot_stride;
             at.ld = c.enc_len;
             at.mode = ATTN_CROSS;
+            at.kv_group = 1;
             at.n_fixed = c.enc_len;
             DEC_TRY(attention(h, at, B, c.enc_len, h->tps_cross, st));
             DEC_TRY(phase_mark(h, st, l, DEC_PHASE_CROSS_ATTN));
@@ -943,20 +958,21 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
         for (int l = 0; l < L && ts == DEC_OK; ++l) {
             LayerDev& D = h->layers[l];
             if (wh) {
-                ts = make_wmap(h, &D.m_qkv, D.wqkv, 3 * d, d, f32w);
+                ts = make_wmap(h, &D.m_qkv, D.wqkv, d + 2 * kv_width(c), d, f32w);
                 if (ts == DEC_OK) ts = make_wmap(h, &D.m_o, D.wo, d, d, f32w);
                 if (ts == DEC_OK) ts = make_wmap(h, &D.m_xq, D.wxq, d, d, f32w);
                 if (ts == DEC_OK) ts = make_wmap(h, &D.m_xo, D.wxo, d, d, f32w);
                 if (ts == DEC_OK) ts = make_wmap(h, &D.m_1, D.w1, F, d, f32w);
                 if (ts == DEC_OK) ts = make_wmap(h, &D.m_2, D.w2, d, F, f32w);
             } else {
-                DEC_TRY(dalloc(h, &D.wqkv_p, size_t(3) * d * d));
+                const int qkv_rows = d + 2 * kv_width(c);
+                DEC_TRY(dalloc(h, &D.wqkv_p, size_t(qkv_rows) * d));
                 DEC_TRY(dalloc(h, &D.wgu, size_t(2) * F * d));
                 DEC_CUDA(h, tc_rows_permute(MAP_ROPE, static_cast<int8_t*>(D.wqkv_p),
-                                            static_cast<const int8_t*>(D.wqkv), nullptr, 3 * d, d, 0));
+                                            static_cast<const int8_t*>(D.wqkv), nullptr, qkv_rows, d, 0));
                 DEC_CUDA(h, tc_rows_permute(MAP_DUAL, static_cast<int8_t*>(D.wgu), static_cast<const int8_t*>(D.wg),
                                             static_cast<const int8_t*>(D.wu), 2 * F, d, 0));
-                ts = make_wmap(h, &D.m_qkv, D.wqkv_p, 3 * d, d, false);
+                ts = make_wmap(h, &D.m_qkv, D.wqkv_p, qkv_rows, d, false);
                 if (ts == DEC_OK) ts = make_wmap(h, &D.m_o, D.wo, d, d, false);
                 if (ts == DEC_OK) ts = make_wmap(h, &D.m_1, D.wgu, 2 * F, d, false);
                 if (ts == DEC_OK) ts = make_wmap(h, &D.m_2, D.wd, d, F, false);
@@ -996,7 +1012,7 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
         DEC_CUDA(h, cudaDeviceSynchronize());
     }
     // caches
-    h->self_slot_stride = (long long)H * c.max_cache_len * 64;
+    h->self_slot_stride = (long long)kv_heads(c) * c.max_cache_len * 64;
     h->self_layer_stride = h->self_slot_stride * c.max_slots;
     const size_t self_bytes = size_t(L) * h->self_layer_stride * 4;
     DEC_TRY(dalloc(h, &h->kc, self_bytes));
@@ -1055,7 +1071,7 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
             cl = std::max(cl, tc_counters(p, MB));
         };
         need_f32(c.vocab, d, 4);
-        const int shapes[4][2] = {{3 * d, d}, {d, d}, {F, d}, {d, F}};
+        const int shapes[4][2] = {{d + 2 * kv_width(c), d}, {d, d}, {F, d}, {d, F}};
         for (const auto& sh : shapes) {
             if (!wh) {
                 need_i8(sh[0] == F ? 2 * F : sh[0], sh[1]);
@@ -1219,9 +1235,9 @@ dec_status dec_kv_append(dec_handle* h, int32_t slot, int32_t start_pos, int32_t
     if (n_rows > 0) {
         dim3 grid(n_rows, c.n_layers);
         k_kv_copy<<<grid, 128, 0, st>>>(h->kc, const_cast<float*>(k), 0, h->self_layer_stride, h->self_slot_stride,
-                                        slot, c.max_cache_len, start_pos, n_rows, c.d_model, 0);
+                                        slot, c.max_cache_len, start_pos, n_rows, kv_width(c), 0);
         k_kv_copy<<<grid, 128, 0, st>>>(h->vc, const_cast<float*>(v), 0, h->self_layer_stride, h->self_slot_stride,
-                                        slot, c.max_cache_len, start_pos, n_rows, c.d_model, 0);
+                                        slot, c.max_cache_len, start_pos, n_rows, kv_width(c), 0);
         DEC_CUDA(h, cudaGetLastError());
     }
     h->slot_len[slot] = start_pos + n_rows;
@@ -1241,9 +1257,9 @@ dec_status dec_kv_read(dec_handle* h, int32_t slot, int32_t layer, int32_t start
     if (n > 0) {
         dim3 grid(n, 1);
         k_kv_copy<<<grid, 128, 0, st>>>(h->kc, k_out, 1, h->self_layer_stride, h->self_slot_stride, slot,
-                                        c.max_cache_len, start, n, c.d_model, layer);
+                                        c.max_cache_len, start, n, kv_width(c), layer);
         k_kv_copy<<<grid, 128, 0, st>>>(h->vc, v_out, 1, h->self_layer_stride, h->self_slot_stride, slot,
-                                        c.max_cache_len, start, n, c.d_model, layer);
+                                        c.max_cache_len, start, n, kv_width(c), layer);
         DEC_CUDA(h, cudaGetLastError());
     }
     return DEC_OK;

@@ -64,7 +64,8 @@ struct GemvArgs {
     float* vc;
     long long slot_stride;
     int ld;                  // cache rows per (slot, head)
-    int d;                   // model width (q/k/v section size)
+    int d;                   // model width (the q section's size)
+    int kvd;                 // K and V section size (kv heads x 64; d without grouped heads)
     const float2* rope;      // [pos][32] (cos, sin), null = no RoPE
     // EPI_HEAD
     unsigned long long* keys;  // [B] packed argmax keys, zero between launches
@@ -529,7 +530,8 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
                         if (primary && live && (r & 1) == 0)
                             a.out[static_cast<long long>(gb) * a.out_ld + n] = __fmul_rn(silu_f(y), yp);
                     } else if (EPI == EPI_QKV) {
-                        const int sec = n / a.d, within = n - sec * a.d;
+                        const int sec = n < a.d ? 0 : (n < a.d + a.kvd ? 1 : 2);
+                        const int within = n - (sec == 0 ? 0 : (sec == 1 ? a.d : a.d + a.kvd));
                         const int hh = within >> 6, i = within & 63;
                         float val = y;
                         if (a.rope != nullptr && sec < 2) {

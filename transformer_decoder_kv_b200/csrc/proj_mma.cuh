@@ -298,7 +298,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_proj_mma(const __grid_consta
         } else if (EPI == EPI_GELU) {
             a.out[static_cast<long long>(gb) * a.out_ld + n] = gelu_tanh_f(y);
         } else if (EPI == EPI_QKV) {
-            const int sec = n / a.d, within = n - sec * a.d;
+            const int sec = n < a.d ? 0 : (n < a.d + a.kvd ? 1 : 2);
+            const int within = n - (sec == 0 ? 0 : (sec == 1 ? a.d : a.d + a.kvd));
             const int hh = within >> 6, i = within & 63;
             if (sec == 0) {
                 a.out[static_cast<long long>(gb) * a.out_ld + within] = y;

@@ -243,8 +243,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
             const float bn = (EPI != EPI_SWIGLU && a.bias != nullptr && row_live) ? a.bias[n] : 0.0f;
             int sec = 0, within = n, hh = 0, col = 0;
             if (EPI == EPI_QKV) {
-                sec = n / a.d;
-                within = n - sec * a.d;
+                sec = n < a.d ? 0 : (n < a.d + a.kvd ? 1 : 2);
+                within = n - (sec == 0 ? 0 : (sec == 1 ? a.d : a.d + a.kvd));
                 hh = within >> 6;
                 col = within & 63;
             }
