@@ -34,14 +34,17 @@ int main() {
     struct Model {
         int d, F, V;
         int kind;   // 0 f32 whisper, 1 W8A32 whisper, 2 W8A8 qwen2
-    } models[] = {{384, 1536, 51865, 0},  {512, 2048, 51865, 0}, {1024, 2816, 151936, 2}, {1280, 5120, 51866, 1},
-                  {128, 384, 1031, 0},    {192, 320, 997, 1},    {128, 352, 1009, 2},     {256, 704, 4099, 2},
-                  {256, 2048, 1031, 0},   {896, 2432, 1009, 2}};
+        int kvd;    // K/V width (grouped-query attention); 0: d
+    } models[] = {{384, 1536, 51865, 0, 0},  {512, 2048, 51865, 0, 0}, {1024, 2816, 151936, 2, 0},
+                  {1280, 5120, 51866, 1, 0}, {128, 384, 1031, 0, 0},   {192, 320, 997, 1, 0},
+                  {128, 352, 1009, 2, 0},    {256, 704, 4099, 2, 0},   {256, 2048, 1031, 0, 0},
+                  {896, 2432, 1009, 2, 0},   {256, 352, 1009, 2, 128}, {896, 2432, 1009, 2, 128},
+                  {896, 4864, 151936, 2, 128}};
     for (const auto& m : models) {
         std::vector<Shape> shapes;
-        const int d = m.d, F = m.F;
+        const int d = m.d, F = m.F, kvd = m.kvd ? m.kvd : m.d;
         if (m.kind == 2) {
-            shapes = {{3 * d, d, 0}, {d, d, 0}, {2 * F, d, 0}, {d, F, 0}};
+            shapes = {{d + 2 * kvd, d, 0}, {d, d, 0}, {2 * F, d, 0}, {d, F, 0}};
         } else {
             const int e = m.kind == 0 ? 4 : 1;
             shapes = {{3 * d, d, e}, {d, d, e}, {F, d, e}, {d, F, e}};
