@@ -75,6 +75,16 @@ enum { DEC_PROJ_F32 = 0, DEC_PROJ_W8A8 = 1, DEC_PROJ_W8A32 = 2 };
  *               must divide n_heads; 0 means one K/V head per query head. The K and
  *               V projections are [n_kv_heads * 64, d] and the caches hold n_kv_heads
  *               heads.
+ *   kv_page_rows  0: each slot owns max_cache_len rows of self-attention cache.
+ *               16, 32 or 64: a paged cache ([wa-dec] `PagedDecoderKVCache`,
+ *               `forward_one_paged`): a pool of kv_pages pages of that many rows
+ *               (per layer, K and V) shared by all slots through a page table; a slot
+ *               takes pages as it grows (dec_step, dec_prefill, dec_kv_append) and
+ *               returns them when it is prefilled again, shortened by dec_kv_append,
+ *               released (dec_release_slot) or reset. A call that would need more
+ *               pages than are free returns DEC_ENOMEM before any work.
+ *               max_cache_len still bounds each slot's length.
+ *   kv_pages    pages in the pool (kv_page_rows > 0).
  *   head_fmt    DEC_HEAD_EXACT: the tied head on the f32 embedding (three-digit
  *               exact-integer split, 3 bytes per weight). DEC_HEAD_INT8_REFINE
  *               ([focr] `LmHead` int8 arm, `got_lm_head`: int8 per-row head, then an
@@ -103,6 +113,8 @@ typedef struct dec_config {
     int32_t max_cache_len;
     int32_t head_fmt;
     int32_t n_kv_heads;
+    int32_t kv_page_rows;
+    int32_t kv_pages;
 } dec_config;
 
 /*
@@ -285,7 +297,8 @@ dec_status dec_get_config(const dec_handle* h, dec_config* out);
  * output) or `max_new` tokens, or when its next row would overflow the cache
  * or the position range; its slot is refilled from the queue before the next
  * step. A stream's tokens are those it would get alone (the step's per-stream
- * arithmetic does not depend on the batch).
+ * arithmetic does not depend on the batch). A retired stream's slot is released
+ * (dec_release_slot), so a paged cache returns its pages to the pool at once.
  *   reqs        host [n_reqs]; prompt host int32 [n_prompt] (n_prompt >= 1);
  *               enc_hidden device f32 [enc_len, d] for whisper, NULL for qwen2
  *   tokens_out  host int32 [n_reqs, stride]: request r's tokens in row r
@@ -302,6 +315,13 @@ typedef struct dec_request {
 } dec_request;
 dec_status dec_generate(dec_handle* h, const dec_request* reqs, int32_t n_reqs, int32_t max_active,
                         int32_t* tokens_out, int32_t stride, int32_t* n_out, void* stream);
+
+/* Empty `slot`: its length becomes 0 and, with a paged cache, its pages return to the
+ * pool. The slot needs dec_prefill or dec_kv_append before its next step. */
+dec_status dec_release_slot(dec_handle* h, int32_t slot);
+
+/* Free pages in the paged cache's pool (0 for a dense cache). */
+dec_status dec_kv_pages_free(const dec_handle* h, int32_t* pages);
 
 /* Current length (cached rows) of `slot` as tracked by the handle. */
 dec_status dec_slot_len(const dec_handle* h, int32_t slot, int32_t* len);

@@ -34,7 +34,7 @@ def test_binding_sets_signatures_without_gpu():
     lib = binding.load_library()
     assert lib.dec_last_error(None) == b""
     # a create call with a bad config is rejected on the host before touching the GPU
-    cfg = binding.DecConfig(7, 1, 128, 2, 64, 256, 10, 10, 0, 0, 1e-5, 0.0, 1, 8, 0, 0)
+    cfg = binding.DecConfig(7, 1, 128, 2, 64, 256, 10, 10, 0, 0, 1e-5, 0.0, 1, 8, 0, 0, 0, 0)
     w = binding.DecWeights()
     h = ctypes.c_void_p()
     st = lib.dec_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h))

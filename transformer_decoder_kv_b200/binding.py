@@ -28,7 +28,7 @@ EXPORTS = ["dec_create", "dec_destroy", "dec_last_error", "dec_prefill", "dec_kv
            "dec_step_host", "dec_slot_len", "dec_kv_read", "dec_hidden", "dec_set_layer_trace", "dec_sync",
            "dec_reset", "dec_set_wait_limit", "dec_debug_inject", "dec_debug_fail_alloc", "dec_step_kernels",
            "dec_next_tokens", "dec_get_config", "dec_generate", "dec_set_prefill_chunk",
-           "dec_set_phase_timing", "dec_phase_times",
+           "dec_set_phase_timing", "dec_phase_times", "dec_release_slot", "dec_kv_pages_free",
            "dec_attention_workspace_size", "dec_attention", "dec_attention_plan", "dec_attention_noalloc",
            "dec_i8_dot"]
 I8_PATH = {"dp4a": 0, "tcgen05": 1}
@@ -50,7 +50,7 @@ class DecConfig(C.Structure):
                 ("vocab", C.c_int32), ("max_pos", C.c_int32), ("enc_len", C.c_int32),
                 ("proj_fmt", C.c_int32), ("norm_eps", C.c_float), ("rope_theta", C.c_float),
                 ("max_slots", C.c_int32), ("max_cache_len", C.c_int32), ("head_fmt", C.c_int32),
-                ("n_kv_heads", C.c_int32)]
+                ("n_kv_heads", C.c_int32), ("kv_page_rows", C.c_int32), ("kv_pages", C.c_int32)]
 
 
 class DecProj(C.Structure):
@@ -97,6 +97,8 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
         "dec_set_layer_trace": (C.c_int, [vp, vp]),
         "dec_sync": (C.c_int, [vp, vp]),
         "dec_reset": (C.c_int, [vp]),
+        "dec_release_slot": (C.c_int, [vp, i32]),
+        "dec_kv_pages_free": (C.c_int, [vp, pi32]),
         "dec_set_prefill_chunk": (C.c_int, [vp, i32]),
         "dec_set_phase_timing": (C.c_int, [vp, i32]),
         "dec_phase_times": (C.c_int, [vp, i32, C.POINTER(C.c_float), pi32, pi32, pi32]),
@@ -149,12 +151,13 @@ def _ptr(a) -> Optional[int]:
 class Decoder:
     """One handle of the CUDA decoder (dec_create ... dec_destroy)."""
 
-    def __init__(self, cfg, weights: dict, max_slots: int, max_cache_len: int, head: str = "exact"):
+    def __init__(self, cfg, weights: dict, max_slots: int, max_cache_len: int, head: str = "exact",
+                 kv_page_rows: int = 0, kv_pages: int = 0):
         self._lib = lib()
         c = DecConfig(FAMILY[cfg.family], cfg.n_layers, cfg.d_model, cfg.n_heads, cfg.head_dim,
                       cfg.d_ff, cfg.vocab, cfg.max_pos, cfg.enc_len, PROJ[cfg.proj_fmt],
                       float(cfg.norm_eps), float(cfg.rope_theta), max_slots, max_cache_len, HEAD[head],
-                      int(getattr(cfg, "n_kv_heads", 0)))
+                      int(getattr(cfg, "n_kv_heads", 0)), kv_page_rows, kv_pages)
         self.cfg = cfg
         self.max_slots = max_slots
         self.max_cache_len = max_cache_len
@@ -297,6 +300,14 @@ class Decoder:
 
     def set_prefill_chunk(self, rows: int):
         self._check(self._lib.dec_set_prefill_chunk(self._h, rows))
+
+    def release_slot(self, slot: int):
+        self._check(self._lib.dec_release_slot(self._h, slot))
+
+    def kv_pages_free(self) -> int:
+        n = C.c_int32(0)
+        self._check(self._lib.dec_kv_pages_free(self._h, C.byref(n)))
+        return int(n.value)
 
     def reset(self):
         self._check(self._lib.dec_reset(self._h))

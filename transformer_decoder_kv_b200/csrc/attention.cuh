@@ -53,18 +53,35 @@ struct AttnArgs {
     int* err;              // device status word
     int drop_first_copy;   // test hook: CTA (0, 0, 0) never issues its first tile's copies
     int kv_group;          // query heads per K/V head (grouped-query attention); 0 or 1: one each
+    KvMap kv;              // ATTN_SELF with a paged cache: where each row lives (table null: dense)
 };
 
+// Rows [64 tile, 64 tile + 64) of one (slot, K/V head), clipped to n: one bulk copy each of K
+// and V when the rows are contiguous (dense cache, Kb/Vb the head's first row), else one per
+// page they span (paged cache, pages of 16, 32 or 64 rows).
 // `drop`: announce the bytes but issue no copy, so that the tile's wait can only run out
 // (the host-side fault injection of the failure-path tests; no memory is touched).
-__device__ __forceinline__ void attn_issue(float* sK, float* sV, uint64_t* bar, const float* Kb,
-                                           const float* Vb, int tile, int n, bool drop = false) {
+__device__ __forceinline__ void attn_issue(float* sK, float* sV, uint64_t* bar, const AttnArgs& a, const float* Kb,
+                                           const float* Vb, int slot, int hk, int tile, int n, bool drop = false) {
     const int rows = min(kAttnTile, n - tile * kAttnTile);
     const uint32_t bytes = static_cast<uint32_t>(rows) * kHeadDim * sizeof(float);
     mbar_arrive_expect_tx(bar, 2 * bytes);
     if (drop) return;
-    bulk_g2s(sK, Kb + static_cast<long long>(tile) * kAttnTile * kHeadDim, bytes, bar);
-    bulk_g2s(sV, Vb + static_cast<long long>(tile) * kAttnTile * kHeadDim, bytes, bar);
+    if (a.kv.table == nullptr) {
+        bulk_g2s(sK, Kb + static_cast<long long>(tile) * kAttnTile * kHeadDim, bytes, bar);
+        bulk_g2s(sV, Vb + static_cast<long long>(tile) * kAttnTile * kHeadDim, bytes, bar);
+        return;
+    }
+    for (int r0 = 0; r0 < rows;) {
+        int page, pr;
+        kv_page_of(a.kv, slot, tile * kAttnTile + r0, page, pr);
+        const int chunk = min(rows - r0, a.kv.page_rows - pr);
+        const long long off = kv_page_off(a.kv, page, hk, pr);
+        const uint32_t cb = static_cast<uint32_t>(chunk) * kHeadDim * sizeof(float);
+        bulk_g2s(sK + r0 * kHeadDim, a.k + off, cb, bar);
+        bulk_g2s(sV + r0 * kHeadDim, a.v + off, cb, bar);
+        r0 += chunk;
+    }
 }
 
 // Internal linkage: each translation unit that launches it carries its own copy.
@@ -125,16 +142,16 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
         for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
         for (; pre < NS && t0 + pre < t1 && t0 + pre < first_new_tile; ++pre)
-            attn_issue(sK + pre * kAttnTile * kHeadDim, sV + pre * kAttnTile * kHeadDim, &bars[pre], Kb,
-                       Vb, t0 + pre, n, drop && pre == 0);
+            attn_issue(sK + pre * kAttnTile * kHeadDim, sV + pre * kAttnTile * kHeadDim, &bars[pre], a, Kb, Vb,
+                       slot, hk, t0 + pre, n, drop && pre == 0);
     }
     pdl_launch_dependents();
     if (a.mode != ATTN_OP) pdl_wait();
     if (tid < kHeadDim) sq[tid] = a.q[b * a.q_bstride + h * kHeadDim + tid];
     if (tid == 0) {
         for (int i = pre; i < NS && t0 + i < t1; ++i)
-            attn_issue(sK + i * kAttnTile * kHeadDim, sV + i * kAttnTile * kHeadDim, &bars[i], Kb,
-                       Vb, t0 + i, n, drop && i == 0);
+            attn_issue(sK + i * kAttnTile * kHeadDim, sV + i * kAttnTile * kHeadDim, &bars[i], a, Kb, Vb, slot,
+                       hk, t0 + i, n, drop && i == 0);
     }
     __syncthreads();
 
@@ -212,8 +229,8 @@ static __global__ void __launch_bounds__(kAttnThreads) k_attention(const AttnArg
         }
         __syncthreads();
         if (tid == 0 && t + NS < t1)
-            attn_issue(sK + stage * kAttnTile * kHeadDim, sV + stage * kAttnTile * kHeadDim,
-                       &bars[stage], Kb, Vb, t + NS, n);
+            attn_issue(sK + stage * kAttnTile * kHeadDim, sV + stage * kAttnTile * kHeadDim, &bars[stage], a, Kb, Vb,
+                       slot, hk, t + NS, n);
     }
 
     // merge the four warps

@@ -15,6 +15,35 @@ constexpr int kMaxBatch = 128;
 // A bounded device wait gives up after this many nanoseconds and reports DEC_ETIMEOUT.
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
+// Where self-attention K/V rows live. Row `row` of K/V head `hh` of stream slot `slot` starts at
+// float offset ((page * heads + hh) * page_rows + r) * 64 of a layer's cache. A paged cache
+// (16, 32 or 64 rows per page) takes page = table[slot * pages_per_slot + row / page_rows] and
+// r = row % page_rows; a dense cache is the same layout with one page per slot (page = slot,
+// page_rows = the slot's rows, r = row).
+struct KvMap {
+    const int* table;     // paged: physical page of each (slot, logical page); null: dense
+    int page_rows;
+    int pages_per_slot;
+    int heads;            // K/V heads
+};
+
+__host__ __device__ __forceinline__ long long kv_page_off(const KvMap& m, int page, int hh, int r) {
+    return ((static_cast<long long>(page) * m.heads + hh) * m.page_rows + r) * kHeadDim;
+}
+__device__ __forceinline__ void kv_page_of(const KvMap& m, int slot, int row, int& page, int& r) {
+    if (m.table) {
+        page = m.table[slot * m.pages_per_slot + row / m.page_rows];
+        r = row % m.page_rows;
+    } else {
+        page = slot;
+        r = row;
+    }
+}
+
+// Page-table entries a step writes before any kernel reads them (paged caches): the first
+// kernel of the step applies them.
+constexpr int kMaxTableUpdates = 256;
+
 // Per-step description of the batch, uploaded once per step and read by every kernel.
 struct StepMeta {
     int B;
@@ -25,6 +54,9 @@ struct StepMeta {
     int len[kMaxBatch];    // cached rows before this step; the new row goes here
     int fresh[kMaxBatch];  // first cache row of the row's slot that this step writes (len, or the
                            // chunk's first row when several rows of one slot run together)
+    int n_upd;             // page-table updates: table[upd_idx[i]] = upd_page[i]
+    int upd_idx[kMaxTableUpdates];
+    int upd_page[kMaxTableUpdates];
 };
 
 __device__ __forceinline__ unsigned long long global_ns() {

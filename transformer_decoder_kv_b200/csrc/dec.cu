@@ -98,6 +98,12 @@ struct dec_handle {
     bool head_tc_ok = false;
     std::vector<LayerDev> layers;
     float *kc = nullptr, *vc = nullptr, *xkc = nullptr, *xvc = nullptr;
+    // paged self-attention cache (page_rows > 0): a pool of pages shared by all slots and a
+    // per-slot page table; a dense cache is one page of max_cache_len rows per slot
+    int page_rows = 0, pages_per_slot = 1, n_pages = 0;
+    int* d_table = nullptr;                    // [max_slots][pages_per_slot] physical pages
+    std::vector<int> free_pages;
+    std::vector<std::vector<int>> slot_pages;
     long long self_slot_stride = 0, self_layer_stride = 0, cross_slot_stride = 0, cross_layer_stride = 0;
     int max_batch = 0;
     int max_rows = 0;                  // rows of the per-step workspaces: max(max_batch, prompt chunk)
@@ -212,6 +218,9 @@ size_t wbytes(const dec_config& c) { return c.proj_fmt == DEC_PROJ_F32 ? 4 : 1; 
 int kv_heads(const dec_config& c) { return c.n_kv_heads > 0 ? c.n_kv_heads : c.n_heads; }
 int kv_width(const dec_config& c) { return kv_heads(c) * 64; }
 
+// Where the self-attention cache rows live (see KvMap).
+KvMap self_kv_map(const dec_handle* h);
+
 // Upload a projection: weights [out, in], optional scales [out] and bias [out].
 dec_status upload_proj(dec_handle* h, const dec_proj& p, int out, int in, bool want_bias, void** w, float** s,
                        float** b, const char* name) {
@@ -270,6 +279,9 @@ dec_status validate_config(const dec_config& c) {
     if (c.max_cache_len < 1) return bad("max_cache_len must be >= 1");
     if (!(c.norm_eps > 0.0f)) return bad("norm_eps must be > 0");
     if (c.head_fmt != DEC_HEAD_EXACT && c.head_fmt != DEC_HEAD_INT8_REFINE) return bad("unknown head_fmt");
+    if (c.kv_page_rows != 0 && c.kv_page_rows != 16 && c.kv_page_rows != 32 && c.kv_page_rows != 64)
+        return bad("kv_page_rows must be 0 (dense), 16, 32 or 64");
+    if (c.kv_page_rows > 0 && c.kv_pages < 1) return bad("a paged cache needs kv_pages >= 1");
     if (c.head_fmt == DEC_HEAD_INT8_REFINE &&
         (c.d_model > 4096 || static_cast<long long>(c.vocab) * DEC_MAX_BATCH >= (1LL << 31)))
         return bad("the int8 head needs d_model <= 4096 and vocab * 128 < 2^31");
@@ -558,7 +570,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
     h->phase_n = 0;
     DEC_TRY(phase_mark(h, st, -1, 0));
     DEC_CUDA(h, launch(k_embed, dim3(B), dim3(128), 0, st, (const float*)h->tok_emb, (const float*)h->pos_emb,
-                       (const StepMeta*)h->dmeta, (const int*)h->last_tok, h->x, d));
+                       (const StepMeta*)h->dmeta, (const int*)h->last_tok, h->x, d, h->d_table));
     DEC_TRY(phase_mark(h, st, -1, DEC_PHASE_EMBED));
     for (int l = 0; l < c.n_layers; ++l) {
         const LayerDev& L = h->layers[l];
@@ -579,8 +591,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
         g.out_ld = d;
         g.kc = kc;
         g.vc = vc;
-        g.slot_stride = h->self_slot_stride;
-        g.ld = c.max_cache_len;
+        g.kv = self_kv_map(h);
         g.d = d;
         g.kvd = kv_width(c);
         if (c.family == DEC_FAMILY_WHISPER) {
@@ -600,6 +611,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
         at.ld = c.max_cache_len;
         at.H = H;
         at.kv_group = H / kv_heads(c);
+        at.kv = self_kv_map(h);
         at.mode = ATTN_SELF;
         at.meta = h->dmeta;
         at.out = h->ctx;
@@ -651,6 +663,7 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
             at.ld = c.enc_len;
             at.mode = ATTN_CROSS;
             at.kv_group = 1;
+            at.kv.table = nullptr;
             at.n_fixed = c.enc_len;
             DEC_TRY(attention(h, at, B, c.enc_len, h->tps_cross, st));
             DEC_TRY(phase_mark(h, st, l, DEC_PHASE_CROSS_ATTN));
@@ -750,6 +763,55 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
     return DEC_OK;
 }
 
+KvMap self_kv_map(const dec_handle* h) {
+    KvMap m;
+    m.heads = kv_heads(h->cfg);
+    if (h->page_rows > 0) {
+        m.table = h->d_table;
+        m.page_rows = h->page_rows;
+        m.pages_per_slot = h->pages_per_slot;
+    } else {
+        m.table = nullptr;
+        m.page_rows = h->cfg.max_cache_len;
+        m.pages_per_slot = 1;
+    }
+    return m;
+}
+
+// Pages a slot needs beyond those it holds to keep `rows` rows (0 for a dense cache).
+int pages_short(const dec_handle* h, int slot, int rows) {
+    if (h->page_rows <= 0) return 0;
+    const int want = (rows + h->page_rows - 1) / h->page_rows;
+    return std::max(0, want - static_cast<int>(h->slot_pages[slot].size()));
+}
+
+// Give `slot` pages for `rows` rows, recording the table entries in m (applied on the device by
+// the step's first kernel); the caller has checked that the pool holds enough.
+void grow_slot(dec_handle* h, int slot, int rows, StepMeta& m) {
+    if (h->page_rows <= 0) return;
+    auto& pg = h->slot_pages[slot];
+    const int want = (rows + h->page_rows - 1) / h->page_rows;
+    while (static_cast<int>(pg.size()) < want) {
+        const int page = h->free_pages.back();
+        h->free_pages.pop_back();
+        m.upd_idx[m.n_upd] = slot * h->pages_per_slot + static_cast<int>(pg.size());
+        m.upd_page[m.n_upd] = page;
+        ++m.n_upd;
+        pg.push_back(page);
+    }
+}
+
+// Return the pages of `slot` beyond those `rows` rows need to the pool.
+void shrink_slot(dec_handle* h, int slot, int rows) {
+    if (h->page_rows <= 0) return;
+    auto& pg = h->slot_pages[slot];
+    const int keep = (rows + h->page_rows - 1) / h->page_rows;
+    while (static_cast<int>(pg.size()) > keep) {
+        h->free_pages.push_back(pg.back());
+        pg.pop_back();
+    }
+}
+
 // Upload the step description through the pinned ring.
 dec_status upload_meta(dec_handle* h, const StepMeta& m, cudaStream_t st) {
     const int i = h->ring;
@@ -813,6 +875,12 @@ dec_status validate_step(dec_handle* h, int B, const int32_t* slots, const int32
         m.fresh[b] = cache_lens[b];
         max_len = std::max(max_len, cache_lens[b] + 1);
     }
+    // a paged cache must have a free page for every slot whose new row starts one
+    int short_pages = 0;
+    for (int b = 0; b < B; ++b) short_pages += pages_short(h, m.slot[b], m.len[b] + 1);
+    if (short_pages > static_cast<int>(h->free_pages.size()))
+        return fail(h, DEC_ENOMEM, "KV page pool exhausted: the step needs " + std::to_string(short_pages) +
+                                       " new pages, " + std::to_string(h->free_pages.size()) + " are free");
     return DEC_OK;
 }
 
@@ -853,8 +921,10 @@ void capture_step(dec_handle* h, const std::array<long long, 5>& key, int B, int
     h->graphs[key] = {exec, kernels};
 }
 
-dec_status step_validated(dec_handle* h, const StepMeta& m, int max_len, float* logits, int* argmax,
+dec_status step_validated(dec_handle* h, StepMeta& m, int max_len, float* logits, int* argmax,
                           cudaStream_t st) {
+    m.n_upd = 0;
+    for (int b = 0; b < m.B; ++b) grow_slot(h, m.slot[b], m.len[b] + 1, m);
     DEC_TRY(upload_meta(h, m, st));
     const std::array<long long, 5> key = {m.B, (max_len + kAttnTile - 1) / kAttnTile,
                                           reinterpret_cast<long long>(logits), reinterpret_cast<long long>(argmax),
@@ -1014,6 +1084,16 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
     // caches
     h->self_slot_stride = (long long)kv_heads(c) * c.max_cache_len * 64;
     h->self_layer_stride = h->self_slot_stride * c.max_slots;
+    h->slot_pages.assign(c.max_slots, {});
+    if (c.kv_page_rows > 0) {
+        h->page_rows = c.kv_page_rows;
+        h->pages_per_slot = (c.max_cache_len + c.kv_page_rows - 1) / c.kv_page_rows;
+        h->n_pages = c.kv_pages;
+        h->self_layer_stride = (long long)c.kv_pages * kv_heads(c) * c.kv_page_rows * 64;
+        DEC_TRY(dalloc(h, &h->d_table, size_t(c.max_slots) * h->pages_per_slot * 4));
+        DEC_CUDA(h, cudaMemset(h->d_table, 0, size_t(c.max_slots) * h->pages_per_slot * 4));
+        for (int pg = c.kv_pages - 1; pg >= 0; --pg) h->free_pages.push_back(pg);   // page 0 first
+    }
     const size_t self_bytes = size_t(L) * h->self_layer_stride * 4;
     DEC_TRY(dalloc(h, &h->kc, self_bytes));
     DEC_TRY(dalloc(h, &h->vc, self_bytes));
@@ -1166,6 +1246,13 @@ dec_status dec_prefill(dec_handle* h, int32_t slot, const int32_t* tokens, int32
     }
     for (int i = 0; i < n_tokens; ++i)
         if (tokens[i] < 0 || tokens[i] >= c.vocab) return fail(h, DEC_ERANGE, "token outside [0, vocab)");
+    if (h->page_rows > 0) {
+        const int need = (n_tokens + h->page_rows - 1) / h->page_rows;
+        const int avail = static_cast<int>(h->free_pages.size() + h->slot_pages[slot].size());
+        if (need > avail)
+            return fail(h, DEC_ENOMEM, "KV page pool exhausted: the prompt needs " + std::to_string(need) +
+                                           " pages, " + std::to_string(avail) + " are available");
+    }
     DEC_TRY(check_device(h));
     if (c.family == DEC_FAMILY_WHISPER) {
         const int d = c.d_model;
@@ -1187,6 +1274,7 @@ dec_status dec_prefill(dec_handle* h, int32_t slot, const int32_t* tokens, int32
     }
     h->slot_len[slot] = 0;
     h->has_tok[slot] = 0;
+    shrink_slot(h, slot, 0);
     // The prompt runs in chunks of up to prefill_chunk rows of this one slot at consecutive
     // positions ([focr] `forward_prefill_seed`: the whole prompt in one forward): each
     // chunk is one step whose projections are m = chunk contractions and whose attention is
@@ -1203,6 +1291,7 @@ dec_status dec_prefill(dec_handle* h, int32_t slot, const int32_t* tokens, int32
             m.len[b] = i0 + b;
             m.fresh[b] = i0;
         }
+        grow_slot(h, slot, i0 + B, m);
         const bool last = i0 + B == n_tokens;
         DEC_TRY(upload_meta(h, m, st));
         const bool timing = h->phase_timing;   // prompt chunks are not phase-timed
@@ -1230,14 +1319,29 @@ dec_status dec_kv_append(dec_handle* h, int32_t slot, int32_t start_pos, int32_t
     if (start_pos < 0 || start_pos > h->slot_len[slot])
         return fail(h, DEC_ESTATE, "start_pos must be within [0, slot length]");
     if (start_pos + n_rows > c.max_cache_len) return fail(h, DEC_EOVERFLOW, "cache overflow");
+    if (pages_short(h, slot, start_pos + n_rows) > static_cast<int>(h->free_pages.size()))
+        return fail(h, DEC_ENOMEM, "KV page pool exhausted");
     DEC_TRY(check_device(h));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // pages: keep those the rows need, then add the missing ones (table entries applied on the
+    // device before the copy, a step description's worth at a time)
+    shrink_slot(h, slot, start_pos + n_rows);
+    while (pages_short(h, slot, start_pos + n_rows) > 0) {
+        StepMeta m{};
+        const int have = static_cast<int>(h->slot_pages[slot].size());
+        const int upto = std::min(start_pos + n_rows, (have + kMaxTableUpdates) * h->page_rows);
+        grow_slot(h, slot, upto, m);
+        DEC_TRY(upload_meta(h, m, st));
+        k_table_update<<<1, 256, 0, st>>>(h->dmeta, h->d_table);
+        DEC_CUDA(h, cudaGetLastError());
+    }
     if (n_rows > 0) {
         dim3 grid(n_rows, c.n_layers);
-        k_kv_copy<<<grid, 128, 0, st>>>(h->kc, const_cast<float*>(k), 0, h->self_layer_stride, h->self_slot_stride,
-                                        slot, c.max_cache_len, start_pos, n_rows, kv_width(c), 0);
-        k_kv_copy<<<grid, 128, 0, st>>>(h->vc, const_cast<float*>(v), 0, h->self_layer_stride, h->self_slot_stride,
-                                        slot, c.max_cache_len, start_pos, n_rows, kv_width(c), 0);
+        const KvMap km = self_kv_map(h);
+        k_kv_copy<<<grid, 128, 0, st>>>(h->kc, const_cast<float*>(k), 0, h->self_layer_stride, km, slot, start_pos,
+                                        n_rows, kv_width(c), 0);
+        k_kv_copy<<<grid, 128, 0, st>>>(h->vc, const_cast<float*>(v), 0, h->self_layer_stride, km, slot, start_pos,
+                                        n_rows, kv_width(c), 0);
         DEC_CUDA(h, cudaGetLastError());
     }
     h->slot_len[slot] = start_pos + n_rows;
@@ -1251,15 +1355,18 @@ dec_status dec_kv_read(dec_handle* h, int32_t slot, int32_t layer, int32_t start
     if (slot < 0 || slot >= c.max_slots || layer < 0 || layer >= c.n_layers)
         return fail(h, DEC_EINVAL, "slot or layer out of range");
     if (start < 0 || n < 0 || start + n > c.max_cache_len) return fail(h, DEC_EINVAL, "rows out of range");
+    if (h->page_rows > 0 && start + n > static_cast<int>(h->slot_pages[slot].size()) * h->page_rows)
+        return fail(h, DEC_EINVAL, "rows beyond the slot's pages");
     if (n > 0 && (!k_out || !v_out)) return fail(h, DEC_EINVAL, "null output");
     DEC_TRY(check_device(h));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (n > 0) {
         dim3 grid(n, 1);
-        k_kv_copy<<<grid, 128, 0, st>>>(h->kc, k_out, 1, h->self_layer_stride, h->self_slot_stride, slot,
-                                        c.max_cache_len, start, n, kv_width(c), layer);
-        k_kv_copy<<<grid, 128, 0, st>>>(h->vc, v_out, 1, h->self_layer_stride, h->self_slot_stride, slot,
-                                        c.max_cache_len, start, n, kv_width(c), layer);
+        const KvMap km = self_kv_map(h);
+        k_kv_copy<<<grid, 128, 0, st>>>(h->kc, k_out, 1, h->self_layer_stride, km, slot, start, n, kv_width(c),
+                                        layer);
+        k_kv_copy<<<grid, 128, 0, st>>>(h->vc, v_out, 1, h->self_layer_stride, km, slot, start, n, kv_width(c),
+                                        layer);
         DEC_CUDA(h, cudaGetLastError());
     }
     return DEC_OK;
@@ -1397,6 +1504,21 @@ dec_status dec_sync(dec_handle* h, void* stream) {
     return DEC_OK;
 }
 
+dec_status dec_release_slot(dec_handle* h, int32_t slot) {
+    if (!h) return fail(nullptr, DEC_EINVAL, "dec_release_slot: null handle");
+    if (slot < 0 || slot >= h->cfg.max_slots) return fail(h, DEC_EINVAL, "slot out of range");
+    shrink_slot(h, slot, 0);
+    h->slot_len[slot] = 0;
+    h->has_tok[slot] = 0;
+    return DEC_OK;
+}
+
+dec_status dec_kv_pages_free(const dec_handle* h, int32_t* pages) {
+    if (!h || !pages) return fail(nullptr, DEC_EINVAL, "dec_kv_pages_free: null pointer");
+    *pages = static_cast<int32_t>(h->free_pages.size());
+    return DEC_OK;
+}
+
 dec_status dec_reset(dec_handle* h) {
     if (!h) return fail(nullptr, DEC_EINVAL, "dec_reset: null handle");
     DEC_TRY(check_device(h));
@@ -1412,6 +1534,7 @@ dec_status dec_reset(dec_handle* h) {
     std::fill(h->slot_len.begin(), h->slot_len.end(), 0);
     std::fill(h->has_tok.begin(), h->has_tok.end(), 0);
     std::fill(h->has_cross.begin(), h->has_cross.end(), 0);
+    for (int s2 = 0; s2 < h->cfg.max_slots; ++s2) shrink_slot(h, s2, 0);
     h->failed = false;
     return DEC_OK;
 }

@@ -62,8 +62,7 @@ struct GemvArgs {
     // EPI_QKV
     float* kc;               // this layer's self K cache base
     float* vc;
-    long long slot_stride;
-    int ld;                  // cache rows per (slot, head)
+    KvMap kv;                // where each (slot, head, row) of the cache lives
     int d;                   // model width (the q section's size)
     int kvd;                 // K and V section size (kv heads x 64; d without grouped heads)
     const float2* rope;      // [pos][32] (cos, sin), null = no RoPE
@@ -547,10 +546,10 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
                             if (sec == 0) {
                                 a.out[static_cast<long long>(gb) * a.out_ld + within] = val;
                             } else {
-                                const int slot = a.meta->slot[gb], row = a.meta->len[gb];
+                                int page, r;
+                                kv_page_of(a.kv, a.meta->slot[gb], a.meta->len[gb], page, r);
                                 float* cache = (sec == 1) ? a.kc : a.vc;
-                                cache[slot * a.slot_stride + (static_cast<long long>(hh) * a.ld + row) * kHeadDim + i] =
-                                    val;
+                                cache[kv_page_off(a.kv, page, hh, r) + i] = val;
                             }
                         }
                     } else if (EPI == EPI_HEAD) {

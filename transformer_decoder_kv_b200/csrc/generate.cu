@@ -27,6 +27,7 @@ struct Stream {
     int emitted;   // tokens written to the request's output
     int len;       // cached rows of the slot
     int last;      // last emitted token
+    int pages;     // cache pages reserved for the stream (paged cache)
 };
 
 dec_status gen_fail(dec_status st, const std::string& msg) {
@@ -58,6 +59,17 @@ extern "C" dec_status dec_generate(dec_handle* h, const dec_request* reqs, int32
         for (int i = 0; i < q.n_prompt; ++i)
             if (q.prompt[i] < 0 || q.prompt[i] >= c.vocab) return gen_fail(DEC_ERANGE, who + "prompt token outside vocab");
     }
+    // A paged cache admits a request only while the pages of its longest possible stream
+    // (prompt + max_new rows, at most max_cache_len) fit next to those reserved by the
+    // streams already running, so no running stream can find the pool empty.
+    const int P = c.kv_page_rows;
+    auto pages_for = [&](int r) {
+        return P > 0 ? (std::min(reqs[r].n_prompt + reqs[r].max_new, c.max_cache_len) + P - 1) / P : 0;
+    };
+    for (int r = 0; r < n_reqs; ++r)
+        if (pages_for(r) > c.kv_pages && P > 0)
+            return gen_fail(DEC_ENOMEM, "request " + std::to_string(r) + " needs more cache pages than the pool has");
+    int reserved = 0;
     const int cap = std::min(std::min(max_active, c.max_slots), DEC_MAX_BATCH);
     std::vector<int> free_slots;
     for (int s = cap - 1; s >= 0; --s) free_slots.push_back(s);   // slot 0 is taken first
@@ -82,21 +94,27 @@ extern "C" dec_status dec_generate(dec_handle* h, const dec_request* reqs, int32
     std::vector<int32_t> slots, pos, toks;
     while (true) {
         // admit waiting requests into free slots
-        while (!free_slots.empty() && !pending.empty()) {
+        while (!free_slots.empty() && !pending.empty() &&
+               (P == 0 || reserved + pages_for(pending.front()) <= c.kv_pages)) {
             const int r = pending.front();
             pending.pop_front();
-            Stream a{r, free_slots.back(), 0, reqs[r].n_prompt, -1};
+            Stream a{r, free_slots.back(), 0, reqs[r].n_prompt, -1, pages_for(r)};
             free_slots.pop_back();
+            reserved += a.pages;
             st = dec_prefill(h, a.slot, reqs[r].prompt, reqs[r].n_prompt, reqs[r].enc_hidden, nullptr, stream);
             if (st != DEC_OK) return st;
             int32_t first = 0;
             st = dec_next_tokens(h, 1, &a.slot, &first, stream);
             if (st != DEC_OK) return st;
             emit(a, first);
-            if (done(a))
+            if (done(a)) {
+                st = dec_release_slot(h, a.slot);
+                if (st != DEC_OK) return st;
                 free_slots.push_back(a.slot);
-            else
+                reserved -= a.pages;
+            } else {
                 act.push_back(a);
+            }
         }
         if (act.empty()) {
             if (pending.empty()) break;
@@ -121,10 +139,14 @@ extern "C" dec_status dec_generate(dec_handle* h, const dec_request* reqs, int32
             Stream& a = act[i];
             a.len += 1;
             emit(a, toks[i]);
-            if (done(a))
+            if (done(a)) {
+                st = dec_release_slot(h, a.slot);
+                if (st != DEC_OK) return st;
                 free_slots.push_back(a.slot);
-            else
+                reserved -= a.pages;
+            } else {
                 keep.push_back(a);
+            }
         }
         act.swap(keep);
     }

@@ -9,8 +9,12 @@ namespace dec {
 // row plus learned position row; franken_ocr decoder_qwen2.rs: token row only).
 // A token of -1 in the step description means the slot's previous greedy pick.
 __global__ void k_embed(const float* __restrict__ E, const float* __restrict__ P, const StepMeta* meta,
-                        const int* __restrict__ last_tok, float* __restrict__ x, int d) {
+                        const int* __restrict__ last_tok, float* __restrict__ x, int d, int* __restrict__ table) {
     pdl_wait();
+    // page-table entries of pages this step starts (a paged cache), before any kernel of the
+    // step reads them
+    if (table && blockIdx.x == 0)
+        for (int i = threadIdx.x; i < meta->n_upd; i += blockDim.x) table[meta->upd_idx[i]] = meta->upd_page[i];
     const int b = blockIdx.x;
     if (b >= meta->B) return;
     int tok = meta->tok[b];
@@ -32,18 +36,26 @@ __global__ void k_embed(const float* __restrict__ E, const float* __restrict__ P
     pdl_launch_dependents();
 }
 
-// Token-major rows [L, n, H*64] <-> head-first cache [L][slot][H][ld][64], bit for bit.
+// Page-table entries of a step description, applied on their own (before a K/V row copy).
+__global__ void k_table_update(const StepMeta* meta, int* __restrict__ table) {
+    for (int i = threadIdx.x; i < meta->n_upd; i += blockDim.x) table[meta->upd_idx[i]] = meta->upd_page[i];
+}
+
+// Token-major rows [L, n, H*64] <-> the head-first cache (dense or paged), bit for bit.
 // dir 0: rows -> cache (KV append / seed); dir 1: cache -> rows (read back).
+// The step description's page-table updates are applied first (a paged cache).
 __global__ void k_kv_copy(float* __restrict__ cache, float* __restrict__ rows, int dir, long long layer_stride,
-                          long long slot_stride, int slot, int ld, int start, int n, int d, int layer0) {
+                          KvMap m, int slot, int start, int n, int d, int layer0) {
     const int r = blockIdx.x;        // row within [0, n)
     const int l = blockIdx.y;        // layer offset
     const long long lay = layer0 + l;
-    float* crow = cache + lay * layer_stride + slot * slot_stride;
+    int page, pr;
+    kv_page_of(m, slot, start + r, page, pr);
+    float* base = cache + lay * layer_stride;
     float* rrow = rows + (static_cast<long long>(l) * n + r) * d;
     for (int e = threadIdx.x; e < d / 4; e += blockDim.x) {
         const int col = e * 4, h = col >> 6, i = col & 63;
-        float4* c = reinterpret_cast<float4*>(crow + (static_cast<long long>(h) * ld + start + r) * kHeadDim + i);
+        float4* c = reinterpret_cast<float4*>(base + kv_page_off(m, page, h, pr) + i);
         float4* t = reinterpret_cast<float4*>(rrow + col);
         if (dir == 0)
             *c = *t;

@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_proj_mma(const __grid_consta
     __shared__ __align__(8) uint64_t empty[kMmaMaxStagesTF];
     __shared__ __align__(8) uint64_t bar_x;
     __shared__ unsigned long long s_key[BT];
-    __shared__ int s_slot[BT], s_len[BT];   // EPI_QKV: the batch tile's cache slots and rows
+    __shared__ int s_slot[BT], s_len[BT];   // EPI_QKV: cache page and row in it of each column's new row
     __shared__ int s_flag, s_last;   // staging succeeded; this CTA arrived last (head)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -251,8 +251,11 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_proj_mma(const __grid_consta
     }
     if (EPI == EPI_HEAD && tid < BT) s_key[tid] = 0ull;
     if (EPI == EPI_QKV && tid < BT) {
-        s_slot[tid] = tid < nb ? a.meta->slot[b0 + tid] : 0;
-        s_len[tid] = tid < nb ? a.meta->len[b0 + tid] : 0;
+        // the cache page and row within it of this step's new row, per batch column
+        int page = 0, r = 0;
+        if (tid < nb) kv_page_of(a.kv, a.meta->slot[b0 + tid], a.meta->len[b0 + tid], page, r);
+        s_slot[tid] = page;
+        s_len[tid] = r;
     }
     __syncthreads();
     if (!s_flag) {
@@ -305,7 +308,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_proj_mma(const __grid_consta
                 a.out[static_cast<long long>(gb) * a.out_ld + within] = y;
             } else {
                 float* cache = (sec == 1) ? a.kc : a.vc;
-                cache[s_slot[b] * a.slot_stride + (static_cast<long long>(hh) * a.ld + s_len[b]) * kHeadDim + i] = y;
+                cache[kv_page_off(a.kv, s_slot[b], hh, s_len[b]) + i] = y;
             }
         } else if (EPI == EPI_HEAD) {
             if (a.out != nullptr) a.out[static_cast<long long>(gb) * a.out_ld + n] = y;

@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
     __shared__ __align__(8) uint64_t tfull[2], tempty[2], bar_x, bar_done;
     __shared__ uint32_t s_tmem;
     __shared__ float s_xs[BT];
-    __shared__ int s_pos[BT], s_slot[BT], s_len[BT];   // EPI_QKV: the batch tile's step description
+    __shared__ int s_pos[BT], s_slot[BT], s_len[BT];   // EPI_QKV: position, cache page, row in the page
     __shared__ int s_fail;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -130,9 +130,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
     if (tid < BT) {
         s_xs[tid] = tid < nb ? A.xs[b0 + tid] : 0.0f;
         if (EPI == EPI_QKV) {
+            // position, and the cache page and row within it of this step's new row
+            int page = 0, r = 0;
+            if (tid < nb) kv_page_of(a.kv, a.meta->slot[b0 + tid], a.meta->len[b0 + tid], page, r);
             s_pos[tid] = tid < nb ? a.meta->pos[b0 + tid] : 0;
-            s_slot[tid] = tid < nb ? a.meta->slot[b0 + tid] : 0;
-            s_len[tid] = tid < nb ? a.meta->len[b0 + tid] : 0;
+            s_slot[tid] = page;
+            s_len[tid] = r;
         }
     }
     __syncthreads();
@@ -295,8 +298,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
                         a.out[static_cast<long long>(gb) * a.out_ld + within] = val;
                     } else {
                         float* cache = (sec == 1) ? a.kc : a.vc;
-                        cache[s_slot[b] * a.slot_stride + (static_cast<long long>(hh) * a.ld + s_len[b]) * kHeadDim + col] =
-                            val;
+                        cache[kv_page_off(a.kv, s_slot[b], hh, s_len[b]) + col] = val;
                     }
                 } else if (EPI == EPI_STORE) {
                     a.out[static_cast<long long>(gb) * a.out_ld + n] = y;
