@@ -42,15 +42,37 @@ def oracle_greedy(ref, prompt, max_new, eos=-1, enc=None, max_len=None, max_pos=
         logits = lg[0]
 
 
-def compare_greedy(gpu_ids, ref_ids, margins, what):
-    """Identical sequences, or a divergence at a near-tie (reported); returns the event."""
+def compare_greedy(gpu_ids, ref_ids, margins, what, env_at=None):
+    """Identical sequences, or a divergence at a near-tie (reported); returns the event.
+
+    A near-tie is a top-2 margin inside twice the logit tolerance. For the W8A8 models
+    `env_at(i)` gives the spread of the oracle ensemble (tests/_harness.py) at pick i with the
+    same history: correct implementations whose int8 activation codes round differently at
+    ties drift apart by that much over the layers, so a margin inside twice the tolerance plus
+    that spread is a near-tie too."""
     for i, (g, o) in enumerate(zip(gpu_ids, ref_ids)):
         if g != o:
             m, top = margins[i]
-            assert m <= 2 * (ATOL + RTOL * abs(top)), (what, i, g, o, m)
-            return (what, "near-tie divergence at token", i, m)
+            env = env_at(i) if env_at is not None else 0.0
+            assert m <= 2 * (ATOL + RTOL * abs(top) + 2 * env), (what, i, g, o, m, env)
+            return (what, "near-tie divergence at token", i, m, env)
     assert len(gpu_ids) == len(ref_ids), (what, len(gpu_ids), len(ref_ids))
     return None
+
+
+def ensemble_env(W, max_len, start, tokens, n_jitter=2):
+    """Largest distance of a jittered oracle's logits from the oracle proper's after `start`
+    (a function giving a fresh decoder's stream state and first logits) and the teacher-forced
+    `tokens` (the same history for all)."""
+    runs = []
+    for seed in [None] + [100 + j for j in range(n_jitter)]:
+        r = oracle.OracleDecoder(W, max_len, quant_jitter=seed)
+        st, lg = start(r)
+        for t in tokens:
+            _, l = r.step([st], [t], [st.n])
+            lg = l[0]
+        runs.append(np.asarray(lg, np.float64))
+    return max(float(np.abs(j - runs[0]).max()) for j in runs[1:])
 
 
 def _requests(cfg, n, seed=0):
@@ -128,9 +150,14 @@ def test_c3_prefill_1024_then_128_greedy_steps_match_oracle():
     got = dec.generate([{"prompt": prompt, "max_new": wl.steps + 1}], max_active=1)[0]
     dec.close()
     ref = oracle.OracleDecoder(W, wl.max_cache_len)
-    del W
     ids, margins = oracle_greedy(ref, prompt, wl.steps + 1)
-    print(compare_greedy(got, ids, margins, "c3"), f"min margin {min(m for m, _ in margins):.4g}")
+
+    def start(r):
+        st = r.new_state(None)
+        return st, r.prefill(st, prompt)
+
+    env_at = lambda i: ensemble_env(W, wl.max_cache_len, start, ids[:i])
+    print(compare_greedy(got, ids, margins, "c3", env_at), f"min margin {min(m for m, _ in margins):.4g}")
 
 
 def test_c5_sampled_stream_200_greedy_steps_match_oracle():
@@ -170,7 +197,6 @@ def test_c4_sampled_streams_32_greedy_steps_match_oracle():
     W = synth.make_weights(cfg, 0)
     dec = Decoder(cfg, W, max_slots=wl.batch, max_cache_len=wl.max_cache_len)
     ref = oracle.OracleDecoder(W, wl.max_cache_len)
-    del W
     lens = synth.cache_lens(wl, 0).astype(np.int64)
     sample = sorted({int(np.argmin(lens)), int(np.argmax(lens))})
     states = {}
@@ -207,4 +233,15 @@ def test_c4_sampled_streams_32_greedy_steps_match_oracle():
             tok = oracle.argmax_first(lg[0])
             ids.append(tok)
             margins.append(_margin(lg[0]))
-        print(compare_greedy(gpu_ids[s], ids, margins, f"c4 stream {s}"), f"min margin {min(m for m, _ in margins):.4g}")
+        n0 = int(synth.cache_lens(wl, 0)[s])
+
+        def start(r, s=s, n0=n0):
+            ks, vs = zip(*(synth.seed_kv(cfg, s, l, n0, 0) for l in range(cfg.n_layers)))
+            st2 = r.new_state(None)
+            r.kv_append(st2, 0, np.stack(ks), np.stack(vs))
+            _, lg0 = r.step([st2], [first[s]], [st2.n])
+            return st2, lg0[0]
+
+        env_at = lambda i, start=start, ids=ids: ensemble_env(W, wl.max_cache_len, start, ids[:i])
+        print(compare_greedy(gpu_ids[s], ids, margins, f"c4 stream {s}", env_at),
+              f"min margin {min(m for m, _ in margins):.4g}")

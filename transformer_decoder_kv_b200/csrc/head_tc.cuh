@@ -43,7 +43,8 @@ constexpr int kHeadKC = 128;                        // K per stage (one 128-byte
 constexpr int kHeadPlaneBox = kHeadRows * kHeadKC;  // 16 KB
 constexpr int kHeadStageBytes = 3 * kHeadPlaneBox;  // 48 KB
 constexpr int kHeadMaxStages = 4;      // three-digit stages (48 KB)
-constexpr int kHeadMaxStagesW1 = 8;    // one-digit stages (16 KB)
+constexpr int kHeadMaxStagesW1 = 8;    // one-digit stages (16 KB); sizes the stage barriers
+static_assert(kHeadMaxStagesW1 >= kHeadMaxStages, "the barrier arrays hold every stage count");
 constexpr int kHeadMaxK = 4096;
 
 struct HeadArgs {
@@ -333,7 +334,7 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
         (reinterpret_cast<uintptr_t>(head_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     unsigned char* ring = smem;                                             // NS stages
     unsigned char* sx = smem + static_cast<size_t>(NS) * kStage;            // 3 x xplane
-    __shared__ __align__(8) uint64_t full[kHeadMaxStages], empty[kHeadMaxStages];
+    __shared__ __align__(8) uint64_t full[kHeadMaxStagesW1], empty[kHeadMaxStagesW1];   // NS <= 8 stages
     __shared__ __align__(8) uint64_t tfull[2], tempty[2], bar_x, bar_done;
     __shared__ uint32_t s_tmem;
     __shared__ unsigned long long s_key[BT];
