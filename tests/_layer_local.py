@@ -28,11 +28,8 @@ import synth
 from tests._harness import ATOL, RTOL
 
 # Code units (of the quantiser's x * 127 / amax) within which the GPU's input to the
-# quantiser may fall on the other side of a rounding boundary. Norm and SwiGLU outputs (sites
-# 0, 2, 3) differ from the oracle by a few f32 ulps, i.e. a few 1e-5 code units; the
-# attention context feeding the o projection (site 1) is an f32 online softmax over up to
-# thousands of keys and carries more.
-TIE_EPS = {0: 2e-4, 1: 5e-3, 2: 2e-4, 3: 2e-4}
+# quantiser may fall on the other side of a rounding boundary (the oracle's NEAR_TIE_EPS).
+TIE_EPS = oracle.decoder.NEAR_TIE_EPS
 
 
 def _clone(st: oracle.decoder.StreamState, l: int) -> oracle.decoder.StreamState:

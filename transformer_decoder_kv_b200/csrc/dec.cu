@@ -410,13 +410,12 @@ dec_status gemv_whisper(dec_handle* h, const GemvArgs& a, cudaStream_t st, const
     return gemv<int8_t, false, PRO, EPI, MAP>(h, a, st);
 }
 
-// Qwen W8A8 projections: tcgen05 int8 tensor cores from batch 8 on for matrices of 2^21
-// weights or more, dp4a otherwise (bit-identical).
+// Qwen W8A8 projections: tcgen05 int8 tensor cores from batch 8 on, dp4a below
+// (bit-identical: exact int32 sums from the same int8 codes).
 template <int PRO, int EPI, int MAP>
 dec_status gemv_qwen(dec_handle* h, const GemvArgs& a, const CUtensorMap& map, cudaStream_t st) {
     const int n_rows = MAP == MAP_DUAL ? 2 * a.N : a.N;
-    if (static_cast<long long>(n_rows) * a.K >= kMmaMinWeights && tc_eligible(h, n_rows, a.K, a.B))
-        return proj_w8a8_tc<PRO, EPI, MAP>(h, a, map, n_rows, st);
+    if (tc_eligible(h, n_rows, a.K, a.B)) return proj_w8a8_tc<PRO, EPI, MAP>(h, a, map, n_rows, st);
     return gemv<int8_t, true, PRO, EPI, MAP>(h, a, st);
 }
 
