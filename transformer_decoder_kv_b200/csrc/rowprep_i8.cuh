@@ -13,6 +13,79 @@ namespace dec {
 // Per-row int8 quantisation (optionally after RMSNorm or LayerNorm), one warp per row,
 // with the arithmetic and reduction order of the CUDA-core kernel's prologue so that both
 // paths produce the same codes and scales.
+// Rows of up to kRowprepRegK4 float4 per lane stay in registers: the row is read from global
+// memory once instead of once per pass; every pass visits the elements in the same order
+// (element lane + 32 j, j ascending) whether they come from registers or from memory.
+constexpr int kRowprepRegK4 = 24;   // K <= 32 * 24 * 4 = 3072
+
+template <int PRO, class Get>
+__device__ __forceinline__ float rowprep_i8_passes(Get get, int K4, int K, int lane, const float4* g4,
+                                                   const float4* be4, float eps, uint32_t* q, int jmax) {
+    float mu = 0.0f, rstd = 1.0f;
+    if (PRO == PRO_LN) {
+        float sum = 0.0f;
+        for (int j = 0; j < jmax; ++j)
+            if (lane + 32 * j < K4) {
+                const float4 v = get(j);
+                sum += (v.x + v.y) + (v.z + v.w);
+            }
+        mu = warp_sum(sum) / static_cast<float>(K);
+        float var = 0.0f;
+        for (int j = 0; j < jmax; ++j)
+            if (lane + 32 * j < K4) {
+                const float4 v = get(j);
+                const float d0 = v.x - mu, d1 = v.y - mu, d2 = v.z - mu, d3 = v.w - mu;
+                var = fmaf(d0, d0, var);
+                var = fmaf(d1, d1, var);
+                var = fmaf(d2, d2, var);
+                var = fmaf(d3, d3, var);
+            }
+        var = warp_sum(var) / static_cast<float>(K);
+        rstd = 1.0f / sqrtf(var + eps);
+    } else if (PRO == PRO_RMS) {
+        float ss = 0.0f;
+        for (int j = 0; j < jmax; ++j)
+            if (lane + 32 * j < K4) {
+                const float4 v = get(j);
+                ss = fmaf(v.x, v.x, ss);
+                ss = fmaf(v.y, v.y, ss);
+                ss = fmaf(v.z, v.z, ss);
+                ss = fmaf(v.w, v.w, ss);
+            }
+        ss = warp_sum(ss) / static_cast<float>(K);
+        rstd = 1.0f / sqrtf(ss + eps);
+    }
+    auto normed = [&](int j) {
+        const int k = lane + 32 * j;
+        const float4 v = get(j);
+        float4 g = make_float4(1.f, 1.f, 1.f, 1.f), be = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (PRO != PRO_NONE) g = __ldg(g4 + k);
+        if (PRO == PRO_LN) be = __ldg(be4 + k);
+        return make_float4(norm_value(PRO, v.x, mu, rstd, g.x, be.x), norm_value(PRO, v.y, mu, rstd, g.y, be.y),
+                           norm_value(PRO, v.z, mu, rstd, g.z, be.z), norm_value(PRO, v.w, mu, rstd, g.w, be.w));
+    };
+    float amax = 0.0f;
+    for (int j = 0; j < jmax; ++j)
+        if (lane + 32 * j < K4) {
+            const float4 y = normed(j);
+            amax = fmaxf(amax, fabsf(y.x));
+            amax = fmaxf(amax, fabsf(y.y));
+            amax = fmaxf(amax, fabsf(y.z));
+            amax = fmaxf(amax, fabsf(y.w));
+        }
+    amax = warp_max(amax);
+    const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    for (int j = 0; j < jmax; ++j)
+        if (lane + 32 * j < K4) {
+            const float4 y = normed(j);
+            q[lane + 32 * j] = (static_cast<uint32_t>(quant_i8(y.x, inv)) & 0xffu) |
+                               ((static_cast<uint32_t>(quant_i8(y.y, inv)) & 0xffu) << 8) |
+                               ((static_cast<uint32_t>(quant_i8(y.z, inv)) & 0xffu) << 16) |
+                               ((static_cast<uint32_t>(quant_i8(y.w, inv)) & 0xffu) << 24);
+        }
+    return amax;
+}
+
 template <int PRO>
 __global__ void __launch_bounds__(128) k_rowprep_i8(const float* __restrict__ x, int x_ld,
                                                     const float* __restrict__ gw, const float* __restrict__ gb,
@@ -27,62 +100,18 @@ __global__ void __launch_bounds__(128) k_rowprep_i8(const float* __restrict__ x,
     const float4* g4 = reinterpret_cast<const float4*>(gw);
     const float4* be4 = reinterpret_cast<const float4*>(gb);
     const int K4 = K >> 2;
-    float mu = 0.0f, rstd = 1.0f;
-    if (PRO == PRO_LN) {
-        float sum = 0.0f;
-        for (int k = lane; k < K4; k += 32) {
-            const float4 v = xr[k];
-            sum += (v.x + v.y) + (v.z + v.w);
-        }
-        mu = warp_sum(sum) / static_cast<float>(K);
-        float var = 0.0f;
-        for (int k = lane; k < K4; k += 32) {
-            const float4 v = xr[k];
-            const float d0 = v.x - mu, d1 = v.y - mu, d2 = v.z - mu, d3 = v.w - mu;
-            var = fmaf(d0, d0, var);
-            var = fmaf(d1, d1, var);
-            var = fmaf(d2, d2, var);
-            var = fmaf(d3, d3, var);
-        }
-        var = warp_sum(var) / static_cast<float>(K);
-        rstd = 1.0f / sqrtf(var + eps);
-    } else if (PRO == PRO_RMS) {
-        float ss = 0.0f;
-        for (int k = lane; k < K4; k += 32) {
-            const float4 v = xr[k];
-            ss = fmaf(v.x, v.x, ss);
-            ss = fmaf(v.y, v.y, ss);
-            ss = fmaf(v.z, v.z, ss);
-            ss = fmaf(v.w, v.w, ss);
-        }
-        ss = warp_sum(ss) / static_cast<float>(K);
-        rstd = 1.0f / sqrtf(ss + eps);
-    }
-    auto normed = [&](int k) {
-        const float4 v = xr[k];
-        float4 g = make_float4(1.f, 1.f, 1.f, 1.f), be = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (PRO != PRO_NONE) g = __ldg(g4 + k);
-        if (PRO == PRO_LN) be = __ldg(be4 + k);
-        return make_float4(norm_value(PRO, v.x, mu, rstd, g.x, be.x), norm_value(PRO, v.y, mu, rstd, g.y, be.y),
-                           norm_value(PRO, v.z, mu, rstd, g.z, be.z), norm_value(PRO, v.w, mu, rstd, g.w, be.w));
-    };
-    float amax = 0.0f;
-    for (int k = lane; k < K4; k += 32) {
-        const float4 y = normed(k);
-        amax = fmaxf(amax, fabsf(y.x));
-        amax = fmaxf(amax, fabsf(y.y));
-        amax = fmaxf(amax, fabsf(y.z));
-        amax = fmaxf(amax, fabsf(y.w));
-    }
-    amax = warp_max(amax);
-    const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
     uint32_t* q = reinterpret_cast<uint32_t*>(xq + static_cast<long long>(b) * K);
-    for (int k = lane; k < K4; k += 32) {
-        const float4 y = normed(k);
-        q[k] = (static_cast<uint32_t>(quant_i8(y.x, inv)) & 0xffu) |
-               ((static_cast<uint32_t>(quant_i8(y.y, inv)) & 0xffu) << 8) |
-               ((static_cast<uint32_t>(quant_i8(y.z, inv)) & 0xffu) << 16) |
-               ((static_cast<uint32_t>(quant_i8(y.w, inv)) & 0xffu) << 24);
+    float amax;
+    if (K4 <= 32 * kRowprepRegK4) {
+        float4 rv[kRowprepRegK4];
+#pragma unroll
+        for (int j = 0; j < kRowprepRegK4; ++j)
+            rv[j] = lane + 32 * j < K4 ? xr[lane + 32 * j] : make_float4(0.f, 0.f, 0.f, 0.f);
+        // every loop below is fully unrolled over the compile-time bound, so rv stays in registers
+        amax = rowprep_i8_passes<PRO>([&](int j) { return rv[j]; }, K4, K, lane, g4, be4, eps, q, kRowprepRegK4);
+    } else {
+        amax = rowprep_i8_passes<PRO>([&](int j) { return xr[lane + 32 * j]; }, K4, K, lane, g4, be4, eps, q,
+                                      (K4 + 31) / 32);
     }
     if (lane == 0) xs[b] = __fdiv_rn(amax, 127.0f);
 }
