@@ -616,12 +616,10 @@ inline MmaPlan mma_plan(int N, int K, int elt, int num_sms) {
     p.n_blocks = (N + kMmaBlockRows - 1) / kMmaBlockRows;
     if (K % 32 != 0 || N <= 0) return p;
     const int kchunks = (K + KC - 1) / KC;
-    // the fewest K slices whose activation slice fits: each split-K exchange (partial tiles,
-    // a fence, an arrival count, the last arriver reading every slice) costs more on the
-    // critical path than the parallelism it buys once the weights stream in during the
-    // previous kernel (measured on B200 for the int8 tensor-core kernel of the same design)
-    (void)num_sms;
-    int n_ks = 1;
+    // one wave: n_blocks x n_ks CTAs within the SM count (the f32 activation slices and the
+    // split TF32 products make this kernel's CTAs heavier than the int8 kernel's, and fewer
+    // slices measured slower on B200 for the C2 and C5 shapes)
+    int n_ks = std::max(1, std::min(kchunks, num_sms / std::max(1, p.n_blocks)));
     auto slice_len = [&](int nks) { return std::min(((kchunks + nks - 1) / nks) * KC, K); };
     auto xbytes = [&](int ksl) { return size_t(kMmaMaxBT) * (ksl + pad) * 4; };
     while (xbytes(slice_len(n_ks)) > kMmaXBudget && n_ks < kchunks) ++n_ks;
