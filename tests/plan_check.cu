@@ -50,6 +50,42 @@ int main() {
             shapes = {{3 * d, d, e}, {d, d, e}, {F, d, e}, {d, F, e}};
         }
         shapes.push_back({m.V, d, 4});   // f32 head on the TF32 kernel (fallback path)
+        // Whisper projections on the tcgen05 digit path (three activation planes)
+        if (m.kind != 2) {
+            for (const auto& s : shapes) {
+                if (s.N == m.V) continue;
+                const MmaPlan p = tc_plan(s.N, s.K, sms, 3);
+                CHECK(p.ok, "digit plan not ok N=%d K=%d", s.N, s.K);
+                if (!p.ok) continue;
+                CHECK(p.n_ks * p.ksl >= s.K && (p.n_ks - 1) * p.ksl < s.K, "digit K cover N=%d K=%d", s.N, s.K);
+                CHECK(p.ksl % kTcKC == 0 || p.ksl == s.K, "digit slice not whole stages N=%d K=%d", s.N, s.K);
+                const int nch = (p.ksl + kTcKC - 1) / kTcKC;
+                CHECK(size_t(3) * kTcMaxBT * nch * 128 <= kTcXBudget, "digit X budget N=%d K=%d", s.N, s.K);
+                for (int wd : {1, 3}) {
+                    // ring: at least two stages of wd weight planes next to the activation slice
+                    const size_t avail = size_t(227 * 1024) - 2048 - size_t(3) * nch * kTcMaxBT * 128;
+                    CHECK(avail / (size_t(wd) * kTcStageBytes) >= 2, "digit ring N=%d K=%d wd=%d", s.N, s.K, wd);
+                }
+                for (int B = 1; B <= DEC_MAX_BATCH; ++B) {
+                    const int BT = B <= 16 ? 16 : 32;
+                    const int gy = (B + BT - 1) / BT;
+                    // part[((grp * n_ks + ks) * 32 + lane) * 3 * (BT / 2) + v], grp < n_blocks * gy * 8
+                    const size_t need = size_t(p.n_blocks) * gy * 8 * p.n_ks * 32 * 3 * (BT / 2) * 4;
+                    if (p.n_ks > 1) CHECK(need <= tc_part_bytes(p, B, 3), "digit scratch N=%d K=%d B=%d", s.N, s.K, B);
+                    CHECK(p.n_blocks * gy * 8 <= tc_counters(p, B), "digit counters N=%d K=%d B=%d", s.N, s.K, B);
+                    for (int sets = 1; sets <= 2; ++sets)
+                        CHECK(tc_tmem_cols(3, BT, sets) <= 256 && uint32_t(sets * 3 * BT) <= tc_tmem_cols(3, BT, sets),
+                              "digit TMEM columns B=%d", B);
+                    // stacked planes: MMA N = 3 BT, 2 BT, BT within the M = 128 limits
+                    CHECK(3 * BT <= 256 && (3 * BT) % 16 == 0 && (2 * BT) % 16 == 0 && BT % 16 == 0,
+                          "digit MMA N B=%d", B);
+                }
+            }
+        }
+        for (int bt : {16, 32})
+            for (int sets = 1; sets <= 2; ++sets)
+                CHECK(tc_tmem_cols(1, bt, sets) <= 256 && uint32_t(sets * bt) <= tc_tmem_cols(1, bt, sets),
+                      "W8A8 TMEM columns");
         for (const auto& s : shapes) {
             if (s.elt == 0) {
                 const MmaPlan p = tc_plan(s.N, s.K, sms);
@@ -62,10 +98,11 @@ int main() {
                 for (int B = 1; B <= DEC_MAX_BATCH; ++B) {
                     const int BT = B <= 16 ? 16 : 32;
                     const int gy = (B + BT - 1) / BT;
-                    // kernel: part[((grp * n_ks + ks) * 32 + lane) * BT + col], grp < n_blocks * gy * 4
-                    const size_t need = size_t(p.n_blocks) * gy * 4 * p.n_ks * 32 * BT * 4;
+                    // kernel: part[((grp * n_ks + ks) * 32 + lane) * (BT / 2) + col],
+                    // grp < n_blocks * gy * 4 lane quarters * 2 column halves
+                    const size_t need = size_t(p.n_blocks) * gy * 4 * 2 * p.n_ks * 32 * (BT / 2) * 4;
                     if (p.n_ks > 1) CHECK(need <= tc_part_bytes(p, B), "tc scratch N=%d K=%d B=%d", s.N, s.K, B);
-                    CHECK(p.n_blocks * gy * 4 <= tc_counters(p, B), "tc counters N=%d K=%d B=%d", s.N, s.K, B);
+                    CHECK(p.n_blocks * gy * 4 * 2 <= tc_counters(p, B), "tc counters N=%d K=%d B=%d", s.N, s.K, B);
                     const MmaPlan q = tc_plan(s.N, s.K, sms);
                     CHECK(q.n_ks == p.n_ks && q.ksl == p.ksl, "tc plan depends on call");
                 }

@@ -68,6 +68,11 @@ struct LayerDev {
     // 2-D TMA descriptors of the projections (tensor-core path); Qwen uses m_qkv (the
     // permuted panel), m_o, m_1 (gate/up) and m_2 (down)
     CUtensorMap m_qkv, m_o, m_xq, m_xo, m_1, m_2;
+    // Whisper with f32 weights, tcgen05 path: each projection's three int8 digit planes
+    // [3][N][K] with row scales, and their TMA descriptors (same order as the maps above)
+    int8_t* dig[6] = {};
+    float* dsc[6] = {};
+    CUtensorMap m_dig[6];
 };
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -75,6 +80,31 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 }  // namespace
+
+// Per-chain step scratch. A decode step of many rows runs as two chains, each over half of
+// the rows, on two streams: while one chain streams its attention K/V from HBM, the other
+// runs its latency-bound projections. Each chain has its own copies of everything a
+// launch writes besides its rows of x, so the two never share scratch.
+struct Chain {
+    float *q = nullptr, *ctx = nullptr, *ffn = nullptr, *xq = nullptr;
+    float* part = nullptr;          // attention split partials
+    int* counters = nullptr;        // attention split arrival counts, zero between launches
+    float* xn = nullptr;            // normalised activation rows (TF32 tensor-core path)
+    int8_t* xq8 = nullptr;          // quantised activation rows and their scales (int8 tensor-core path)
+    int xq8_rows = 0;               // rows of xq8 (>= max batch, >= 32)
+    CUtensorMap m_xq8[2][2];        // xq8 as [rows, K] for K = d, F and boxes of 16, 32 rows
+    float* xs8 = nullptr;
+    // Whisper tcgen05 path: activation rows as three int8 digit planes [3][xd_rows][K]
+    int8_t* xd3 = nullptr;
+    float* xsd = nullptr;
+    int xd_rows = 0;
+    CUtensorMap m_xd3[2][2];        // xd3 as [3 rows, K] for K = d, F and boxes of 16, 32 rows
+    void* mma_part = nullptr;       // split-K partial tiles (tensor-core path)
+    size_t mma_part_bytes = 0;
+    int* mma_cnt = nullptr;         // split-K arrival counts, zero between launches
+    int mma_cnt_len = 0;
+    StepMeta* meta = nullptr;       // the chain's rows of the step description
+};
 
 struct dec_handle {
     dec_config cfg{};
@@ -109,19 +139,15 @@ struct dec_handle {
     int max_rows = 0;                  // rows of the per-step workspaces: max(max_batch, prompt chunk)
     int prefill_chunk = kPrefillChunk; // prompt rows per prefill step
     int tps_self = 1, tps_cross = 1;   // attention tiles per split (handle constants)
-    // workspace
-    float *x = nullptr, *q = nullptr, *ctx = nullptr, *ffn = nullptr, *xq = nullptr;
-    float* part = nullptr;
-    int* counters = nullptr;
-    float* xn = nullptr;            // normalised activation rows (tensor-core path)
-    int8_t* xq8 = nullptr;          // quantised activation rows and their scales (int8 tensor-core path)
-    int xq8_rows = 0;               // rows of xq8 (>= max batch, >= 32)
-    CUtensorMap m_xq8[2][2];        // xq8 as [rows, K] for K = d, F and boxes of 16, 32 rows
-    float* xs8 = nullptr;
-    void* mma_part = nullptr;       // split-K partial tiles (tensor-core path)
-    size_t mma_part_bytes = 0;
-    int* mma_cnt = nullptr;         // split-K arrival counts, zero between launches
-    int mma_cnt_len = 0;
+    // workspace: the residual rows x are shared by both chains (each owns a row range); the
+    // rest of the per-step scratch is per chain (see Chain)
+    float* x = nullptr;
+    Chain chain[2];
+    Chain* w = &chain[0];           // the chain whose launches are being issued
+    int n_chains = 1;               // 2: decode steps of kSplitMinBatch rows or more run as two chains
+    cudaStream_t side = nullptr;    // the second chain's stream (eager steps)
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr, ev_attn[2] = {nullptr, nullptr};
+    bool tcd_ok = false;            // Whisper digit-path descriptors and planes built
     unsigned long long* keys = nullptr;
     int* head_counter = nullptr;
     int* last_tok = nullptr;
@@ -130,8 +156,7 @@ struct dec_handle {
     int* host_tok = nullptr;        // pinned copy of every slot's greedy continuation token
     bool failed = false;            // a bounded device wait gave up; dec_reset required
     int inject_drop = 0;            // test hook: drop one attention tile copy per step
-    int mma_cnt_bytes = 0;
-    StepMeta* dmeta = nullptr;
+    StepMeta* dmeta = nullptr;      // [3]: the whole step, then the rows of chain 0 and chain 1
     StepMeta* hmeta[kMetaRing] = {};
     cudaEvent_t hev[kMetaRing] = {};
     int ring = 0;
@@ -342,6 +367,10 @@ dec_status gemv(dec_handle* h, const GemvArgs& a, cudaStream_t st) {
 // CUDA-core kernel's whole run, except for int8 weights with f32 activations, whose
 // CUDA-core kernel is arithmetic-bound from batch 8 on.
 constexpr int kMmaMinBatch = 8;
+// Decode steps of this many rows or more run as two chains (run_step); each chain's half is
+// a multiple of 16 rows, so each stays on the tensor-core paths.
+constexpr int kSplitMinBatch = 32;
+inline int split_rows(int B) { return std::min(B - kMmaMinBatch, ((B / 2 + 15) / 16) * 16); }
 constexpr long long kMmaMinWeights = 1LL << 21;
 
 bool mma_worth(int N, int K, bool w8a32) {
@@ -352,17 +381,17 @@ bool mma_eligible(const dec_handle* h, int N, int K, int elt, int B) {
     if (!h->tma_ok || B < kMmaMinBatch) return false;
     const MmaPlan p = mma_plan(N, K, elt, h->num_sms);
     if (!p.ok || K > kRowprepMaxK) return false;
-    return p.n_ks == 1 || (mma_part_bytes(p, B) <= h->mma_part_bytes && mma_counters(p, B) <= h->mma_cnt_len);
+    return p.n_ks == 1 || (mma_part_bytes(p, B) <= h->w->mma_part_bytes && mma_counters(p, B) <= h->w->mma_cnt_len);
 }
 
-// Norm prologue of the tensor-core path: normalised rows into h->xn, which becomes the
+// Norm prologue of the tensor-core path: normalised rows into h->w->xn, which becomes the
 // projection's input.
 template <int PRO>
 dec_status mma_input(dec_handle* h, GemvArgs& g, cudaStream_t st) {
     if (PRO == PRO_NONE) return DEC_OK;
-    const cudaError_t e = rowprep_launch<PRO>(g, h->xn, st);
+    const cudaError_t e = rowprep_launch<PRO>(g, h->w->xn, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "row normalisation launch");
-    g.x = h->xn;
+    g.x = h->w->xn;
     g.x_ld = g.K;
     return DEC_OK;
 }
@@ -372,7 +401,7 @@ dec_status proj_mma(dec_handle* h, const GemvArgs& a, const CUtensorMap& map, cu
     GemvArgs g = a;
     DEC_TRY(mma_input<PRO>(h, g, st));
     const cudaError_t e =
-        proj_mma_launch<WT, EPI>(h->num_sms, map, h->mma_part, h->mma_part_bytes, h->mma_cnt, h->mma_cnt_len, g, st);
+        proj_mma_launch<WT, EPI>(h->num_sms, map, h->w->mma_part, h->w->mma_part_bytes, h->w->mma_cnt, h->w->mma_cnt_len, g, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "tensor-core projection launch");
     return DEC_OK;
 }
@@ -381,30 +410,72 @@ bool tc_eligible(const dec_handle* h, int n_rows, int K, int B) {
     if (!h->tma_ok || B < kMmaMinBatch) return false;
     const MmaPlan p = tc_plan(n_rows, K, h->num_sms);
     if (!p.ok) return false;
-    return p.n_ks == 1 || (tc_part_bytes(p, B) <= h->mma_part_bytes && tc_counters(p, B) <= h->mma_cnt_len);
+    return p.n_ks == 1 || (tc_part_bytes(p, B) <= h->w->mma_part_bytes && tc_counters(p, B) <= h->w->mma_cnt_len);
 }
 
 // W8A8 on tcgen05 int8 tensor cores: rows quantised by k_rowprep_i8, exact int32 products.
 template <int PRO, int EPI, int MAP>
 dec_status proj_w8a8_tc(dec_handle* h, const GemvArgs& a, const CUtensorMap& map, int n_rows, cudaStream_t st) {
-    cudaError_t e = rowprep_i8_launch<PRO>(a, h->xq8, h->xs8, st);
+    cudaError_t e = rowprep_i8_launch<PRO>(a, h->w->xq8, h->w->xs8, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "row quantisation launch");
     const int kx = a.K == h->cfg.d_model ? 0 : 1;
-    e = proj_tc_launch<EPI, MAP>(h->num_sms, map, h->m_xq8[kx][0], h->m_xq8[kx][1], n_rows, h->xs8, h->mma_part,
-                                 h->mma_part_bytes, h->mma_cnt, h->mma_cnt_len, a, st);
+    e = proj_tc_launch<EPI, MAP, 1, 1>(h->num_sms, map, h->w->m_xq8[kx][0], h->w->m_xq8[kx][1], n_rows, h->w->xq8_rows, h->w->xs8,
+                                       h->w->mma_part, h->w->mma_part_bytes, h->w->mma_cnt, h->w->mma_cnt_len, a, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "tcgen05 projection launch");
     return DEC_OK;
 }
 
-// Whisper projections exist as f32 or W8A32: tensor cores from batch 8 on, the
-// CUDA-core kernel below.
-template <int PRO, int EPI, int MAP>
-dec_status gemv_whisper(dec_handle* h, const GemvArgs& a, cudaStream_t st, const CUtensorMap* map = nullptr) {
+bool tcd_eligible(const dec_handle* h, int N, int K, int B) {
+    if (!h->tcd_ok || B < kMmaMinBatch || B > h->w->xd_rows) return false;
+    const MmaPlan p = tc_plan(N, K, h->num_sms, 3);
+    if (!p.ok) return false;
+    return p.n_ks == 1 || (tc_part_bytes(p, B, 3) <= h->w->mma_part_bytes && tc_counters(p, B) <= h->w->mma_cnt_len);
+}
+
+// Whisper projections on tcgen05 int8 tensor cores: the (normalised) activation rows split
+// into three int8 digit planes by k_rowprep_digits, times the int8 weights (W8A32, one
+// plane, three products per K step) or the f32 weights' three digit planes (six products),
+// with exact int32 sums; y = s_n s_b (A0 + (A1 + A2 / 254) / 254) + bias.
+template <int PRO, int EPI>
+dec_status proj_digits_tc(dec_handle* h, const GemvArgs& a, const LayerDev* L, int m, cudaStream_t st) {
     const bool f32w = h->cfg.proj_fmt == DEC_PROJ_F32;
-    if (map != nullptr) {
+    cudaError_t e = rowprep_digits_launch<PRO>(a.x, a.x_ld, a.norm_w, a.norm_b, a.eps, a.K, a.B,
+                                               static_cast<long long>(h->w->xd_rows) * a.K, h->w->xd3, h->w->xsd, nullptr,
+                                               true, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "row digit split launch");
+    const int kx = a.K == h->cfg.d_model ? 0 : 1;
+    GemvArgs g = a;
+    if (f32w) {
+        g.scale = L->dsc[m];
+        e = proj_tc_launch<EPI, MAP_ADJ, 3, 3>(h->num_sms, L->m_dig[m], h->w->m_xd3[kx][0], h->w->m_xd3[kx][1], a.N,
+                                               h->w->xd_rows, h->w->xsd, h->w->mma_part, h->w->mma_part_bytes, h->w->mma_cnt,
+                                               h->w->mma_cnt_len, g, st);
+    } else {
+        const CUtensorMap* maps[6] = {&L->m_qkv, &L->m_o, &L->m_xq, &L->m_xo, &L->m_1, &L->m_2};
+        e = proj_tc_launch<EPI, MAP_ADJ, 3, 1>(h->num_sms, *maps[m], h->w->m_xd3[kx][0], h->w->m_xd3[kx][1], a.N,
+                                               h->w->xd_rows, h->w->xsd, h->w->mma_part, h->w->mma_part_bytes, h->w->mma_cnt,
+                                               h->w->mma_cnt_len, g, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(h, e, "tcgen05 digit projection launch");
+    return DEC_OK;
+}
+
+// Whisper projections exist as f32 or W8A32: from batch 8 on, tcgen05 on digit planes (or
+// TF32 mma.sync when those are unavailable), the CUDA-core kernel below. `m` names the
+// layer's matrix (0 q|k|v, 1 o, 2 cross q, 3 cross o, 4 fc1, 5 fc2).
+template <int PRO, int EPI, int MAP>
+dec_status gemv_whisper(dec_handle* h, const GemvArgs& a, cudaStream_t st, const LayerDev& layer, int m) {
+    const bool f32w = h->cfg.proj_fmt == DEC_PROJ_F32;
+    const LayerDev* L = &layer;
+    if (h->tma_ok) {
+        // f32 weights take the tensor cores only for the larger matrices (below, the CUDA-core
+        // kernel's whole run is shorter than the extra row-split launch); W8A32 always
+        if ((!f32w || mma_worth(a.N, a.K, false)) && tcd_eligible(h, a.N, a.K, a.B))
+            return proj_digits_tc<PRO, EPI>(h, a, L, m, st);
+        const CUtensorMap* maps[6] = {&L->m_qkv, &L->m_o, &L->m_xq, &L->m_xo, &L->m_1, &L->m_2};
         if (f32w && mma_worth(a.N, a.K, false) && mma_eligible(h, a.N, a.K, 4, a.B))
-            return proj_mma<float, PRO, EPI>(h, a, *map, st);
-        if (!f32w && mma_eligible(h, a.N, a.K, 1, a.B)) return proj_mma<int8_t, PRO, EPI>(h, a, *map, st);
+            return proj_mma<float, PRO, EPI>(h, a, *maps[m], st);
+        if (!f32w && mma_eligible(h, a.N, a.K, 1, a.B)) return proj_mma<int8_t, PRO, EPI>(h, a, *maps[m], st);
     }
     if (f32w) return gemv<float, false, PRO, EPI, MAP>(h, a, st);
     return gemv<int8_t, false, PRO, EPI, MAP>(h, a, st);
@@ -534,7 +605,7 @@ GemvArgs base_args(dec_handle* h, int B) {
     GemvArgs g{};
     g.B = B;
     g.eps = h->cfg.norm_eps;
-    g.meta = h->dmeta;
+    g.meta = h->w->meta;
     g.err = h->dev_err;
     return g;
 }
@@ -554,188 +625,232 @@ dec_status phase_mark(dec_handle* h, cudaStream_t st, int layer, int kind) {
     return DEC_OK;
 }
 
+// One decoder layer for the rows of the current chain (h->w): X holds their residual rows.
+// wait_ev / done_ev order the layer's largest attention (self for Qwen2, cross for Whisper)
+// against the other chain's: it starts after wait_ev and records done_ev.
+dec_status layer_step(dec_handle* h, int l, int B, float* X, int max_len_plus1, cudaStream_t st,
+                      cudaEvent_t wait_ev, cudaEvent_t done_ev) {
+    const dec_config& c = h->cfg;
+    const int d = c.d_model, F = c.d_ff, H = c.n_heads;
+    (void)H;
+    const bool wh = c.family == DEC_FAMILY_WHISPER;
+    const LayerDev& L = h->layers[l];
+    float* kc = h->kc + l * h->self_layer_stride;
+    float* vc = h->vc + l * h->self_layer_stride;
+    // ---- q|k|v with the cache append ----
+    GemvArgs g = base_args(h, B);
+    g.x = X;
+    g.x_ld = d;
+    g.norm_w = L.n1w;
+    g.norm_b = L.n1b;
+    g.K = d;
+    g.N = d + 2 * kv_width(c);
+    g.W = L.wqkv;
+    g.scale = L.sqkv;
+    g.bias = L.bqkv;
+    g.out = h->w->q;
+    g.out_ld = d;
+    g.kc = kc;
+    g.vc = vc;
+    g.kv = self_kv_map(h);
+    g.d = d;
+    g.kvd = kv_width(c);
+    if (c.family == DEC_FAMILY_WHISPER) {
+        DEC_TRY((gemv_whisper<PRO_LN, EPI_QKV, MAP_ADJ>(h, g, st, L, 0)));
+    } else {
+        g.rope = h->rope;
+        DEC_TRY((gemv_qwen<PRO_RMS, EPI_QKV, MAP_ROPE>(h, g, L.m_qkv, st)));
+    }
+    DEC_TRY(phase_mark(h, st, l, DEC_PHASE_QKV));
+    // ---- self-attention over rows 0..len ----
+    AttnArgs at{};
+    at.q = h->w->q;
+    at.q_bstride = d;
+    at.k = kc;
+    at.v = vc;
+    at.slot_stride = h->self_slot_stride;
+    at.ld = c.max_cache_len;
+    at.H = H;
+    at.kv_group = H / kv_heads(c);
+    at.kv = self_kv_map(h);
+    at.mode = ATTN_SELF;
+    at.meta = h->w->meta;
+    at.out = h->w->ctx;
+    at.out_bstride = d;
+    at.part = h->w->part;
+    at.counters = h->w->counters;
+    at.err = h->dev_err;
+    at.drop_first_copy = (l == 0) ? h->inject_drop : 0;
+    if (!wh && wait_ev) DEC_CUDA(h, cudaStreamWaitEvent(st, wait_ev, 0));
+    DEC_TRY(attention(h, at, B, max_len_plus1, h->tps_self, st));
+    if (!wh && done_ev) DEC_CUDA(h, cudaEventRecord(done_ev, st));
+    DEC_TRY(phase_mark(h, st, l, DEC_PHASE_SELF_ATTN));
+    at.drop_first_copy = 0;
+    // ---- output projection + residual ----
+    g = base_args(h, B);
+    g.x = h->w->ctx;
+    g.x_ld = d;
+    g.K = d;
+    g.N = d;
+    g.W = L.wo;
+    g.scale = L.so;
+    g.bias = L.bo;
+    g.out = X;
+    g.out_ld = d;
+    if (c.family == DEC_FAMILY_WHISPER) {
+        DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st, L, 1)));
+    } else {
+        DEC_TRY((gemv_qwen<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, L.m_o, st)));
+    }
+    DEC_TRY(phase_mark(h, st, l, DEC_PHASE_O));
+    if (c.family == DEC_FAMILY_WHISPER) {
+        // ---- cross-attention block ----
+        g = base_args(h, B);
+        g.x = X;
+        g.x_ld = d;
+        g.norm_w = L.n2w;
+        g.norm_b = L.n2b;
+        g.K = d;
+        g.N = d;
+        g.W = L.wxq;
+        g.scale = L.sxq;
+        g.bias = L.bxq;
+        g.out = h->w->xq;
+        g.out_ld = d;
+        DEC_TRY((gemv_whisper<PRO_LN, EPI_STORE, MAP_ADJ>(h, g, st, L, 2)));
+        DEC_TRY(phase_mark(h, st, l, DEC_PHASE_CROSS_Q));
+        at.q = h->w->xq;
+        at.k = h->xkc + l * h->cross_layer_stride;
+        at.v = h->xvc + l * h->cross_layer_stride;
+        at.slot_stride = h->cross_slot_stride;
+        at.ld = c.enc_len;
+        at.mode = ATTN_CROSS;
+        at.kv_group = 1;
+        at.kv.table = nullptr;
+        at.n_fixed = c.enc_len;
+        if (wait_ev) DEC_CUDA(h, cudaStreamWaitEvent(st, wait_ev, 0));
+        DEC_TRY(attention(h, at, B, c.enc_len, h->tps_cross, st));
+        if (done_ev) DEC_CUDA(h, cudaEventRecord(done_ev, st));
+        DEC_TRY(phase_mark(h, st, l, DEC_PHASE_CROSS_ATTN));
+        g = base_args(h, B);
+        g.x = h->w->ctx;
+        g.x_ld = d;
+        g.K = d;
+        g.N = d;
+        g.W = L.wxo;
+        g.scale = L.sxo;
+        g.bias = L.bxo;
+        g.out = X;
+        g.out_ld = d;
+        DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st, L, 3)));
+        DEC_TRY(phase_mark(h, st, l, DEC_PHASE_CROSS_O));
+        // ---- GELU FFN ----
+        g = base_args(h, B);
+        g.x = X;
+        g.x_ld = d;
+        g.norm_w = L.n3w;
+        g.norm_b = L.n3b;
+        g.K = d;
+        g.N = F;
+        g.W = L.w1;
+        g.scale = L.s1;
+        g.bias = L.b1;
+        g.out = h->w->ffn;
+        g.out_ld = F;
+        DEC_TRY((gemv_whisper<PRO_LN, EPI_GELU, MAP_ADJ>(h, g, st, L, 4)));
+        DEC_TRY(phase_mark(h, st, l, DEC_PHASE_FFN_UP));
+        g = base_args(h, B);
+        g.x = h->w->ffn;
+        g.x_ld = F;
+        g.K = F;
+        g.N = d;
+        g.W = L.w2;
+        g.scale = L.s2;
+        g.bias = L.b2;
+        g.out = X;
+        g.out_ld = d;
+        DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st, L, 5)));
+        DEC_TRY(phase_mark(h, st, l, DEC_PHASE_FFN_DOWN));
+    } else {
+        // ---- SwiGLU MLP ----
+        g = base_args(h, B);
+        g.x = X;
+        g.x_ld = d;
+        g.norm_w = L.n2w;
+        g.K = d;
+        g.N = F;
+        g.W = L.wg;
+        g.W2 = L.wu;
+        g.scale = L.sg;
+        g.scale2 = L.su;
+        g.out = h->w->ffn;
+        g.out_ld = F;
+        DEC_TRY((gemv_qwen<PRO_RMS, EPI_SWIGLU, MAP_DUAL>(h, g, L.m_1, st)));
+        DEC_TRY(phase_mark(h, st, l, DEC_PHASE_FFN_UP));
+        g = base_args(h, B);
+        g.x = h->w->ffn;
+        g.x_ld = F;
+        g.K = F;
+        g.N = d;
+        g.W = L.wd;
+        g.scale = L.sd;
+        g.out = X;
+        g.out_ld = d;
+        DEC_TRY((gemv_qwen<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, L.m_2, st)));
+        DEC_TRY(phase_mark(h, st, l, DEC_PHASE_FFN_DOWN));
+    }
+    return DEC_OK;
+}
+
 // One step for the batch described in h->dmeta (already uploaded).
 // head_row0 / head_rows: the rows whose logits the head computes (all by default; a prompt
 // chunk needs its last row only, or none). trace: copy each layer's residual (decode steps).
+// split: run the layers as two chains over the two halves of the rows (the metas of both
+// halves uploaded too), on st and h->side, alternating their large attentions.
 dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int* argmax, cudaStream_t st,
-                    int head_row0 = 0, int head_rows = -1, bool trace = true) {
+                    int head_row0 = 0, int head_rows = -1, bool trace = true, bool split = false) {
     if (head_rows < 0) head_rows = B;
     const dec_config& c = h->cfg;
-    const int d = c.d_model, F = c.d_ff, H = c.n_heads;
+    const int d = c.d_model;
     {
         thread_local int attr_dev = -1;
         DEC_CUDA(h, prefer_max_shared_once(k_embed, attr_dev));
     }
+    h->w = &h->chain[0];
+    h->chain[0].meta = h->dmeta;
     h->phase_n = 0;
     DEC_TRY(phase_mark(h, st, -1, 0));
     DEC_CUDA(h, launch(k_embed, dim3(B), dim3(128), 0, st, (const float*)h->tok_emb, (const float*)h->pos_emb,
                        (const StepMeta*)h->dmeta, (const int*)h->last_tok, h->x, d, h->d_table));
     DEC_TRY(phase_mark(h, st, -1, DEC_PHASE_EMBED));
-    for (int l = 0; l < c.n_layers; ++l) {
-        const LayerDev& L = h->layers[l];
-        float* kc = h->kc + l * h->self_layer_stride;
-        float* vc = h->vc + l * h->self_layer_stride;
-        // ---- q|k|v with the cache append ----
-        GemvArgs g = base_args(h, B);
-        g.x = h->x;
-        g.x_ld = d;
-        g.norm_w = L.n1w;
-        g.norm_b = L.n1b;
-        g.K = d;
-        g.N = d + 2 * kv_width(c);
-        g.W = L.wqkv;
-        g.scale = L.sqkv;
-        g.bias = L.bqkv;
-        g.out = h->q;
-        g.out_ld = d;
-        g.kc = kc;
-        g.vc = vc;
-        g.kv = self_kv_map(h);
-        g.d = d;
-        g.kvd = kv_width(c);
-        if (c.family == DEC_FAMILY_WHISPER) {
-            DEC_TRY((gemv_whisper<PRO_LN, EPI_QKV, MAP_ADJ>(h, g, st, &L.m_qkv)));
-        } else {
-            g.rope = h->rope;
-            DEC_TRY((gemv_qwen<PRO_RMS, EPI_QKV, MAP_ROPE>(h, g, L.m_qkv, st)));
+    if (!split) {
+        for (int l = 0; l < c.n_layers; ++l) {
+            DEC_TRY(layer_step(h, l, B, h->x, max_len_plus1, st, nullptr, nullptr));
+            if (trace && h->trace)
+                DEC_CUDA(h, cudaMemcpyAsync(h->trace + static_cast<size_t>(l) * B * d, h->x, size_t(B) * d * 4,
+                                            cudaMemcpyDeviceToDevice, st));
         }
-        DEC_TRY(phase_mark(h, st, l, DEC_PHASE_QKV));
-        // ---- self-attention over rows 0..len ----
-        AttnArgs at{};
-        at.q = h->q;
-        at.q_bstride = d;
-        at.k = kc;
-        at.v = vc;
-        at.slot_stride = h->self_slot_stride;
-        at.ld = c.max_cache_len;
-        at.H = H;
-        at.kv_group = H / kv_heads(c);
-        at.kv = self_kv_map(h);
-        at.mode = ATTN_SELF;
-        at.meta = h->dmeta;
-        at.out = h->ctx;
-        at.out_bstride = d;
-        at.part = h->part;
-        at.counters = h->counters;
-        at.err = h->dev_err;
-        at.drop_first_copy = (l == 0) ? h->inject_drop : 0;
-        DEC_TRY(attention(h, at, B, max_len_plus1, h->tps_self, st));
-        DEC_TRY(phase_mark(h, st, l, DEC_PHASE_SELF_ATTN));
-        at.drop_first_copy = 0;
-        // ---- output projection + residual ----
-        g = base_args(h, B);
-        g.x = h->ctx;
-        g.x_ld = d;
-        g.K = d;
-        g.N = d;
-        g.W = L.wo;
-        g.scale = L.so;
-        g.bias = L.bo;
-        g.out = h->x;
-        g.out_ld = d;
-        if (c.family == DEC_FAMILY_WHISPER) {
-            DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st, &L.m_o)));
-        } else {
-            DEC_TRY((gemv_qwen<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, L.m_o, st)));
+    } else {
+        const int n0 = split_rows(B);
+        DEC_CUDA(h, cudaEventRecord(h->ev_fork, st));
+        DEC_CUDA(h, cudaStreamWaitEvent(h->side, h->ev_fork, 0));
+        h->chain[0].meta = h->dmeta + 1;
+        h->chain[1].meta = h->dmeta + 2;
+        dec_status r = DEC_OK;
+        for (int l = 0; l < c.n_layers && r == DEC_OK; ++l) {
+            h->w = &h->chain[0];
+            r = layer_step(h, l, n0, h->x, max_len_plus1, st, l > 0 ? h->ev_attn[1] : nullptr, h->ev_attn[0]);
+            if (r != DEC_OK) break;
+            h->w = &h->chain[1];
+            r = layer_step(h, l, B - n0, h->x + static_cast<size_t>(n0) * d, max_len_plus1, h->side, h->ev_attn[0],
+                           h->ev_attn[1]);
         }
-        DEC_TRY(phase_mark(h, st, l, DEC_PHASE_O));
-        if (c.family == DEC_FAMILY_WHISPER) {
-            // ---- cross-attention block ----
-            g = base_args(h, B);
-            g.x = h->x;
-            g.x_ld = d;
-            g.norm_w = L.n2w;
-            g.norm_b = L.n2b;
-            g.K = d;
-            g.N = d;
-            g.W = L.wxq;
-            g.scale = L.sxq;
-            g.bias = L.bxq;
-            g.out = h->xq;
-            g.out_ld = d;
-            DEC_TRY((gemv_whisper<PRO_LN, EPI_STORE, MAP_ADJ>(h, g, st, &L.m_xq)));
-            DEC_TRY(phase_mark(h, st, l, DEC_PHASE_CROSS_Q));
-            at.q = h->xq;
-            at.k = h->xkc + l * h->cross_layer_stride;
-            at.v = h->xvc + l * h->cross_layer_stride;
-            at.slot_stride = h->cross_slot_stride;
-            at.ld = c.enc_len;
-            at.mode = ATTN_CROSS;
-            at.kv_group = 1;
-            at.kv.table = nullptr;
-            at.n_fixed = c.enc_len;
-            DEC_TRY(attention(h, at, B, c.enc_len, h->tps_cross, st));
-            DEC_TRY(phase_mark(h, st, l, DEC_PHASE_CROSS_ATTN));
-            g = base_args(h, B);
-            g.x = h->ctx;
-            g.x_ld = d;
-            g.K = d;
-            g.N = d;
-            g.W = L.wxo;
-            g.scale = L.sxo;
-            g.bias = L.bxo;
-            g.out = h->x;
-            g.out_ld = d;
-            DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st, &L.m_xo)));
-            DEC_TRY(phase_mark(h, st, l, DEC_PHASE_CROSS_O));
-            // ---- GELU FFN ----
-            g = base_args(h, B);
-            g.x = h->x;
-            g.x_ld = d;
-            g.norm_w = L.n3w;
-            g.norm_b = L.n3b;
-            g.K = d;
-            g.N = F;
-            g.W = L.w1;
-            g.scale = L.s1;
-            g.bias = L.b1;
-            g.out = h->ffn;
-            g.out_ld = F;
-            DEC_TRY((gemv_whisper<PRO_LN, EPI_GELU, MAP_ADJ>(h, g, st, &L.m_1)));
-            DEC_TRY(phase_mark(h, st, l, DEC_PHASE_FFN_UP));
-            g = base_args(h, B);
-            g.x = h->ffn;
-            g.x_ld = F;
-            g.K = F;
-            g.N = d;
-            g.W = L.w2;
-            g.scale = L.s2;
-            g.bias = L.b2;
-            g.out = h->x;
-            g.out_ld = d;
-            DEC_TRY((gemv_whisper<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, st, &L.m_2)));
-            DEC_TRY(phase_mark(h, st, l, DEC_PHASE_FFN_DOWN));
-        } else {
-            // ---- SwiGLU MLP ----
-            g = base_args(h, B);
-            g.x = h->x;
-            g.x_ld = d;
-            g.norm_w = L.n2w;
-            g.K = d;
-            g.N = F;
-            g.W = L.wg;
-            g.W2 = L.wu;
-            g.scale = L.sg;
-            g.scale2 = L.su;
-            g.out = h->ffn;
-            g.out_ld = F;
-            DEC_TRY((gemv_qwen<PRO_RMS, EPI_SWIGLU, MAP_DUAL>(h, g, L.m_1, st)));
-            DEC_TRY(phase_mark(h, st, l, DEC_PHASE_FFN_UP));
-            g = base_args(h, B);
-            g.x = h->ffn;
-            g.x_ld = F;
-            g.K = F;
-            g.N = d;
-            g.W = L.wd;
-            g.scale = L.sd;
-            g.out = h->x;
-            g.out_ld = d;
-            DEC_TRY((gemv_qwen<PRO_NONE, EPI_RESID, MAP_ADJ>(h, g, L.m_2, st)));
-            DEC_TRY(phase_mark(h, st, l, DEC_PHASE_FFN_DOWN));
-        }
-        if (trace && h->trace)
-            DEC_CUDA(h, cudaMemcpyAsync(h->trace + static_cast<size_t>(l) * B * d, h->x, size_t(B) * d * 4,
-                                        cudaMemcpyDeviceToDevice, st));
+        // the second chain always joins, so that a capture ends with every stream joined
+        h->w = &h->chain[0];
+        h->chain[0].meta = h->dmeta;
+        DEC_CUDA(h, cudaEventRecord(h->ev_join, h->side));
+        DEC_CUDA(h, cudaStreamWaitEvent(st, h->ev_join, 0));
+        DEC_TRY(r);
     }
     // ---- final norm + tied head + greedy argmax ----
     if (head_rows == 0) return DEC_OK;
@@ -812,12 +927,31 @@ void shrink_slot(dec_handle* h, int slot, int rows) {
 }
 
 // Upload the step description through the pinned ring.
-dec_status upload_meta(dec_handle* h, const StepMeta& m, cudaStream_t st) {
+// With split, the rows of the two chains follow as metas of their own (rows renumbered from
+// 0; page-table updates stay with the whole step's meta, which k_embed applies).
+dec_status upload_meta(dec_handle* h, const StepMeta& m, cudaStream_t st, bool split = false) {
     const int i = h->ring;
     h->ring = (h->ring + 1) % kMetaRing;
     DEC_CUDA(h, cudaEventSynchronize(h->hev[i]));
     std::memcpy(h->hmeta[i], &m, sizeof(StepMeta));
-    DEC_CUDA(h, cudaMemcpyAsync(h->dmeta, h->hmeta[i], sizeof(StepMeta), cudaMemcpyHostToDevice, st));
+    if (split) {
+        const int n0 = split_rows(m.B);
+        for (int ci = 0; ci < 2; ++ci) {
+            StepMeta& o = h->hmeta[i][1 + ci];
+            const int r0 = ci == 0 ? 0 : n0, n = ci == 0 ? n0 : m.B - n0;
+            o.B = n;
+            o.n_upd = 0;
+            for (int b = 0; b < n; ++b) {
+                o.slot[b] = m.slot[r0 + b];
+                o.tok[b] = m.tok[r0 + b];
+                o.pos[b] = m.pos[r0 + b];
+                o.len[b] = m.len[r0 + b];
+                o.fresh[b] = m.fresh[r0 + b];
+            }
+        }
+    }
+    DEC_CUDA(h, cudaMemcpyAsync(h->dmeta, h->hmeta[i], (split ? 3 : 1) * sizeof(StepMeta), cudaMemcpyHostToDevice,
+                                st));
     DEC_CUDA(h, cudaEventRecord(h->hev[i], st));
     return DEC_OK;
 }
@@ -886,7 +1020,7 @@ dec_status validate_step(dec_handle* h, int B, const int32_t* slots, const int32
 // Record the step's launch sequence into a graph for later identical steps. Capture
 // problems are not errors: the key is marked and such steps keep running eagerly.
 void capture_step(dec_handle* h, const std::array<long long, 5>& key, int B, int max_len, float* logits,
-                  int* argmax) {
+                  int* argmax, bool split) {
     if (h->graphs.size() >= 256) {
         for (auto& kv : h->graphs)
             if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
@@ -896,7 +1030,7 @@ void capture_step(dec_handle* h, const std::array<long long, 5>& key, int B, int
     int kernels = -1;
     if (cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal) == cudaSuccess) {
         const std::string saved = h->err;
-        const dec_status s = run_step(h, B, max_len, logits, argmax, h->cap_stream);
+        const dec_status s = run_step(h, B, max_len, logits, argmax, h->cap_stream, 0, -1, true, split);
         cudaGraph_t g = nullptr;
         const cudaError_t e = cudaStreamEndCapture(h->cap_stream, &g);
         if (s == DEC_OK && e == cudaSuccess && g != nullptr) {
@@ -924,7 +1058,11 @@ dec_status step_validated(dec_handle* h, StepMeta& m, int max_len, float* logits
                           cudaStream_t st) {
     m.n_upd = 0;
     for (int b = 0; b < m.B; ++b) grow_slot(h, m.slot[b], m.len[b] + 1, m);
-    DEC_TRY(upload_meta(h, m, st));
+    // two chains for large batches, unless per-layer copies, phase timing or fault injection
+    // need the single launch sequence
+    const bool split =
+        h->n_chains == 2 && m.B >= kSplitMinBatch && !h->trace && !h->phase_timing && !h->inject_drop;
+    DEC_TRY(upload_meta(h, m, st, split));
     const std::array<long long, 5> key = {m.B, (max_len + kAttnTile - 1) / kAttnTile,
                                           reinterpret_cast<long long>(logits), reinterpret_cast<long long>(argmax),
                                           reinterpret_cast<long long>(h->trace)};
@@ -937,8 +1075,8 @@ dec_status step_validated(dec_handle* h, StepMeta& m, int max_len, float* logits
         DEC_CUDA(h, cudaGraphLaunch(it->second.exec, st));
         h->last_step_kernels = it->second.kernels;
     } else {
-        DEC_TRY(run_step(h, m.B, max_len, logits, argmax, st));
-        if (it == h->graphs.end()) capture_step(h, key, m.B, max_len, logits, argmax);
+        DEC_TRY(run_step(h, m.B, max_len, logits, argmax, st, 0, -1, true, split));
+        if (it == h->graphs.end()) capture_step(h, key, m.B, max_len, logits, argmax, split);
         h->last_step_kernels = h->graphs[key].kernels;
     }
     for (int b = 0; b < m.B; ++b) {
@@ -964,6 +1102,9 @@ dec_status dec_destroy(dec_handle* h) {
         if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
     for (cudaEvent_t e : h->phase_ev) cudaEventDestroy(e);
     if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
+    if (h->side) cudaStreamDestroy(h->side);
+    for (cudaEvent_t e : {h->ev_fork, h->ev_join, h->ev_attn[0], h->ev_attn[1]})
+        if (e) cudaEventDestroy(e);
     for (void* p : h->dallocs) cudaFree(p);
     for (void* p : h->hallocs) cudaFreeHost(p);
     for (int i = 0; i < kMetaRing; ++i)
@@ -1113,29 +1254,34 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
     h->max_rows = std::max(h->max_batch, kPrefillChunk);
     const int MB = h->max_rows;
     DEC_TRY(dalloc(h, &h->x, size_t(MB) * d * 4));
-    DEC_TRY(dalloc(h, &h->q, size_t(MB) * d * 4));
-    DEC_TRY(dalloc(h, &h->ctx, size_t(MB) * d * 4));
-    DEC_TRY(dalloc(h, &h->xq, size_t(MB) * d * 4));
-    DEC_TRY(dalloc(h, &h->ffn, size_t(MB) * F * 4));
-    DEC_TRY(dalloc(h, &h->part, size_t(MB) * H * kMaxSplits * kAttnPartStride * 4));
-    DEC_TRY(dalloc(h, &h->counters, size_t(MB) * H * 4));
-    DEC_CUDA(h, cudaMemset(h->counters, 0, size_t(MB) * H * 4));
-    // tensor-core path: normalised / quantised rows and the split-K scratch of the
-    // largest plan
-    if (h->tma_ok) {
-        DEC_TRY(dalloc(h, &h->xn, size_t(MB) * std::max(d, F) * 4));
-        h->xq8_rows = std::max(MB, 32);
-        DEC_TRY(dalloc(h, &h->xq8, size_t(h->xq8_rows) * std::max(d, F)));
-        DEC_CUDA(h, cudaMemset(h->xq8, 0, size_t(h->xq8_rows) * std::max(d, F)));
-        if (!wh) {
-            const int ks[2] = {d, F};
-            for (int i = 0; i < 2; ++i)
-                for (int j = 0; j < 2; ++j)
-                    DEC_TRY(make_wmap(h, &h->m_xq8[i][j], h->xq8, h->xq8_rows, ks[i], false, j ? 32 : 16));
+    // Whisper f32 weights, tcgen05 path: each matrix's three digit planes, made once like the
+    // head's embedding planes
+    bool digit_maps_ok = h->tma_ok && wh;
+    if (digit_maps_ok && c.proj_fmt == DEC_PROJ_F32) {
+        dec_status ts = DEC_OK;
+        for (int l = 0; l < L && ts == DEC_OK; ++l) {
+            LayerDev& D = h->layers[l];
+            const void* ws[6] = {D.wqkv, D.wo, D.wxq, D.wxo, D.w1, D.w2};
+            const int ns[6] = {d + 2 * kv_width(c), d, d, d, F, d};
+            const int kk[6] = {d, d, d, d, d, F};
+            for (int m = 0; m < 6 && ts == DEC_OK; ++m) {
+                const long long nk = static_cast<long long>(ns[m]) * kk[m];
+                DEC_TRY(dalloc(h, &D.dig[m], size_t(3) * nk));
+                DEC_TRY(dalloc(h, &D.dsc[m], size_t(ns[m]) * 4));
+                DEC_CUDA(h, rowprep_digits_launch<PRO_NONE>(static_cast<const float*>(ws[m]), kk[m], nullptr, nullptr,
+                                                           0.0f, kk[m], ns[m], nk, D.dig[m], D.dsc[m], nullptr, false,
+                                                           0));
+                ts = make_wmap(h, &D.m_dig[m], D.dig[m], 3 * ns[m], kk[m], false);
+            }
         }
-        DEC_TRY(dalloc(h, &h->xs8, size_t(MB) * 4));
-        size_t pb = 16;
-        int cl = 1;
+        DEC_CUDA(h, cudaDeviceSynchronize());
+        digit_maps_ok = (ts == DEC_OK);
+        if (!digit_maps_ok) h->err.clear();
+    }
+    // split-K scratch of the largest tensor-core plan
+    size_t pb = 16;
+    int cl = 1;
+    if (h->tma_ok) {
         const int welt = c.proj_fmt == DEC_PROJ_F32 ? 4 : 1;
         auto need_f32 = [&](int n, int k, int elt) {
             const MmaPlan p = mma_plan(n, k, elt, h->num_sms);
@@ -1149,6 +1295,12 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
             pb = std::max(pb, tc_part_bytes(p, MB));
             cl = std::max(cl, tc_counters(p, MB));
         };
+        auto need_digits = [&](int n, int k) {
+            const MmaPlan p = tc_plan(n, k, h->num_sms, 3);
+            if (!p.ok) return;
+            pb = std::max(pb, tc_part_bytes(p, MB, 3));
+            cl = std::max(cl, tc_counters(p, MB));
+        };
         need_f32(c.vocab, d, 4);
         const int shapes[4][2] = {{d + 2 * kv_width(c), d}, {d, d}, {F, d}, {d, F}};
         for (const auto& sh : shapes) {
@@ -1156,15 +1308,57 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
                 need_i8(sh[0] == F ? 2 * F : sh[0], sh[1]);
             } else {
                 need_f32(sh[0], sh[1], welt);
+                need_digits(sh[0], sh[1]);
             }
         }
-        DEC_TRY(dalloc(h, &h->mma_part, pb));
-        h->mma_part_bytes = pb;
-        DEC_TRY(dalloc(h, &h->mma_cnt, size_t(cl) * 4));
-        DEC_CUDA(h, cudaMemset(h->mma_cnt, 0, size_t(cl) * 4));
-        h->mma_cnt_bytes = cl * 4;
-        h->mma_cnt_len = cl;
     }
+    // per-chain scratch: chain 0 always, chain 1 when decode batches can be split in two
+    h->n_chains = h->max_batch >= kSplitMinBatch ? 2 : 1;
+    for (int ci = 0; ci < h->n_chains; ++ci) {
+        Chain& ch = h->chain[ci];
+        DEC_TRY(dalloc(h, &ch.q, size_t(MB) * d * 4));
+        DEC_TRY(dalloc(h, &ch.ctx, size_t(MB) * d * 4));
+        DEC_TRY(dalloc(h, &ch.xq, size_t(MB) * d * 4));
+        DEC_TRY(dalloc(h, &ch.ffn, size_t(MB) * F * 4));
+        DEC_TRY(dalloc(h, &ch.part, size_t(MB) * H * kMaxSplits * kAttnPartStride * 4));
+        DEC_TRY(dalloc(h, &ch.counters, size_t(MB) * H * 4));
+        DEC_CUDA(h, cudaMemset(ch.counters, 0, size_t(MB) * H * 4));
+        if (!h->tma_ok) continue;
+        // tensor-core path: normalised / quantised rows and the split-K scratch
+        DEC_TRY(dalloc(h, &ch.xn, size_t(MB) * std::max(d, F) * 4));
+        ch.xq8_rows = std::max(MB, 32);
+        DEC_TRY(dalloc(h, &ch.xq8, size_t(ch.xq8_rows) * std::max(d, F)));
+        DEC_CUDA(h, cudaMemset(ch.xq8, 0, size_t(ch.xq8_rows) * std::max(d, F)));
+        const int ks[2] = {d, F};
+        if (!wh)
+            for (int i = 0; i < 2; ++i)
+                for (int j = 0; j < 2; ++j)
+                    DEC_TRY(make_wmap(h, &ch.m_xq8[i][j], ch.xq8, ch.xq8_rows, ks[i], false, j ? 32 : 16));
+        DEC_TRY(dalloc(h, &ch.xs8, size_t(MB) * 4));
+        if (digit_maps_ok) {
+            // Whisper tcgen05 path: the activation rows' digit planes
+            ch.xd_rows = ((std::max(MB, 32) + 31) / 32) * 32;
+            const size_t xb = size_t(3) * ch.xd_rows * std::max(d, F);
+            DEC_TRY(dalloc(h, &ch.xd3, xb));
+            DEC_CUDA(h, cudaMemset(ch.xd3, 0, xb));
+            DEC_TRY(dalloc(h, &ch.xsd, size_t(ch.xd_rows) * 4));
+            DEC_CUDA(h, cudaMemset(ch.xsd, 0, size_t(ch.xd_rows) * 4));
+            dec_status ts = DEC_OK;
+            for (int i = 0; i < 2 && ts == DEC_OK; ++i)
+                for (int j = 0; j < 2 && ts == DEC_OK; ++j)
+                    ts = make_wmap(h, &ch.m_xd3[i][j], ch.xd3, 3 * ch.xd_rows, ks[i], false, j ? 32 : 16);
+            if (ts != DEC_OK) {
+                digit_maps_ok = false;
+                h->err.clear();
+            }
+        }
+        DEC_TRY(dalloc(h, &ch.mma_part, pb));
+        ch.mma_part_bytes = pb;
+        DEC_TRY(dalloc(h, &ch.mma_cnt, size_t(cl) * 4));
+        DEC_CUDA(h, cudaMemset(ch.mma_cnt, 0, size_t(cl) * 4));
+        ch.mma_cnt_len = cl;
+    }
+    h->tcd_ok = digit_maps_ok;
     DEC_TRY(dalloc(h, &h->keys, size_t(MB) * 8));
     DEC_CUDA(h, cudaMemset(h->keys, 0, size_t(MB) * 8));
     DEC_TRY(dalloc(h, &h->head_counter, 16));
@@ -1173,7 +1367,15 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
     DEC_CUDA(h, cudaMemset(h->last_tok, 0, size_t(c.max_slots) * 4));
     DEC_TRY(dalloc(h, &h->dev_err, kStatusWords * 4));
     DEC_CUDA(h, cudaMemset(h->dev_err, 0, kStatusWords * 4));
-    DEC_TRY(dalloc(h, &h->dmeta, sizeof(StepMeta)));
+    DEC_TRY(dalloc(h, &h->dmeta, 3 * sizeof(StepMeta)));
+    h->chain[0].meta = h->dmeta;
+    h->chain[1].meta = h->dmeta + 2;
+    if (h->n_chains == 2) {
+        DEC_CUDA(h, cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking));
+        DEC_CUDA(h, cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming));
+        DEC_CUDA(h, cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming));
+        for (int i = 0; i < 2; ++i) DEC_CUDA(h, cudaEventCreateWithFlags(&h->ev_attn[i], cudaEventDisableTiming));
+    }
     DEC_TRY(dalloc(h, &h->stage_logits, size_t(h->max_batch) * c.vocab * 4));
     DEC_TRY(dalloc(h, &h->stage_argmax, size_t(h->max_batch) * 4));
     auto halloc = [&](void** p, size_t bytes) {
@@ -1187,7 +1389,7 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
     };
     for (int i = 0; i < kMetaRing; ++i) {
         void* p = nullptr;
-        DEC_TRY(halloc(&p, sizeof(StepMeta)));
+        DEC_TRY(halloc(&p, 3 * sizeof(StepMeta)));
         h->hmeta[i] = static_cast<StepMeta*>(p);
         DEC_CUDA(h, cudaEventCreateWithFlags(&h->hev[i], cudaEventDisableTiming));
     }
@@ -1524,8 +1726,11 @@ dec_status dec_reset(dec_handle* h) {
     // every kernel of the handle has ended before the counters are cleared
     DEC_CUDA(h, cudaDeviceSynchronize());
     const int MB = h->max_rows, H = h->cfg.n_heads;
-    DEC_CUDA(h, cudaMemset(h->counters, 0, size_t(MB) * H * 4));
-    if (h->mma_cnt) DEC_CUDA(h, cudaMemset(h->mma_cnt, 0, size_t(h->mma_cnt_bytes)));
+    for (int ci = 0; ci < h->n_chains; ++ci) {
+        const Chain& ch = h->chain[ci];
+        DEC_CUDA(h, cudaMemset(ch.counters, 0, size_t(MB) * H * 4));
+        if (ch.mma_cnt) DEC_CUDA(h, cudaMemset(ch.mma_cnt, 0, size_t(ch.mma_cnt_len) * 4));
+    }
     DEC_CUDA(h, cudaMemset(h->head_counter, 0, 16));
     DEC_CUDA(h, cudaMemset(h->keys, 0, size_t(MB) * 8));
     DEC_CUDA(h, cudaMemset(h->dev_err, 0, 4));   // the status word; the wait limit stays
@@ -1666,7 +1871,7 @@ dec_status dec_i8_dot(const int8_t* xq, const int8_t* wq, int32_t m, int32_t n, 
     if (e == cudaSuccess) e = cudaMemsetAsync(cnt, 0, size_t(cl) * 4, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(xs, 0, size_t(m) * 4, st);
     if (e == cudaSuccess)
-        e = proj_tc_launch<EPI_I32, MAP_ADJ>(tmp.num_sms, wmap, x16, x32, n, xs, part, pb, cnt, cl, g, st);
+        e = proj_tc_launch<EPI_I32, MAP_ADJ, 1, 1>(tmp.num_sms, wmap, x16, x32, n, m, xs, part, pb, cnt, cl, g, st);
     const cudaError_t launch_err = e;
     if (part) cudaFreeAsync(part, st);
     if (cnt) cudaFreeAsync(cnt, st);

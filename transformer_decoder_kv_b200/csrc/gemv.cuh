@@ -442,6 +442,11 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
         }
     } else {
         AccT acc[R][BT];
+        struct EpiPre {
+            float s, bias, prev;
+            float2 cs;
+            int page, row;
+        } pre[NC];
         for (int it = 0; it < n_items; ++it) {
             const int stage = it % NS;
             const uint32_t phase = static_cast<uint32_t>(it / NS) & 1u;
@@ -459,6 +464,44 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
                 for (int r = 0; r < R; ++r)
 #pragma unroll
                     for (int b = 0; b < BT; ++b) acc[r][b] = AccT(0);
+                // the epilogue's global inputs of this task (row scale, bias, residual value,
+                // RoPE table entry, cache page) are loaded now, so that their latency hides
+                // behind the dot products instead of following the reduction
+                if (task < n_tasks) {
+                    int rows[R];
+                    task_rows(task, rows);
+#pragma unroll
+                    for (int cc = 0; cc < NC; ++cc) {
+                        const int v = cc * 32 + (lane >> SH);
+                        const int r = v % R, b = v / R;
+                        const int n = rows[r];
+                        const bool live = (b < nb) && (n >= 0);
+                        const bool primary = (lane & ((1 << SH) - 1)) == 0;
+                        const int gb = b0 + b;
+                        const float* sc = (MAP == MAP_DUAL && (r & 1)) ? a.scale2 : a.scale;
+                        pre[cc].s = (EPI != EPI_I32 && (I8 || std::is_same<WT, int8_t>::value)) ? sc[live ? n : 0]
+                                                                                               : 1.0f;
+                        pre[cc].bias = (EPI != EPI_HEAD && EPI != EPI_SWIGLU && EPI != EPI_I32 && a.bias != nullptr &&
+                                        live)
+                                           ? a.bias[n]
+                                           : 0.0f;
+                        pre[cc].prev = (EPI == EPI_RESID && primary && live)
+                                           ? a.out[static_cast<long long>(gb) * a.out_ld + n]
+                                           : 0.0f;
+                        if (EPI == EPI_QKV) {
+                            const int sec = n < a.d ? 0 : (n < a.d + a.kvd ? 1 : 2);
+                            const int i = (n - (sec == 0 ? 0 : (sec == 1 ? a.d : a.d + a.kvd))) & 63;
+                            pre[cc].cs = (a.rope != nullptr && sec < 2)
+                                             ? a.rope[static_cast<long long>(a.meta->pos[gb < a.B ? gb : 0]) * 32 +
+                                                      (i & 31)]
+                                             : make_float2(1.0f, 0.0f);
+                            pre[cc].page = 0;
+                            pre[cc].row = 0;
+                            if (primary && live && sec > 0)
+                                kv_page_of(a.kv, a.meta->slot[gb], a.meta->len[gb], pre[cc].page, pre[cc].row);
+                        }
+                    }
+                }
             }
             if (task < n_tasks) {
                 const WT* wbase = reinterpret_cast<const WT*>(ring + static_cast<size_t>(stage) * stage_bytes) +
@@ -501,14 +544,13 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
                     if (EPI == EPI_I32) {
                         y = 0.0f;  // raw accumulators only: no scales exist for this epilogue
                     } else if (I8) {
-                        const float* sc = (MAP == MAP_DUAL && (r & 1)) ? a.scale2 : a.scale;
-                        y = __fmul_rn(static_cast<float>(red), __fmul_rn(s_a[b], sc[live ? n : 0]));
+                        y = __fmul_rn(static_cast<float>(red), __fmul_rn(s_a[b], pre[cc].s));
                     } else {
                         y = static_cast<float>(red);
-                        if (std::is_same<WT, int8_t>::value) y = __fmul_rn(y, a.scale[live ? n : 0]);
+                        if (std::is_same<WT, int8_t>::value) y = __fmul_rn(y, pre[cc].s);
                     }
                     if (EPI != EPI_HEAD && EPI != EPI_SWIGLU && EPI != EPI_I32 && a.bias != nullptr && live)
-                        y = __fadd_rn(y, a.bias[n]);
+                        y = __fadd_rn(y, pre[cc].bias);
                     // partner value (other row of the pair, same batch row): value index v ^ 1
                     const float yp = __shfl_xor_sync(0xffffffffu, y, 1 << SH);
                     const int gb = b0 + b;
@@ -518,10 +560,7 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
                     } else if (EPI == EPI_STORE) {
                         if (primary && live) a.out[static_cast<long long>(gb) * a.out_ld + n] = y;
                     } else if (EPI == EPI_RESID) {
-                        if (primary && live) {
-                            float* p = a.out + static_cast<long long>(gb) * a.out_ld + n;
-                            *p = __fadd_rn(*p, y);
-                        }
+                        if (primary && live) a.out[static_cast<long long>(gb) * a.out_ld + n] = __fadd_rn(pre[cc].prev, y);
                     } else if (EPI == EPI_GELU) {
                         if (primary && live) a.out[static_cast<long long>(gb) * a.out_ld + n] = gelu_tanh_f(y);
                     } else if (EPI == EPI_SWIGLU) {
@@ -534,8 +573,7 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
                         const int hh = within >> 6, i = within & 63;
                         float val = y;
                         if (a.rope != nullptr && sec < 2) {
-                            const float2 cs =
-                                a.rope[static_cast<long long>(a.meta->pos[gb < a.B ? gb : 0]) * 32 + (i & 31)];
+                            const float2 cs = pre[cc].cs;
                             // pair (i, i + 32): x_i' = x_i c - x_{i+32} s ; x_{i+32}' = x_i s + x_{i+32} c
                             if (i < 32)
                                 val = __fsub_rn(__fmul_rn(y, cs.x), __fmul_rn(yp, cs.y));
@@ -546,10 +584,8 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
                             if (sec == 0) {
                                 a.out[static_cast<long long>(gb) * a.out_ld + within] = val;
                             } else {
-                                int page, r;
-                                kv_page_of(a.kv, a.meta->slot[gb], a.meta->len[gb], page, r);
                                 float* cache = (sec == 1) ? a.kc : a.vc;
-                                cache[kv_page_off(a.kv, page, hh, r) + i] = val;
+                                cache[kv_page_off(a.kv, pre[cc].page, hh, pre[cc].row) + i] = val;
                             }
                         }
                     } else if (EPI == EPI_HEAD) {

@@ -22,12 +22,17 @@
 // CTA (192 threads, one per SM): warp 0 streams the three digit planes of 128-row
 // embedding blocks with 2-D TMA loads (128 rows x 128 bytes per plane, 128-byte swizzle,
 // no multicast) into a ring of 48 KB stages; warp 1 owns the TMEM allocation and issues
-// the MMAs (M = 128 embedding rows, N = BT batch columns, K = 32 per instruction) into one
-// of two TMEM accumulator sets, committing each stage back to the producer and each block
-// to the epilogue; warps 2..5 read the accumulators (tcgen05.ld, one TMEM lane quarter
-// each), write the logits and keep a running argmax key per batch column. The hidden
-// digit planes of the CTA's batch tile are loaded once, by TMA, in the same swizzled
-// K-major layout.
+// the MMAs (M = 128 embedding rows, K = 32 per instruction) into one of two TMEM
+// accumulator sets, committing each stage back to the producer and each block to the
+// epilogue; warps 2..5 read the accumulators (tcgen05.ld, one TMEM lane quarter each),
+// write the logits and keep a running argmax key per batch column. The hidden digit
+// planes of the CTA's batch tile are loaded once, by TMA, in the same swizzled K-major
+// layout, the three planes of each 128-column chunk stacked along N (D1 | D2 | D3, BT rows
+// each) and the accumulators A0 | A1 | A2 side by side in TMEM: then E1 [D1 D2 D3]
+// (N = 3 BT), E2 [D1 D2] (N = 2 BT, into A1 | A2) and E3 D1 (N = BT, into A2) are the six
+// products in three instructions. An M = 128, K = 32 int8 MMA takes about 135 SM cycles
+// whatever its N (measured on B200 from N = 16 to 256), so the instruction count, not the
+// columns, sets the MMA time of a block.
 #pragma once
 
 #include <cuda.h>
@@ -87,49 +92,60 @@ __device__ __forceinline__ void digits3(float v, float inv, int& d1, int& d2, in
 }
 
 // One row's three digit planes, computed by one warp (the final LayerNorm / RMSNorm first
-// when PRO says so, with the CUDA-core projection prologue's arithmetic): `sink(k4, p1, p2,
-// p3)` receives the packed digits of elements 4 k4 .. 4 k4 + 3; returns the row scale.
-// Every caller uses this one function, so the digits do not depend on where they are made.
-template <int PRO, class Sink>
-__device__ __forceinline__ float row_digits_warp(const float* __restrict__ x, const float* __restrict__ gw,
-                                                 const float* __restrict__ gb, float eps, int K, int lane,
-                                                 Sink sink, int* s12 = nullptr) {
-    const float4* xr = reinterpret_cast<const float4*>(x);
+// when PRO says so, with the CUDA-core projection prologue's arithmetic): `get(j)` returns
+// the row's float4 element lane + 32 j (j < jmax; elements at or past K / 4 are skipped), and
+// `sink(k4, p1, p2, p3)` receives the packed digits of elements 4 k4 .. 4 k4 + 3; returns the
+// row scale. Every caller uses this one function, whether the row comes from memory or from
+// registers, so the digits do not depend on where they are made.
+template <int PRO, class Get, class Sink>
+__device__ __forceinline__ float row_digits_passes(Get get, int jmax, const float* __restrict__ gw,
+                                                   const float* __restrict__ gb, float eps, int K, int lane,
+                                                   Sink sink, int* s12) {
     const int K4 = K >> 2;
     float mu = 0.0f, rstd = 1.0f;
     if (PRO == PRO_LN) {
         float sum = 0.0f;
-        for (int k = lane; k < K4; k += 32) {
-            const float4 v = xr[k];
-            sum += (v.x + v.y) + (v.z + v.w);
-        }
+#pragma unroll
+    #pragma unroll
+    for (int j = 0; j < jmax; ++j)
+            if (lane + 32 * j < K4) {
+                const float4 v = get(j);
+                sum += (v.x + v.y) + (v.z + v.w);
+            }
         mu = warp_sum(sum) / static_cast<float>(K);
         float var = 0.0f;
-        for (int k = lane; k < K4; k += 32) {
-            const float4 v = xr[k];
-            const float d0 = v.x - mu, d1 = v.y - mu, d2 = v.z - mu, d3 = v.w - mu;
-            var = fmaf(d0, d0, var);
-            var = fmaf(d1, d1, var);
-            var = fmaf(d2, d2, var);
-            var = fmaf(d3, d3, var);
-        }
+#pragma unroll
+    #pragma unroll
+    for (int j = 0; j < jmax; ++j)
+            if (lane + 32 * j < K4) {
+                const float4 v = get(j);
+                const float d0 = v.x - mu, d1 = v.y - mu, d2 = v.z - mu, d3 = v.w - mu;
+                var = fmaf(d0, d0, var);
+                var = fmaf(d1, d1, var);
+                var = fmaf(d2, d2, var);
+                var = fmaf(d3, d3, var);
+            }
         var = warp_sum(var) / static_cast<float>(K);
         rstd = 1.0f / sqrtf(var + eps);
     } else if (PRO == PRO_RMS) {
         float ss = 0.0f;
-        for (int k = lane; k < K4; k += 32) {
-            const float4 v = xr[k];
-            ss = fmaf(v.x, v.x, ss);
-            ss = fmaf(v.y, v.y, ss);
-            ss = fmaf(v.z, v.z, ss);
-            ss = fmaf(v.w, v.w, ss);
-        }
+#pragma unroll
+    #pragma unroll
+    for (int j = 0; j < jmax; ++j)
+            if (lane + 32 * j < K4) {
+                const float4 v = get(j);
+                ss = fmaf(v.x, v.x, ss);
+                ss = fmaf(v.y, v.y, ss);
+                ss = fmaf(v.z, v.z, ss);
+                ss = fmaf(v.w, v.w, ss);
+            }
         ss = warp_sum(ss) / static_cast<float>(K);
         rstd = 1.0f / sqrtf(ss + eps);
     }
-    auto normed = [&](int k) {
-        float4 v = xr[k];
+    auto normed = [&](int j) {
+        float4 v = get(j);
         if (PRO != PRO_NONE) {
+            const int k = lane + 32 * j;
             const float4 g = __ldg(reinterpret_cast<const float4*>(gw) + k);
             float4 be = make_float4(0.f, 0.f, 0.f, 0.f);
             if (PRO == PRO_LN) be = __ldg(reinterpret_cast<const float4*>(gb) + k);
@@ -139,29 +155,33 @@ __device__ __forceinline__ float row_digits_warp(const float* __restrict__ x, co
         return v;
     };
     float amax = 0.0f;
-    for (int k = lane; k < K4; k += 32) {
-        const float4 v = normed(k);
-        amax = fmaxf(fmaxf(amax, fabsf(v.x)), fmaxf(fabsf(v.y), fmaxf(fabsf(v.z), fabsf(v.w))));
-    }
+#pragma unroll
+    for (int j = 0; j < jmax; ++j)
+        if (lane + 32 * j < K4) {
+            const float4 v = normed(j);
+            amax = fmaxf(fmaxf(amax, fabsf(v.x)), fmaxf(fabsf(v.y), fmaxf(fabsf(v.z), fabsf(v.w))));
+        }
     amax = warp_max(amax);
     const float inv = amax > 0.0f ? 127.0f / amax : 0.0f;
     int sum1 = 0, sum2 = 0;
-    for (int k = lane; k < K4; k += 32) {
-        const float4 v = normed(k);
-        const float e[4] = {v.x, v.y, v.z, v.w};
-        uint32_t p1 = 0, p2 = 0, p3 = 0;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            int a, b, c;
-            digits3(e[j], inv, a, b, c);
-            sum1 += abs(a);
-            sum2 += abs(b);
-            p1 |= (static_cast<uint32_t>(a) & 0xffu) << (8 * j);
-            p2 |= (static_cast<uint32_t>(b) & 0xffu) << (8 * j);
-            p3 |= (static_cast<uint32_t>(c) & 0xffu) << (8 * j);
+    for (int j = 0; j < jmax; ++j)
+        if (lane + 32 * j < K4) {
+            const float4 v = normed(j);
+            const float e[4] = {v.x, v.y, v.z, v.w};
+            uint32_t p1 = 0, p2 = 0, p3 = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                int d1, d2, d3;
+                digits3(e[i], inv, d1, d2, d3);
+                sum1 += abs(d1);
+                sum2 += abs(d2);
+                p1 |= (static_cast<uint32_t>(d1) & 0xffu) << (8 * i);
+                p2 |= (static_cast<uint32_t>(d2) & 0xffu) << (8 * i);
+                p3 |= (static_cast<uint32_t>(d3) & 0xffu) << (8 * i);
+            }
+            sink(lane + 32 * j, p1, p2, p3);
         }
-        sink(k, p1, p2, p3);
-    }
     if (s12) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -172,6 +192,16 @@ __device__ __forceinline__ float row_digits_warp(const float* __restrict__ x, co
         s12[1] = sum2;
     }
     return amax / 127.0f;
+}
+
+// The same for a row read from memory (x: K floats, 16-byte aligned).
+template <int PRO, class Sink>
+__device__ __forceinline__ float row_digits_warp(const float* __restrict__ x, const float* __restrict__ gw,
+                                                 const float* __restrict__ gb, float eps, int K, int lane,
+                                                 Sink sink, int* s12 = nullptr) {
+    const float4* xr = reinterpret_cast<const float4*>(x);
+    return row_digits_passes<PRO>([&](int j) { return xr[lane + 32 * j]; }, ((K >> 2) + 31) / 32, gw, gb, eps, K,
+                                  lane, sink, s12);
 }
 
 // One logit from the three exact digit-product sums: s_n s_b (A0 + (A1 + A2 / 254) / 254), every
@@ -202,7 +232,9 @@ __device__ __forceinline__ float argmax_key_value(unsigned long long k) {
 }
 
 // Digit planes of rows of a row-major f32 matrix: out[p][r][k], scale[r]. One warp per
-// row (the embedding once at load; the hidden rows of batches above 16 every step).
+// row (the embedding and f32 projection weights once at load; the hidden rows of batches
+// above 16 and the Whisper projections' input rows every step).
+constexpr int kDigitsRegK4 = 12;   // rows of K <= 32 * 12 * 4 = 1536 stay in registers
 template <int PRO>
 __global__ void __launch_bounds__(128) k_rowprep_digits(const float* __restrict__ x, int x_ld,
                                                         const float* __restrict__ gw, const float* __restrict__ gb,
@@ -218,13 +250,25 @@ __global__ void __launch_bounds__(128) k_rowprep_digits(const float* __restrict_
     uint32_t* o2 = reinterpret_cast<uint32_t*>(out + plane_stride + static_cast<long long>(r) * K);
     uint32_t* o3 = reinterpret_cast<uint32_t*>(out + 2 * plane_stride + static_cast<long long>(r) * K);
     int s12[2];
-    const float sc = row_digits_warp<PRO>(x + static_cast<long long>(r) * x_ld, gw, gb, eps, K, lane,
-                                          [&](int k4, uint32_t p1, uint32_t p2, uint32_t p3) {
-                                              o1[k4] = p1;
-                                              o2[k4] = p2;
-                                              o3[k4] = p3;
-                                          },
-                                          s12);
+    auto sink = [&](int k4, uint32_t p1, uint32_t p2, uint32_t p3) {
+        o1[k4] = p1;
+        o2[k4] = p2;
+        o3[k4] = p3;
+    };
+    const float* xrow = x + static_cast<long long>(r) * x_ld;
+    float sc;
+    if ((K >> 2) <= 32 * kDigitsRegK4) {
+        // the row read once into registers (every loop of the passes fully unrolled over the
+        // compile-time bound); same elements, same order as the memory path
+        const float4* xr = reinterpret_cast<const float4*>(xrow);
+        float4 rv[kDigitsRegK4];
+#pragma unroll
+        for (int j = 0; j < kDigitsRegK4; ++j)
+            rv[j] = lane + 32 * j < (K >> 2) ? xr[lane + 32 * j] : make_float4(0.f, 0.f, 0.f, 0.f);
+        sc = row_digits_passes<PRO>([&](int j) { return rv[j]; }, kDigitsRegK4, gw, gb, eps, K, lane, sink, s12);
+    } else {
+        sc = row_digits_warp<PRO>(xrow, gw, gb, eps, K, lane, sink, s12);
+    }
     if (lane == 0) {
         scale[r] = sc;
         if (sums) {
@@ -284,6 +328,14 @@ __host__ __device__ constexpr uint32_t idesc_i8(int n) {
 template <int BT>
 struct HeadTmemLd;
 template <>
+struct HeadTmemLd<8> {
+    __device__ __forceinline__ static void run(uint32_t taddr, int (&r)[8]) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                     : "r"(taddr));
+    }
+};
+template <>
 struct HeadTmemLd<16> {
     __device__ __forceinline__ static void run(uint32_t taddr, int (&r)[16]) {
         asm volatile(
@@ -325,15 +377,18 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
     constexpr int kStage = WD * kHeadPlaneBox;
     constexpr int ACC = 3 * BT;                           // TMEM columns of one accumulator set
     constexpr uint32_t TCOLS = BT == 16 ? 128 : 256;      // two sets, power of two
-    constexpr uint32_t IDESC = idesc_i8(BT);
+    constexpr int XC = 3 * BT * 128;                      // one chunk of the three stacked hidden planes
+    constexpr uint32_t IDESC1 = idesc_i8(3 * BT);         // E1 against D1 | D2 | D3
+    constexpr uint32_t IDESC2 = idesc_i8(2 * BT);         // E2 against D1 | D2
+    constexpr uint32_t IDESC3 = idesc_i8(BT);             // E3 against D1
     const int nch = (A.K + kHeadKC - 1) / kHeadKC;
-    const int xplane = nch * BT * 128;                    // bytes of one hidden digit plane
+    const int xplane = nch * BT * 128;                    // bytes of one hidden digit plane (all chunks)
 
     extern __shared__ unsigned char head_smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(head_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     unsigned char* ring = smem;                                             // NS stages
-    unsigned char* sx = smem + static_cast<size_t>(NS) * kStage;            // 3 x xplane
+    unsigned char* sx = smem + static_cast<size_t>(NS) * kStage;            // nch chunks of XC bytes
     __shared__ __align__(8) uint64_t full[kHeadMaxStagesW1], empty[kHeadMaxStagesW1];   // NS <= 8 stages
     __shared__ __align__(8) uint64_t tfull[2], tempty[2], bar_x, bar_done;
     __shared__ uint32_t s_tmem;
@@ -412,10 +467,10 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
                 A.x + static_cast<long long>(b0 + b) * A.x_ld, A.norm_w, A.norm_b, A.eps, A.K, lane,
                 [&](int k4, uint32_t p1, uint32_t p2, uint32_t p3) {
                     const int j = (4 * k4) & 127;   // byte within the 128-byte row of chunk (4 k4) / 128
-                    const int off = ((4 * k4) >> 7) * BT * 128 + b * 128 + (((j >> 4) ^ (b & 7)) << 4) + (j & 15);
+                    const int off = ((4 * k4) >> 7) * XC + b * 128 + (((j >> 4) ^ (b & 7)) << 4) + (j & 15);
                     *reinterpret_cast<uint32_t*>(sx + off) = p1;
-                    *reinterpret_cast<uint32_t*>(sx + xplane + off) = p2;
-                    *reinterpret_cast<uint32_t*>(sx + 2 * xplane + off) = p3;
+                    *reinterpret_cast<uint32_t*>(sx + BT * 128 + off) = p2;
+                    *reinterpret_cast<uint32_t*>(sx + 2 * BT * 128 + off) = p3;
                 });
             if (lane == 0) s_xs[b] = sc;
         }
@@ -429,7 +484,7 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
             mbar_arrive_expect_tx(&bar_x, 3 * xplane);
             for (int p = 0; p < 3; ++p)
                 for (int c = 0; c < nch; ++c)
-                    tma_load_2d(sx + p * xplane + c * BT * 128, BT == 16 ? &A.xmap16 : &A.xmap32, c * kHeadKC,
+                    tma_load_2d(sx + c * XC + p * BT * 128, BT == 16 ? &A.xmap16 : &A.xmap32, c * kHeadKC,
                                 p * A.MB + b0, &bar_x);
         }
         // remaining weight stages
@@ -465,25 +520,18 @@ __global__ void __launch_bounds__(kHeadThreads, 1) k_head_tc(const __grid_consta
 #pragma unroll
                 for (int s = 0; s < kHeadKC / 32; ++s) {
                     const uint64_t w1 = smem_desc_sw128(st) + 2 * s;
-                    const unsigned char* xc = sx + c * BT * 128;
-                    const uint64_t x1 = smem_desc_sw128(xc) + 2 * s, x2 = smem_desc_sw128(xc + xplane) + 2 * s,
-                                   x3 = smem_desc_sw128(xc + 2 * xplane) + 2 * s;
+                    // the chunk's hidden planes D1 | D2 | D3 stacked along N; the accumulators
+                    // A0 | A1 | A2 side by side in TMEM
+                    const uint64_t xs = smem_desc_sw128(sx + c * XC) + 2 * s;
                     const uint32_t first = (c == 0 && s == 0) ? 0u : 1u;
+                    // E1 D1 -> A0, E1 D2 -> A1, E1 D3 -> A2 (the int8 head stops here)
+                    umma_i8(dacc, w1, xs, IDESC1, first);
                     if (WD == 3) {
-                        // six digit products, grouped by weight into three accumulators
+                        // E2 D1 -> A1, E2 D2 -> A2; E3 D1 -> A2
                         const uint64_t w2 = smem_desc_sw128(st + kHeadPlaneBox) + 2 * s,
                                        w3 = smem_desc_sw128(st + 2 * kHeadPlaneBox) + 2 * s;
-                        umma_i8(dacc, w1, x1, IDESC, first);
-                        umma_i8(dacc + BT, w1, x2, IDESC, first);
-                        umma_i8(dacc + BT, w2, x1, IDESC, 1u);
-                        umma_i8(dacc + 2 * BT, w1, x3, IDESC, first);
-                        umma_i8(dacc + 2 * BT, w2, x2, IDESC, 1u);
-                        umma_i8(dacc + 2 * BT, w3, x1, IDESC, 1u);
-                    } else {
-                        // the embedding's first digit against the hidden row's three
-                        umma_i8(dacc, w1, x1, IDESC, first);
-                        umma_i8(dacc + BT, w1, x2, IDESC, first);
-                        umma_i8(dacc + 2 * BT, w1, x3, IDESC, first);
+                        umma_i8(dacc + BT, w2, xs, IDESC2, 1u);
+                        umma_i8(dacc + 2 * BT, w3, xs, IDESC3, 1u);
                     }
                 }
                 umma_commit(&empty[stage]);   // stage free once these MMAs have read it

@@ -8,15 +8,22 @@
 // dequantisation y = float(acc) * (a_b * s_n) + bias (decoder_qwen2.rs,
 // gemv_i8_bias_prequant) are bit-identical to the dp4a kernel used below batch 8.
 //
-// CTA (192 threads, one per SM): warp 0 streams 128-row x 128-column weight boxes by TMA
+// CTA (320 threads, one per SM): warp 0 streams 128-row x 128-column weight boxes by TMA
 // (no multicast) into a ring of 16 KB stages and loads the CTA's K slice of the activation
 // rows once; warp 1 owns the TMEM allocation (two accumulator sets) and issues the MMAs,
 // committing each stage back to the producer and each finished row block to the
-// epilogue; warps 2..5 read the accumulators with tcgen05.ld (one TMEM lane quarter, i.e.
-// 32 weight rows, each), one row and all batch columns per thread. K is split across CTA
+// epilogue; warps 2..9 read the accumulators with tcgen05.ld. A warp may only touch the
+// TMEM lane quarter (warp id mod 4), i.e. 32 weight rows, so two warps share each quarter
+// and each finishes one row and half of the batch columns per thread, which halves the
+// serial chain of dequantise-and-store work behind the last MMA. A tcgen05.mma .kind::i8 of
+// M = 128, K = 32 takes about 135 SM cycles whatever its N (measured on B200 for N = 16 to
+// 256, with one or many independent accumulators), so the MMA phase costs one such time per
+// instruction: the activation digit planes of a batch tile are stacked along N in shared
+// memory, and one instruction multiplies a weight plane by all the planes it pairs with.
+// K is split across CTA
 // groups so that small matrices still reach every SM; with more than one slice, each
 // epilogue warp stores its exact partial sums and the last of the n_ks warps that own a
-// 32-row group (an arrival count; nothing waits) adds the slices and finishes.
+// 32-row, half-tile group (an arrival count; nothing waits) adds the slices and finishes.
 //
 // Row maps: the NEOX RoPE pair (i, i + 32) of a head and the SwiGLU pair (gate n, up n) are
 // stored in adjacent weight rows (MAP_ROPE: row 2j holds i = j, row 2j + 1 holds i = 32 + j
@@ -30,20 +37,22 @@
 
 namespace dec {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 320;                 // producer, MMA issuer, 8 epilogue warps
+constexpr int kTcEpiWarps = 8;                  // two per TMEM lane quarter, half the columns each
 constexpr int kTcKC = 128;                      // K per stage (one 128-byte box)
 constexpr int kTcStageBytes = 128 * kTcKC;      // 16 KB
 constexpr int kTcMaxStages = 12;
 constexpr int kTcMaxBT = 32;
-constexpr size_t kTcXBudget = 96 * 1024;        // activation slice bytes at most
+constexpr size_t kTcXBudget = 120 * 1024;       // activation slice bytes at most (all planes)
 
 struct TcArgs {
-    CUtensorMap wmap;      // int8 weights [n_rows, K]: box {128 bytes, 128 rows}
-    CUtensorMap xmap;      // int8 activations [MB, K]: box {128 bytes, BT rows}
+    CUtensorMap wmap;      // int8 weight planes [WD * n_rows, K]: box {128 bytes, 128 rows}
+    CUtensorMap xmap;      // int8 activation planes [XD * MB, K]: box {128 bytes, BT rows}
     const float* xs;       // [B] activation scales
     int* part;             // split-K partial sums
-    int* cnt;              // arrival counts per (row block, batch tile, lane quarter), zero between launches
+    int* cnt;              // arrival counts per (row block, batch tile, lane quarter, half), zero between launches
     int n_ks, ksl, n_rows, n_by;
+    int MB;                // rows of one activation plane
     GemvArgs g;            // shapes and epilogue arguments
 };
 
@@ -58,18 +67,48 @@ __host__ __device__ __forceinline__ int tc_logical_row(int p) {
     return p;
 }
 
-template <int BT, int EPI, int MAP>
+// Digit planes of the two operands: XD activation planes and WD weight planes, each an
+// int8 matrix; the products summed into accumulator j are those whose weight is 254^-j.
+//   XD = 1, WD = 1 (W8A8):   A0 = W X
+//   XD = 3, WD = 1 (W8A32):  A0 = W X1, A1 = W X2, A2 = W X3
+//   XD = 3, WD = 3 (f32):    A0 = W1 X1, A1 = W1 X2 + W2 X1, A2 = W1 X3 + W2 X2 + W3 X1
+// In shared memory the activation planes of each 128-column chunk are stacked along N
+// (plane p in rows p BT .. p BT + BT - 1), and the accumulators A0 | A1 | A2 sit side by side
+// in TMEM, so W1 [X1; X2; X3] (N = 3 BT) writes all three at once, W2 [X1; X2] (N = 2 BT) adds
+// into A1 | A2 and W3 X1 (N = BT) into A2: one, one and three instructions per K step.
+template <int XD, int WD>
+struct TcDigits {
+    static_assert((XD == 1 && WD == 1) || (XD == 3 && (WD == 1 || WD == 3)), "digit planes");
+};
+
+// TMEM columns of one CTA: `sets` accumulator sets (two when the CTA owns more than one row
+// block, so that the epilogue of one overlaps the MMAs of the next) of XD BT columns; at most
+// 256, so that two CTAs of consecutive kernels can hold TMEM at once.
+__host__ __device__ inline uint32_t tc_tmem_cols(int xd, int bt, int sets) {
+    const int need = sets * xd * bt;
+    uint32_t t = 32;
+    while (t < static_cast<uint32_t>(need)) t <<= 1;
+    return t;
+}
+
+template <int BT, int EPI, int MAP, int XD, int WD>
 __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant__ TcArgs A, int NS) {
     static_assert(BT == 16 || BT == 32, "batch tile");
-    constexpr uint32_t TCOLS = 2 * BT >= 32 ? 2 * BT : 32;   // two accumulator sets
-    constexpr uint32_t IDESC = idesc_i8(BT);
+    static_assert(XD == 1 || (MAP == MAP_ADJ && EPI != EPI_I32 && EPI != EPI_SWIGLU), "digit planes: plain rows");
+    (void)sizeof(TcDigits<XD, WD>);
+    constexpr int NACC = XD;                              // accumulators A0 .. A(XD-1)
+    constexpr int kStage = WD * kTcStageBytes;
+    constexpr int XC = XD * BT * 128;                     // bytes of one chunk's stacked planes
+    constexpr uint32_t IDESC1 = idesc_i8(XD * BT);        // W1 against every activation plane
+    constexpr uint32_t IDESC2 = idesc_i8(2 * BT);         // W2 against X1, X2
+    constexpr uint32_t IDESC3 = idesc_i8(BT);             // W3 against X1
     const GemvArgs& a = A.g;
 
     extern __shared__ unsigned char tc_smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     unsigned char* ring = smem;
-    unsigned char* sx = smem + static_cast<size_t>(NS) * kTcStageBytes;
+    unsigned char* sx = smem + static_cast<size_t>(NS) * kStage;
     __shared__ __align__(8) uint64_t full[kTcMaxStages], empty[kTcMaxStages];
     __shared__ __align__(8) uint64_t tfull[2], tempty[2], bar_x, bar_done;
     __shared__ uint32_t s_tmem;
@@ -91,6 +130,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
     const int nch = (klen + kTcKC - 1) / kTcKC;
     const int my_blocks = c0 < n_blocks ? (n_blocks - 1 - c0) / cps + 1 : 0;
     const int n_items = my_blocks * nch;
+    const int sets = my_blocks > 1 ? 2 : 1;
+    const int setc = XD * BT;                            // TMEM columns of one accumulator set
+    const uint32_t tcols = tc_tmem_cols(XD, BT, sets);
 
     if (tid == 0) {
         for (int i = 0; i < NS; ++i) {
@@ -99,7 +141,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], 4);
+            mbar_init(&tempty[i], kTcEpiWarps);
         }
         mbar_init(&bar_x, 1);
         mbar_init(&bar_done, 1);
@@ -107,7 +149,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
         s_fail = 0;
     }
     if (warp == 1) {
-        tmem_alloc(&s_tmem, TCOLS);
+        tmem_alloc(&s_tmem, tcols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -115,12 +157,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
     tc_fence_after();
     const uint32_t tbase = s_tmem;
 
+    // weight stage `it`: the WD planes of one 128-row block and 128 columns of K
     auto issue = [&](int it) {
         const int jb = c0 + (it / nch) * cps;
         const int c = it % nch;
-        mbar_arrive_expect_tx(&full[it % NS], kTcStageBytes);
-        tma_load_2d(ring + static_cast<size_t>(it % NS) * kTcStageBytes, &A.wmap, kstart + c * kTcKC, jb * 128,
-                    &full[it % NS]);
+        unsigned char* dst = ring + static_cast<size_t>(it % NS) * kStage;
+        mbar_arrive_expect_tx(&full[it % NS], kStage);
+#pragma unroll
+        for (int p = 0; p < WD; ++p)
+            tma_load_2d(dst + p * kTcStageBytes, &A.wmap, kstart + c * kTcKC, p * A.n_rows + jb * 128,
+                        &full[it % NS]);
     };
     int n_issued = 0;
     if (warp == 0 && lane == 0)
@@ -141,10 +187,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
     __syncthreads();
 
     if (warp == 0 && lane == 0) {
-        // the activation slice of this batch tile, one box per 128 columns
-        mbar_arrive_expect_tx(&bar_x, static_cast<uint32_t>(nch) * BT * 128);
-        for (int c = 0; c < nch; ++c)
-            tma_load_2d(sx + c * BT * 128, &A.xmap, kstart + c * kTcKC, b0, &bar_x);
+        // the activation slice of this batch tile: XD planes, one box per 128 columns
+        mbar_arrive_expect_tx(&bar_x, static_cast<uint32_t>(XD * nch) * BT * 128);
+        for (int p = 0; p < XD; ++p)
+            for (int c = 0; c < nch; ++c)
+                tma_load_2d(sx + c * XC + p * BT * 128, &A.xmap, kstart + c * kTcKC, p * A.MB + b0, &bar_x);
         for (int it = n_issued; it < n_items; ++it) {
             if (!mbar_wait_bounded(&empty[it % NS], static_cast<uint32_t>(it / NS - 1) & 1u, a.err)) {
                 s_fail = 1;
@@ -165,7 +212,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
                 break;
             }
             tc_fence_after();
-            const uint32_t dacc = tbase + static_cast<uint32_t>(ab * BT);
+            const uint32_t dset = tbase + static_cast<uint32_t>(ab * setc);
             for (int c = 0; c < nch; ++c, ++it) {
                 const int stage = it % NS;
                 if (!mbar_wait_bounded(&full[stage], static_cast<uint32_t>(it / NS) & 1u, a.err)) {
@@ -173,11 +220,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
                     break;
                 }
                 tc_fence_after();
-                const uint64_t wd = smem_desc_sw128(ring + static_cast<size_t>(stage) * kTcStageBytes);
-                const uint64_t xd = smem_desc_sw128(sx + c * BT * 128);
+                const unsigned char* st = ring + static_cast<size_t>(stage) * kStage;
 #pragma unroll
-                for (int s = 0; s < kTcKC / 32; ++s)
-                    umma_i8(dacc, wd + 2 * s, xd + 2 * s, IDESC, (c == 0 && s == 0) ? 0u : 1u);
+                for (int s = 0; s < kTcKC / 32; ++s) {
+                    const uint32_t first = (c == 0 && s == 0) ? 0u : 1u;
+                    const uint64_t w1 = smem_desc_sw128(st) + 2 * s;
+                    const uint64_t xs = smem_desc_sw128(sx + c * XC) + 2 * s;
+                    umma_i8(dset, w1, xs, IDESC1, first);
+                    if (WD == 3) {
+                        const uint64_t w2 = smem_desc_sw128(st + kTcStageBytes) + 2 * s,
+                                       w3 = smem_desc_sw128(st + 2 * kTcStageBytes) + 2 * s;
+                        umma_i8(dset + BT, w2, xs, IDESC2, 1u);
+                        umma_i8(dset + 2 * BT, w3, xs, IDESC3, 1u);
+                    }
+                }
                 umma_commit(&empty[stage]);
             }
             if (!ok) break;
@@ -187,8 +243,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
         umma_commit(&bar_done);
         mbar_wait_bounded(&bar_done, 0, nullptr);
     } else if (warp >= 2) {
-        // ---- epilogue: lane quarter q holds weight rows 32 q .. 32 q + 31 ----
+        // ---- epilogue: lane quarter q holds weight rows 32 q .. 32 q + 31; two warps per
+        // quarter, each finishing half of the batch columns (c0b .. c0b + HB - 1) ----
+        constexpr int HB = BT / 2;
         const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
+        const int c0b = half * HB;
         for (int i = 0; i < my_blocks; ++i) {
             const int ab = i & 1;
             if (!mbar_wait_bounded(&tfull[ab], static_cast<uint32_t>(i >> 1) & 1u, a.err)) {
@@ -196,19 +256,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
                 break;
             }
             tc_fence_after();
-            int acc[BT];
-            HeadTmemLd<BT>::run(tbase + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BT), acc);
+            int acc[NACC][HB];
+            const uint32_t tq = tbase + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * setc + c0b);
+#pragma unroll
+            for (int j = 0; j < NACC; ++j) HeadTmemLd<HB>::run(tq + static_cast<uint32_t>(j * BT), acc[j]);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[ab]);
             const int jb = c0 + i * cps;
             if (A.n_ks > 1) {
-                // exact partial sums of this slice: each thread's BT values contiguous
-                const long long grp = (static_cast<long long>(jb) * n_by + by) * 4 + q;
-                int4* mine = reinterpret_cast<int4*>(A.part + ((grp * A.n_ks + ks) * 32 + lane) * BT);
+                // exact partial sums of this slice: each thread's NACC x HB values contiguous
+                constexpr int NV = NACC * HB;
+                const long long grp = ((static_cast<long long>(jb) * n_by + by) * 4 + q) * 2 + half;
+                int4* mine = reinterpret_cast<int4*>(A.part + ((grp * A.n_ks + ks) * 32 + lane) * NV);
 #pragma unroll
-                for (int v = 0; v < BT / 4; ++v) mine[v] = make_int4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+                for (int j = 0; j < NACC; ++j)
+#pragma unroll
+                    for (int v = 0; v < HB / 4; ++v)
+                        mine[j * (HB / 4) + v] =
+                            make_int4(acc[j][4 * v], acc[j][4 * v + 1], acc[j][4 * v + 2], acc[j][4 * v + 3]);
                 __threadfence();
                 __syncwarp();
                 int last = 0;
@@ -217,23 +284,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
                 if (!last) continue;
                 __threadfence();
 #pragma unroll
-                for (int b = 0; b < BT; ++b) acc[b] = 0;
+                for (int j = 0; j < NACC; ++j)
+#pragma unroll
+                    for (int b = 0; b < HB; ++b) acc[j][b] = 0;
                 for (int sl = 0; sl < A.n_ks; ++sl) {
-                    const int4* src = reinterpret_cast<const int4*>(A.part + ((grp * A.n_ks + sl) * 32 + lane) * BT);
-                    int4 v4[BT / 4];
+                    const int4* src = reinterpret_cast<const int4*>(A.part + ((grp * A.n_ks + sl) * 32 + lane) * NV);
+                    int4 v4[NV / 4];
 #pragma unroll
-                    for (int v = 0; v < BT / 4; ++v) v4[v] = __ldcg(src + v);
+                    for (int v = 0; v < NV / 4; ++v) v4[v] = __ldcg(src + v);
 #pragma unroll
-                    for (int v = 0; v < BT / 4; ++v) {
-                        acc[4 * v] += v4[v].x;
-                        acc[4 * v + 1] += v4[v].y;
-                        acc[4 * v + 2] += v4[v].z;
-                        acc[4 * v + 3] += v4[v].w;
-                    }
+                    for (int j = 0; j < NACC; ++j)
+#pragma unroll
+                        for (int v = 0; v < HB / 4; ++v) {
+                            acc[j][4 * v] += v4[j * (HB / 4) + v].x;
+                            acc[j][4 * v + 1] += v4[j * (HB / 4) + v].y;
+                            acc[j][4 * v + 2] += v4[j * (HB / 4) + v].z;
+                            acc[j][4 * v + 3] += v4[j * (HB / 4) + v].w;
+                        }
                 }
                 if (lane == 0) A.cnt[grp] = 0;
             }
-            // ---- dequantise and finish row p for every batch column ----
+            // ---- dequantise and finish row p for this warp's batch columns ----
             // Every global input of the epilogue (row scale, bias, the residual values, the
             // RoPE table entries) is loaded before the first store: a load placed after a
             // store to memory it might alias would wait for that store, one L2 round trip
@@ -252,42 +323,55 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
                 col = within & 63;
             }
             constexpr bool kRope = EPI == EPI_QKV && MAP == MAP_ROPE;
-            float prev[EPI == EPI_RESID ? BT : 1];
-            float2 cs[kRope ? BT : 1];
+            float prev[EPI == EPI_RESID ? HB : 1];
+            float2 cs[kRope ? HB : 1];
             if (EPI == EPI_RESID) {
 #pragma unroll
-                for (int b = 0; b < BT; ++b)
-                    prev[b] = (b < nb && row_live) ? a.out[static_cast<long long>(b0 + b) * a.out_ld + n] : 0.0f;
+                for (int j = 0; j < HB; ++j) {
+                    const int b = c0b + j;
+                    prev[j] = (b < nb && row_live) ? a.out[static_cast<long long>(b0 + b) * a.out_ld + n] : 0.0f;
+                }
             }
             if (kRope) {
                 const bool rot = a.rope != nullptr && sec < 2 && row_live;
 #pragma unroll
-                for (int b = 0; b < BT; ++b)
-                    cs[b] = (rot && b < nb) ? a.rope[static_cast<long long>(s_pos[b]) * 32 + (col & 31)]
+                for (int j = 0; j < HB; ++j) {
+                    const int b = c0b + j;
+                    cs[j] = (rot && b < nb) ? a.rope[static_cast<long long>(s_pos[b]) * 32 + (col & 31)]
                                             : make_float2(1.0f, 0.0f);
+                }
             }
             if (EPI == EPI_I32) {
                 // the exact int32 sums themselves (kernel-level check of the integer products)
 #pragma unroll
-                for (int b = 0; b < BT; ++b)
-                    if (b < nb && row_live) a.out_i32[static_cast<long long>(b0 + b) * a.out_ld + n] = acc[b];
+                for (int j = 0; j < HB; ++j) {
+                    const int b = c0b + j;
+                    if (b < nb && row_live) a.out_i32[static_cast<long long>(b0 + b) * a.out_ld + n] = acc[0][j];
+                }
                 continue;
             }
 #pragma unroll
-            for (int b = 0; b < BT; ++b) {
-                float y = __fmul_rn(static_cast<float>(acc[b]), __fmul_rn(s_xs[b], sn));
+            for (int j = 0; j < HB; ++j) {
+                const int b = c0b + j;
+                float y;
+                if (XD == 1)
+                    y = __fmul_rn(static_cast<float>(acc[0][j]), __fmul_rn(s_xs[b], sn));
+                else
+                    y = digit_logit(acc[0][j], acc[NACC > 1 ? 1 : 0][j], acc[NACC > 2 ? 2 : 0][j], sn, s_xs[b]);
                 if (EPI != EPI_SWIGLU && a.bias != nullptr) y = __fadd_rn(y, bn);
                 const float yp = __shfl_xor_sync(0xffffffffu, y, 1);   // partner row of a pair
                 if (b >= nb || !row_live) continue;
                 const int gb = b0 + b;
                 if (EPI == EPI_RESID) {
-                    a.out[static_cast<long long>(gb) * a.out_ld + n] = __fadd_rn(prev[EPI == EPI_RESID ? b : 0], y);
+                    a.out[static_cast<long long>(gb) * a.out_ld + n] = __fadd_rn(prev[EPI == EPI_RESID ? j : 0], y);
                 } else if (EPI == EPI_SWIGLU) {
                     if ((p & 1) == 0) a.out[static_cast<long long>(gb) * a.out_ld + n] = __fmul_rn(silu_f(y), yp);
+                } else if (EPI == EPI_GELU) {
+                    a.out[static_cast<long long>(gb) * a.out_ld + n] = gelu_tanh_f(y);
                 } else if (EPI == EPI_QKV) {
                     float val = y;
                     if (kRope && a.rope != nullptr && sec < 2) {
-                        const float2 c = cs[kRope ? b : 0];
+                        const float2 c = cs[kRope ? j : 0];
                         // pair (i, i + 32): x_i' = x_i c - x_{i+32} s ; x_{i+32}' = x_i s + x_{i+32} c
                         if (col < 32)
                             val = __fsub_rn(__fmul_rn(y, c.x), __fmul_rn(yp, c.y));
@@ -313,20 +397,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tbase, TCOLS);
+        tmem_dealloc(tbase, tcols);
     }
 }
 
 // ---------------------------------------------------------------- launch planning
 
-// K split of one W8A8 projection on tcgen05; a function of the shape only. A CTA takes whole
-// 128-row blocks over all of K whenever the batch tile's activation slice fits: measured on B200
-// (per-phase timestamps inside the kernel at batch 16 and 64), exchanging split-K partials --
-// partial tiles to global memory, a fence, an arrival count, and the last arriver reading every
-// slice -- cost 5-10 us on the critical path, more than the parallelism it bought, since the
-// weights are already streamed in during the previous kernel. Longer K is split into the fewest
-// slices whose activation slice fits.
-inline MmaPlan tc_plan(int n_rows, int K, int num_sms) {
+// K split of one projection on tcgen05 with XD activation planes; a function of the shape
+// only. A CTA takes whole 128-row blocks over all of K whenever the batch tile's activation
+// slice fits: measured on B200 (per-phase timestamps inside the kernel at batch 16 and 64),
+// exchanging split-K partials -- partial tiles to global memory, a fence, an arrival count,
+// and the last arriver reading every slice -- cost 5-10 us on the critical path, more than
+// the parallelism it bought, since the weights are already streamed in during the previous
+// kernel. Longer K is split into the fewest slices whose activation slice fits.
+inline MmaPlan tc_plan(int n_rows, int K, int num_sms, int xd = 1) {
     (void)num_sms;
     MmaPlan p{};
     p.nbx = 1;
@@ -334,22 +418,25 @@ inline MmaPlan tc_plan(int n_rows, int K, int num_sms) {
     if (K % 32 != 0 || n_rows <= 0) return p;
     const int kchunks = (K + kTcKC - 1) / kTcKC;
     auto slice_len = [&](int nks) { return std::min(((kchunks + nks - 1) / nks) * kTcKC, K); };
+    auto xbytes = [&](int len) { return size_t(xd) * kTcMaxBT * ((len + kTcKC - 1) / kTcKC) * 128; };
     int n_ks = 1;
-    while (size_t(kTcMaxBT) * ((slice_len(n_ks) + kTcKC - 1) / kTcKC) * 128 > kTcXBudget && n_ks < kchunks) ++n_ks;
+    while (xbytes(slice_len(n_ks)) > kTcXBudget && n_ks < kchunks) ++n_ks;
     p.ksl = slice_len(n_ks);
     p.n_ks = (K + p.ksl - 1) / p.ksl;
-    p.ok = size_t(kTcMaxBT) * ((p.ksl + kTcKC - 1) / kTcKC) * 128 <= kTcXBudget;
+    p.ok = xbytes(p.ksl) <= kTcXBudget;
     return p;
 }
-inline size_t tc_part_bytes(const MmaPlan& p, int B) {
+inline size_t tc_part_bytes(const MmaPlan& p, int B, int xd = 1) {
     const int gy = (B + kTcMaxBT - 1) / kTcMaxBT;
-    return p.n_ks > 1 ? size_t(p.n_blocks) * gy * p.n_ks * 128 * kTcMaxBT * 4 : 0;
+    return p.n_ks > 1 ? size_t(p.n_blocks) * gy * p.n_ks * 128 * kTcMaxBT * 4 * (xd == 3 ? 3 : 1) : 0;
 }
-inline int tc_counters(const MmaPlan& p, int B) { return p.n_blocks * ((B + kTcMaxBT - 1) / kTcMaxBT) * 4; }
+inline int tc_counters(const MmaPlan& p, int B) { return p.n_blocks * ((B + kTcMaxBT - 1) / kTcMaxBT) * 4 * 2; }
 
-template <int EPI, int MAP>
+// One projection on tcgen05: wmap over the WD weight planes, xmap16 / xmap32 over the XD
+// activation planes (MB rows each) with boxes of 16 / 32 rows; xs the activation row scales.
+template <int EPI, int MAP, int XD, int WD>
 cudaError_t proj_tc_launch(int num_sms, const CUtensorMap& wmap, const CUtensorMap& xmap16, const CUtensorMap& xmap32,
-                           int n_rows, const float* xs, void* part, size_t part_bytes, int* cnt, int cnt_len,
+                           int n_rows, int MB, const float* xs, void* part, size_t part_bytes, int* cnt, int cnt_len,
                            const GemvArgs& g, cudaStream_t st);
 
 // dst [n_rows, K] from src (and src2 for MAP_DUAL) in the tensor-core row order.
@@ -358,6 +445,7 @@ cudaError_t tc_rows_permute(int map, int8_t* dst, const int8_t* src, const int8_
 
 #ifdef DEC_PROJ_TC_DEFINE
 
+#ifdef DEC_PROJ_TC_PERMUTE_DEFINE
 template <int MAP>
 __global__ void k_tc_rows_permute(int8_t* __restrict__ dst, const int8_t* __restrict__ src,
                                   const int8_t* __restrict__ src2, int n_rows, int K) {
@@ -384,14 +472,16 @@ cudaError_t tc_rows_permute(int map, int8_t* dst, const int8_t* src, const int8_
     }
     return cudaGetLastError();
 }
+#endif  // DEC_PROJ_TC_PERMUTE_DEFINE
 
-template <int BT, int EPI, int MAP>
+template <int BT, int EPI, int MAP, int XD, int WD>
 cudaError_t proj_tc_launch_bt(int num_sms, TcArgs A, int n_blocks, cudaStream_t st) {
-    auto kern = k_proj_tc<BT, EPI, MAP>;
+    auto kern = k_proj_tc<BT, EPI, MAP, XD, WD>;
+    constexpr int kStage = WD * kTcStageBytes;
     const int nch = (A.ksl + kTcKC - 1) / kTcKC;
-    const size_t xbytes = size_t(nch) * BT * 128;
+    const size_t xbytes = size_t(XD) * nch * BT * 128;
     const size_t avail = size_t(227 * 1024) - 1024 - 1024 - xbytes;
-    const int ns_max = int(std::min<size_t>(kTcMaxStages, avail / kTcStageBytes));
+    const int ns_max = int(std::min<size_t>(kTcMaxStages, avail / kStage));
     if (ns_max < 2) return cudaErrorNotSupported;
     thread_local int attr_dev = -1;   // attributes are per device; set again when it changes
     int dev = 0;
@@ -409,7 +499,7 @@ cudaError_t proj_tc_launch_bt(int num_sms, TcArgs A, int n_blocks, cudaStream_t 
     // one CTA per SM (TMEM and the ring); the ring holds no more stages than a CTA streams
     const int cps = std::max(1, std::min(n_blocks, std::max(1, num_sms / gy) / A.n_ks));
     const int NS = std::min(ns_max, std::max(2, ((n_blocks + cps - 1) / cps) * nch));
-    const size_t smem = 1024 + size_t(NS) * kTcStageBytes + xbytes;
+    const size_t smem = 1024 + size_t(NS) * kStage + xbytes;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cps * A.n_ks * gy);
     cfg.blockDim = dim3(kTcThreads);
@@ -423,14 +513,14 @@ cudaError_t proj_tc_launch_bt(int num_sms, TcArgs A, int n_blocks, cudaStream_t 
     return cudaLaunchKernelEx(&cfg, kern, A, NS);
 }
 
-template <int EPI, int MAP>
+template <int EPI, int MAP, int XD, int WD>
 cudaError_t proj_tc_launch(int num_sms, const CUtensorMap& wmap, const CUtensorMap& xmap16, const CUtensorMap& xmap32,
-                           int n_rows, const float* xs, void* part, size_t part_bytes, int* cnt, int cnt_len,
+                           int n_rows, int MB, const float* xs, void* part, size_t part_bytes, int* cnt, int cnt_len,
                            const GemvArgs& g, cudaStream_t st) {
-    if (g.B < 1) return cudaErrorNotSupported;
-    const MmaPlan p = tc_plan(n_rows, g.K, num_sms);
+    if (g.B < 1 || g.B > MB) return cudaErrorNotSupported;
+    const MmaPlan p = tc_plan(n_rows, g.K, num_sms, XD);
     if (!p.ok) return cudaErrorNotSupported;
-    if (p.n_ks > 1 && (tc_part_bytes(p, g.B) > part_bytes || tc_counters(p, g.B) > cnt_len))
+    if (p.n_ks > 1 && (tc_part_bytes(p, g.B, XD) > part_bytes || tc_counters(p, g.B) > cnt_len))
         return cudaErrorNotSupported;
     TcArgs A;
     A.wmap = wmap;
@@ -441,19 +531,20 @@ cudaError_t proj_tc_launch(int num_sms, const CUtensorMap& wmap, const CUtensorM
     A.ksl = p.ksl;
     A.n_rows = n_rows;
     A.n_by = 1;
+    A.MB = MB;
     A.g = g;
     if (g.B <= 16) {
         A.xmap = xmap16;
-        return proj_tc_launch_bt<16, EPI, MAP>(num_sms, A, p.n_blocks, st);
+        return proj_tc_launch_bt<16, EPI, MAP, XD, WD>(num_sms, A, p.n_blocks, st);
     }
     A.xmap = xmap32;
-    return proj_tc_launch_bt<32, EPI, MAP>(num_sms, A, p.n_blocks, st);
+    return proj_tc_launch_bt<32, EPI, MAP, XD, WD>(num_sms, A, p.n_blocks, st);
 }
 
-#define DEC_PROJ_TC_INSTANTIATE(EPI, MAP)                                                                         \
-    template cudaError_t proj_tc_launch<EPI, MAP>(int, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, \
-                                                  int, const float*, void*, size_t, int*, int, const GemvArgs&,   \
-                                                  cudaStream_t);
+#define DEC_PROJ_TC_INSTANTIATE(EPI, MAP, XD, WD)                                                                 \
+    template cudaError_t proj_tc_launch<EPI, MAP, XD, WD>(int, const CUtensorMap&, const CUtensorMap&,           \
+                                                          const CUtensorMap&, int, int, const float*, void*, size_t, \
+                                                          int*, int, const GemvArgs&, cudaStream_t);
 
 #endif  // DEC_PROJ_TC_DEFINE
 
