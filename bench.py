@@ -348,7 +348,7 @@ def dominant_kernel_roofline(wl, cfg, lens, tiles_per_split: int) -> dict:
     ms = e0.elapsed_time(e1) / reps
     alg = sum(n * 64 * 4 * 2 for n in n_keys) * H + 2 * B * H * 64 * 4
     achieved = alg / (ms / 1e3) / 1e9
-    traffic = recorded_traffic(wl.name)
+    traffic = recorded_traffic(wl.name, alg)
     max_tiles = (ld + 63) // 64
     grid = [-(-max_tiles // tiles_per_split), H, B]
     return {"kernel": name, "grid": grid, "tiles_per_split": tiles_per_split, "bound": "hbm",
@@ -358,9 +358,10 @@ def dominant_kernel_roofline(wl, cfg, lens, tiles_per_split: int) -> dict:
             "launch_us": round(ms * 1e3, 2)}
 
 
-def recorded_traffic(wl_name: str):
+def recorded_traffic(wl_name: str, algorithmic_bytes: int):
     """DRAM bytes per launch from the committed ncu summary, if the kernel source is
-    unchanged since the capture; otherwise null."""
+    unchanged since the capture; otherwise null. A record taken on a smaller case of the
+    same launch shape holds DRAM bytes per algorithmic byte, scaled here to this launch."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -371,7 +372,11 @@ def recorded_traffic(wl_name: str):
         return None
     src = os.path.join(ROOT, "transformer_decoder_kv_b200", "csrc", "attention.cuh")
     h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return rec.get("dram_bytes_per_launch") if rec.get("source_sha") == h else None
+    if rec.get("source_sha") != h:
+        return None
+    if "dram_per_algorithmic_byte" in rec:
+        return int(round(rec["dram_per_algorithmic_byte"] * algorithmic_bytes))
+    return rec.get("dram_bytes_per_launch")
 
 
 # ---------------------------------------------------------------- CPU oracle

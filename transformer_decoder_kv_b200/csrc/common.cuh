@@ -148,11 +148,16 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t phase,
 // drains the SM first, which stops a dependent kernel's CTAs from starting early under
 // programmatic dependent launch. Applied once per kernel and device (`attr_dev` is the
 // caller's per-kernel record of the device it was last applied on).
+// max_dyn_smem > 0 also raises the kernel's dynamic shared-memory limit to that many bytes.
 template <typename K>
-inline cudaError_t prefer_max_shared_once(K kern, int& attr_dev) {
+inline cudaError_t prefer_max_shared_once(K kern, int& attr_dev, int max_dyn_smem = 0) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || attr_dev == dev) return e;
+    if (max_dyn_smem > 0) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn_smem);
+        if (e != cudaSuccess) return e;
+    }
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e == cudaSuccess) attr_dev = dev;
     return e;

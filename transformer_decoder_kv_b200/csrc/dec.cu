@@ -68,11 +68,6 @@ struct LayerDev {
     // 2-D TMA descriptors of the projections (tensor-core path); Qwen uses m_qkv (the
     // permuted panel), m_o, m_1 (gate/up) and m_2 (down)
     CUtensorMap m_qkv, m_o, m_xq, m_xo, m_1, m_2;
-    // Whisper with f32 weights, tcgen05 path: each projection's three int8 digit planes
-    // [3][N][K] with row scales, and their TMA descriptors (same order as the maps above)
-    int8_t* dig[6] = {};
-    float* dsc[6] = {};
-    CUtensorMap m_dig[6];
 };
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -438,24 +433,15 @@ bool tcd_eligible(const dec_handle* h, int N, int K, int B) {
 // with exact int32 sums; y = s_n s_b (A0 + (A1 + A2 / 254) / 254) + bias.
 template <int PRO, int EPI>
 dec_status proj_digits_tc(dec_handle* h, const GemvArgs& a, const LayerDev* L, int m, cudaStream_t st) {
-    const bool f32w = h->cfg.proj_fmt == DEC_PROJ_F32;
     cudaError_t e = rowprep_digits_launch<PRO>(a.x, a.x_ld, a.norm_w, a.norm_b, a.eps, a.K, a.B,
-                                               static_cast<long long>(h->w->xd_rows) * a.K, h->w->xd3, h->w->xsd, nullptr,
-                                               true, st);
+                                               static_cast<long long>(h->w->xd_rows) * a.K, h->w->xd3, h->w->xsd,
+                                               nullptr, true, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "row digit split launch");
     const int kx = a.K == h->cfg.d_model ? 0 : 1;
-    GemvArgs g = a;
-    if (f32w) {
-        g.scale = L->dsc[m];
-        e = proj_tc_launch<EPI, MAP_ADJ, 3, 3>(h->num_sms, L->m_dig[m], h->w->m_xd3[kx][0], h->w->m_xd3[kx][1], a.N,
-                                               h->w->xd_rows, h->w->xsd, h->w->mma_part, h->w->mma_part_bytes, h->w->mma_cnt,
-                                               h->w->mma_cnt_len, g, st);
-    } else {
-        const CUtensorMap* maps[6] = {&L->m_qkv, &L->m_o, &L->m_xq, &L->m_xo, &L->m_1, &L->m_2};
-        e = proj_tc_launch<EPI, MAP_ADJ, 3, 1>(h->num_sms, *maps[m], h->w->m_xd3[kx][0], h->w->m_xd3[kx][1], a.N,
-                                               h->w->xd_rows, h->w->xsd, h->w->mma_part, h->w->mma_part_bytes, h->w->mma_cnt,
-                                               h->w->mma_cnt_len, g, st);
-    }
+    const CUtensorMap* maps[6] = {&L->m_qkv, &L->m_o, &L->m_xq, &L->m_xo, &L->m_1, &L->m_2};
+    e = proj_tc_launch<EPI, MAP_ADJ, 3, 1>(h->num_sms, *maps[m], h->w->m_xd3[kx][0], h->w->m_xd3[kx][1], a.N,
+                                           h->w->xd_rows, h->w->xsd, h->w->mma_part, h->w->mma_part_bytes,
+                                           h->w->mma_cnt, h->w->mma_cnt_len, a, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "tcgen05 digit projection launch");
     return DEC_OK;
 }
@@ -468,10 +454,10 @@ dec_status gemv_whisper(dec_handle* h, const GemvArgs& a, cudaStream_t st, const
     const bool f32w = h->cfg.proj_fmt == DEC_PROJ_F32;
     const LayerDev* L = &layer;
     if (h->tma_ok) {
-        // f32 weights take the tensor cores only for the larger matrices (below, the CUDA-core
-        // kernel's whole run is shorter than the extra row-split launch); W8A32 always
-        if ((!f32w || mma_worth(a.N, a.K, false)) && tcd_eligible(h, a.N, a.K, a.B))
-            return proj_digits_tc<PRO, EPI>(h, a, L, m, st);
+        // W8A32 on the digit path; f32 weights stay on TF32 / CUDA cores (a three-plane digit
+        // path for them measured slower at the C2 shapes: its row split is a launch of its
+        // own and fc2's activation planes need a split-K exchange)
+        if (!f32w && tcd_eligible(h, a.N, a.K, a.B)) return proj_digits_tc<PRO, EPI>(h, a, L, m, st);
         const CUtensorMap* maps[6] = {&L->m_qkv, &L->m_o, &L->m_xq, &L->m_xo, &L->m_1, &L->m_2};
         if (f32w && mma_worth(a.N, a.K, false) && mma_eligible(h, a.N, a.K, 4, a.B))
             return proj_mma<float, PRO, EPI>(h, a, *maps[m], st);
@@ -1017,6 +1003,39 @@ dec_status validate_step(dec_handle* h, int B, const int32_t* slots, const int32
     return DEC_OK;
 }
 
+// Two-chain steps: every kernel but the attention gets the device's highest launch priority,
+// so that when an SM frees up, the chain in its latency-bound projection phase gets it
+// before the other chain's next attention CTA (the attention streams HBM with whatever SMs
+// it holds). Best effort: a failure leaves the default priorities.
+void prioritise_latency_kernels(cudaGraph_t g) {
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) {
+        cudaGetLastError();
+        return;
+    }
+    size_t n = 0;
+    if (cudaGraphGetNodes(g, nullptr, &n) != cudaSuccess || n == 0) {
+        cudaGetLastError();
+        return;
+    }
+    std::vector<cudaGraphNode_t> nodes(n);
+    if (cudaGraphGetNodes(g, nodes.data(), &n) != cudaSuccess) {
+        cudaGetLastError();
+        return;
+    }
+    for (auto nd : nodes) {
+        cudaGraphNodeType t;
+        cudaKernelNodeParams kp;
+        if (cudaGraphNodeGetType(nd, &t) != cudaSuccess || t != cudaGraphNodeTypeKernel ||
+            cudaGraphKernelNodeGetParams(nd, &kp) != cudaSuccess)
+            continue;
+        cudaKernelNodeAttrValue v{};
+        v.priority = kp.func == reinterpret_cast<void*>(k_attention) ? least : greatest;
+        cudaGraphKernelNodeSetAttribute(nd, cudaLaunchAttributePriority, &v);
+    }
+    cudaGetLastError();
+}
+
 // Record the step's launch sequence into a graph for later identical steps. Capture
 // problems are not errors: the key is marked and such steps keep running eagerly.
 void capture_step(dec_handle* h, const std::array<long long, 5>& key, int B, int max_len, float* logits,
@@ -1034,6 +1053,7 @@ void capture_step(dec_handle* h, const std::array<long long, 5>& key, int B, int
         cudaGraph_t g = nullptr;
         const cudaError_t e = cudaStreamEndCapture(h->cap_stream, &g);
         if (s == DEC_OK && e == cudaSuccess && g != nullptr) {
+            if (split) prioritise_latency_kernels(g);
             if (cudaGraphInstantiate(&exec, g, 0) != cudaSuccess) exec = nullptr;
             size_t n = 0;
             if (exec && cudaGraphGetNodes(g, nullptr, &n) == cudaSuccess) {
@@ -1254,30 +1274,8 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
     h->max_rows = std::max(h->max_batch, kPrefillChunk);
     const int MB = h->max_rows;
     DEC_TRY(dalloc(h, &h->x, size_t(MB) * d * 4));
-    // Whisper f32 weights, tcgen05 path: each matrix's three digit planes, made once like the
-    // head's embedding planes
-    bool digit_maps_ok = h->tma_ok && wh;
-    if (digit_maps_ok && c.proj_fmt == DEC_PROJ_F32) {
-        dec_status ts = DEC_OK;
-        for (int l = 0; l < L && ts == DEC_OK; ++l) {
-            LayerDev& D = h->layers[l];
-            const void* ws[6] = {D.wqkv, D.wo, D.wxq, D.wxo, D.w1, D.w2};
-            const int ns[6] = {d + 2 * kv_width(c), d, d, d, F, d};
-            const int kk[6] = {d, d, d, d, d, F};
-            for (int m = 0; m < 6 && ts == DEC_OK; ++m) {
-                const long long nk = static_cast<long long>(ns[m]) * kk[m];
-                DEC_TRY(dalloc(h, &D.dig[m], size_t(3) * nk));
-                DEC_TRY(dalloc(h, &D.dsc[m], size_t(ns[m]) * 4));
-                DEC_CUDA(h, rowprep_digits_launch<PRO_NONE>(static_cast<const float*>(ws[m]), kk[m], nullptr, nullptr,
-                                                           0.0f, kk[m], ns[m], nk, D.dig[m], D.dsc[m], nullptr, false,
-                                                           0));
-                ts = make_wmap(h, &D.m_dig[m], D.dig[m], 3 * ns[m], kk[m], false);
-            }
-        }
-        DEC_CUDA(h, cudaDeviceSynchronize());
-        digit_maps_ok = (ts == DEC_OK);
-        if (!digit_maps_ok) h->err.clear();
-    }
+    // Whisper W8A32, tcgen05 path: the activation digit planes (per chain, below)
+    bool digit_maps_ok = h->tma_ok && wh && c.proj_fmt == DEC_PROJ_W8A32;
     // split-K scratch of the largest tensor-core plan
     size_t pb = 16;
     int cl = 1;
@@ -1308,7 +1306,7 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
                 need_i8(sh[0] == F ? 2 * F : sh[0], sh[1]);
             } else {
                 need_f32(sh[0], sh[1], welt);
-                need_digits(sh[0], sh[1]);
+                if (welt == 1) need_digits(sh[0], sh[1]);
             }
         }
     }

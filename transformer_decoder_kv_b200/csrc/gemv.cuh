@@ -197,9 +197,15 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
     float* sXraw = RAW_STAGE ? reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(sX) +
                                                          static_cast<size_t>(BT) * a.K * sizeof(XT))
                              : reinterpret_cast<float*>(sX);
+    // the norm's weight (and LayerNorm bias) rows, copied in before the dependency wait
+    constexpr bool NORM_W = PRO == PRO_RMS || PRO == PRO_LN;
+    float* sNw = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(sX) +
+                                          static_cast<size_t>(BT) * a.K * sizeof(XT) +
+                                          (RAW_STAGE ? static_cast<size_t>(BT) * a.K * 4 : 0));
+    float* sNb = sNw + a.K;
     __shared__ __align__(8) uint64_t full[kGemvMaxStages];
     __shared__ __align__(8) uint64_t empty[kGemvMaxStages];
-    __shared__ __align__(8) uint64_t bar_x;
+    __shared__ __align__(8) uint64_t bar_x, bar_g;
     __shared__ float s_mu[BT], s_rstd[BT], s_inv[BT], s_a[BT];
     __shared__ unsigned long long s_key[BT];
     __shared__ int s_flag;
@@ -288,7 +294,14 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
             mbar_init(&empty[i], NWC);
         }
         mbar_init(&bar_x, 1);
+        mbar_init(&bar_g, 1);
         mbar_fence_init();
+        if (NORM_W) {
+            const uint32_t nbytes = static_cast<uint32_t>(a.K) * 4;
+            mbar_arrive_expect_tx(&bar_g, PRO == PRO_LN ? 2 * nbytes : nbytes);
+            bulk_g2s(sNw, a.norm_w, nbytes, &bar_g);
+            if (PRO == PRO_LN) bulk_g2s(sNb, a.norm_b, nbytes, &bar_g);
+        }
         for (; n_issued < NS && n_issued < n_items; ++n_issued) issue(n_issued);
     }
     pdl_launch_dependents();
@@ -307,16 +320,19 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
                 bulk_g2s(sXraw + static_cast<size_t>(b) * a.K, a.x + static_cast<long long>(b0 + b) * a.x_ld,
                          row_bytes, &bar_x);
         }
-        s_flag = mbar_wait_bounded(&bar_x, 0, a.err) ? 1 : 0;
+        s_flag = (mbar_wait_bounded(&bar_x, 0, a.err) && (!NORM_W || mbar_wait_bounded(&bar_g, 0, a.err))) ? 1 : 0;
     }
     __syncthreads();
     if (!s_flag) {
-        if (producer && lane == 0)
+        if (producer && lane == 0) {
             for (int i2 = 0; i2 < n_issued; ++i2) mbar_wait_bounded(&full[i2], 0, nullptr);
+            if (NORM_W) mbar_wait_bounded(&bar_g, 0, nullptr);
+        }
         __syncthreads();
         return;
     }
     (void)mbar_try_wait(&bar_x, 0);
+    if (NORM_W) (void)mbar_try_wait(&bar_g, 0);
 
     // ---- per-row statistics from shared memory ----
     if (PRO != PRO_RAW_I8 && !producer) {
@@ -324,8 +340,8 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
             float mu = 0.0f, rstd = 1.0f, inv = 0.0f, ascale = 0.0f;
             if (b < nb) {
                 const float4* xr = reinterpret_cast<const float4*>(sXraw + static_cast<size_t>(b) * a.K);
-                const float4* g4 = reinterpret_cast<const float4*>(a.norm_w);
-                const float4* be4 = reinterpret_cast<const float4*>(a.norm_b);
+                const float4* g4 = reinterpret_cast<const float4*>(sNw);
+                const float4* be4 = reinterpret_cast<const float4*>(sNb);
                 const int K4 = a.K >> 2;
                 if (PRO == PRO_LN) {
                     float sum = 0.0f;
@@ -362,8 +378,8 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
                     for (int k = lane; k < K4; k += 32) {
                         const float4 v = xr[k];
                         float4 g = make_float4(1.f, 1.f, 1.f, 1.f), be = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (PRO != PRO_NONE) g = __ldg(g4 + k);
-                        if (PRO == PRO_LN) be = __ldg(be4 + k);
+                        if (PRO != PRO_NONE) g = g4[k];
+                        if (PRO == PRO_LN) be = be4[k];
                         amax = fmaxf(amax, fabsf(norm_value(PRO, v.x, mu, rstd, g.x, be.x)));
                         amax = fmaxf(amax, fabsf(norm_value(PRO, v.y, mu, rstd, g.y, be.y)));
                         amax = fmaxf(amax, fabsf(norm_value(PRO, v.z, mu, rstd, g.z, be.z)));
@@ -395,8 +411,8 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
             if (b < nb) {
                 const float4 v = reinterpret_cast<const float4*>(sXraw)[e];
                 float4 g = make_float4(1.f, 1.f, 1.f, 1.f), be = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (PRO != PRO_NONE) g = __ldg(reinterpret_cast<const float4*>(a.norm_w) + k4);
-                if (PRO == PRO_LN) be = __ldg(reinterpret_cast<const float4*>(a.norm_b) + k4);
+                if (PRO != PRO_NONE) g = reinterpret_cast<const float4*>(sNw)[k4];
+                if (PRO == PRO_LN) be = reinterpret_cast<const float4*>(sNb)[k4];
                 y.x = norm_value(PRO, v.x, s_mu[b], s_rstd[b], g.x, be.x);
                 y.y = norm_value(PRO, v.y, s_mu[b], s_rstd[b], g.y, be.y);
                 y.z = norm_value(PRO, v.z, s_mu[b], s_rstd[b], g.z, be.z);

@@ -25,11 +25,14 @@ struct GemvPlan {
     size_t smem;
 };
 
-// Activation bytes in shared memory: the tile, plus the raw f32 rows for the int8 path.
+// Activation bytes in shared memory: the tile, plus the raw f32 rows for the int8 path,
+// plus the norm's weight (and LayerNorm bias) rows.
 template <bool I8, int PRO>
 size_t gemv_xbytes(int BT, int K) {
     size_t x = size_t(BT) * K * (I8 ? 1 : 4);
     if (I8 && PRO != PRO_RAW_I8) x += size_t(BT) * K * 4;
+    if (PRO == PRO_RMS || PRO == PRO_LN) x += size_t(K) * 4;
+    if (PRO == PRO_LN) x += size_t(K) * 4;
     return x;
 }
 

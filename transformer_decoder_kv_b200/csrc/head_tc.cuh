@@ -146,9 +146,9 @@ __device__ __forceinline__ float row_digits_passes(Get get, int jmax, const floa
         float4 v = get(j);
         if (PRO != PRO_NONE) {
             const int k = lane + 32 * j;
-            const float4 g = __ldg(reinterpret_cast<const float4*>(gw) + k);
+            const float4 g = reinterpret_cast<const float4*>(gw)[k];
             float4 be = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (PRO == PRO_LN) be = __ldg(reinterpret_cast<const float4*>(gb) + k);
+            if (PRO == PRO_LN) be = reinterpret_cast<const float4*>(gb)[k];
             v = make_float4(norm_value(PRO, v.x, mu, rstd, g.x, be.x), norm_value(PRO, v.y, mu, rstd, g.y, be.y),
                             norm_value(PRO, v.z, mu, rstd, g.z, be.z), norm_value(PRO, v.w, mu, rstd, g.w, be.w));
         }
@@ -241,8 +241,20 @@ __global__ void __launch_bounds__(128) k_rowprep_digits(const float* __restrict_
                                                         float eps, int K, int rows, long long plane_stride,
                                                         int8_t* __restrict__ out, float* __restrict__ scale,
                                                         int* __restrict__ sums) {
+    // the norm's weight (and LayerNorm bias) rows do not depend on the previous kernel: they
+    // are copied into shared memory before the dependency wait
+    extern __shared__ float4 rd_norm[];
+    const int K4 = K >> 2;
+    if (PRO != PRO_NONE)
+        for (int i = threadIdx.x; i < K4; i += blockDim.x) {
+            rd_norm[i] = reinterpret_cast<const float4*>(gw)[i];
+            if (PRO == PRO_LN) rd_norm[K4 + i] = reinterpret_cast<const float4*>(gb)[i];
+        }
     pdl_launch_dependents();
     pdl_wait();
+    __syncthreads();
+    const float* gws = reinterpret_cast<const float*>(rd_norm);
+    const float* gbs = reinterpret_cast<const float*>(rd_norm + K4);
     const int lane = threadIdx.x & 31;
     const int r = blockIdx.x * 4 + (threadIdx.x >> 5);
     if (r >= rows) return;
@@ -257,17 +269,17 @@ __global__ void __launch_bounds__(128) k_rowprep_digits(const float* __restrict_
     };
     const float* xrow = x + static_cast<long long>(r) * x_ld;
     float sc;
-    if ((K >> 2) <= 32 * kDigitsRegK4) {
+    if (K4 <= 32 * kDigitsRegK4) {
         // the row read once into registers (every loop of the passes fully unrolled over the
         // compile-time bound); same elements, same order as the memory path
         const float4* xr = reinterpret_cast<const float4*>(xrow);
         float4 rv[kDigitsRegK4];
 #pragma unroll
         for (int j = 0; j < kDigitsRegK4; ++j)
-            rv[j] = lane + 32 * j < (K >> 2) ? xr[lane + 32 * j] : make_float4(0.f, 0.f, 0.f, 0.f);
-        sc = row_digits_passes<PRO>([&](int j) { return rv[j]; }, kDigitsRegK4, gw, gb, eps, K, lane, sink, s12);
+            rv[j] = lane + 32 * j < K4 ? xr[lane + 32 * j] : make_float4(0.f, 0.f, 0.f, 0.f);
+        sc = row_digits_passes<PRO>([&](int j) { return rv[j]; }, kDigitsRegK4, gws, gbs, eps, K, lane, sink, s12);
     } else {
-        sc = row_digits_warp<PRO>(xrow, gw, gb, eps, K, lane, sink, s12);
+        sc = row_digits_warp<PRO>(xrow, gws, gbs, eps, K, lane, sink, s12);
     }
     if (lane == 0) {
         scale[r] = sc;
@@ -772,12 +784,15 @@ cudaError_t rowprep_digits_launch(const float* x, int x_ld, const float* gw, con
                                   int rows, long long plane_stride, int8_t* out, float* scale, int* sums, bool pdl,
                                   cudaStream_t st) {
     if (K % 4 != 0 || rows <= 0) return cudaErrorInvalidValue;
+    const size_t smem = size_t(K) * 4 * (PRO == PRO_LN ? 2 : (PRO == PRO_RMS ? 1 : 0));
+    if (smem > size_t(227 * 1024)) return cudaErrorInvalidValue;
     thread_local int attr_dev = -1;
-    const cudaError_t e = prefer_max_shared_once(k_rowprep_digits<PRO>, attr_dev);
+    const cudaError_t e = prefer_max_shared_once(k_rowprep_digits<PRO>, attr_dev, 227 * 1024);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((rows + 3) / 4);
     cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -1,4 +1,4 @@
-// W8A8 projections on the 5th-generation tensor cores for batches of 8 or more:
+// W8A8 and Whisper W8A32 projections on the 5th-generation tensor cores for batches of 8 or more:
 // tcgen05.mma .kind::i8 (M = 128 weight rows, N = 16 or 32 batch columns, K = 32 per
 // instruction) with exact int32 accumulation in TMEM.
 //
@@ -80,6 +80,8 @@ template <int XD, int WD>
 struct TcDigits {
     static_assert((XD == 1 && WD == 1) || (XD == 3 && (WD == 1 || WD == 3)), "digit planes");
 };
+// (WD = 3, f32 weights split like the head's embedding, is supported by the kernel but not
+// instantiated: it measured slower than the TF32 kernel at the shapes that use f32 weights.)
 
 // TMEM columns of one CTA: `sets` accumulator sets (two when the CTA owns more than one row
 // block, so that the epilogue of one overlaps the MMAs of the next) of XD BT columns; at most

@@ -1,5 +1,5 @@
-// Whisper projections (W8A32 and f32 weights) on tcgen05 int8 tensor cores: activation rows
-// as three int8 digit planes, weights as one (int8) or three (f32) digit planes.
+// Whisper W8A32 projections on tcgen05 int8 tensor cores: the activation rows as three int8
+// digit planes, stacked along N, times the int8 weights.
 #define DEC_PROJ_TC_DEFINE
 #include <algorithm>
 
@@ -10,8 +10,4 @@ DEC_PROJ_TC_INSTANTIATE(EPI_QKV, MAP_ADJ, 3, 1)
 DEC_PROJ_TC_INSTANTIATE(EPI_RESID, MAP_ADJ, 3, 1)
 DEC_PROJ_TC_INSTANTIATE(EPI_STORE, MAP_ADJ, 3, 1)
 DEC_PROJ_TC_INSTANTIATE(EPI_GELU, MAP_ADJ, 3, 1)
-DEC_PROJ_TC_INSTANTIATE(EPI_QKV, MAP_ADJ, 3, 3)
-DEC_PROJ_TC_INSTANTIATE(EPI_RESID, MAP_ADJ, 3, 3)
-DEC_PROJ_TC_INSTANTIATE(EPI_STORE, MAP_ADJ, 3, 3)
-DEC_PROJ_TC_INSTANTIATE(EPI_GELU, MAP_ADJ, 3, 3)
 }  // namespace dec

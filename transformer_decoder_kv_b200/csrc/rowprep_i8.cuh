@@ -59,8 +59,8 @@ __device__ __forceinline__ float rowprep_i8_passes(Get get, int K4, int K, int l
         const int k = lane + 32 * j;
         const float4 v = get(j);
         float4 g = make_float4(1.f, 1.f, 1.f, 1.f), be = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (PRO != PRO_NONE) g = __ldg(g4 + k);
-        if (PRO == PRO_LN) be = __ldg(be4 + k);
+        if (PRO != PRO_NONE) g = g4[k];
+        if (PRO == PRO_LN) be = be4[k];
         return make_float4(norm_value(PRO, v.x, mu, rstd, g.x, be.x), norm_value(PRO, v.y, mu, rstd, g.y, be.y),
                            norm_value(PRO, v.z, mu, rstd, g.z, be.z), norm_value(PRO, v.w, mu, rstd, g.w, be.w));
     };
@@ -91,15 +91,24 @@ __global__ void __launch_bounds__(128) k_rowprep_i8(const float* __restrict__ x,
                                                     const float* __restrict__ gw, const float* __restrict__ gb,
                                                     float eps, int K, int B, int8_t* __restrict__ xq,
                                                     float* __restrict__ xs) {
+    // the norm's weight (and LayerNorm bias) rows do not depend on the previous kernel: they
+    // are copied into shared memory before the dependency wait
+    extern __shared__ float4 rp_norm[];
+    const int K4 = K >> 2;
+    if (PRO != PRO_NONE)
+        for (int i = threadIdx.x; i < K4; i += blockDim.x) {
+            rp_norm[i] = reinterpret_cast<const float4*>(gw)[i];
+            if (PRO == PRO_LN) rp_norm[K4 + i] = reinterpret_cast<const float4*>(gb)[i];
+        }
     pdl_launch_dependents();
     pdl_wait();
+    __syncthreads();
     const int lane = threadIdx.x & 31;
     const int b = blockIdx.x * 4 + (threadIdx.x >> 5);
     if (b >= B) return;
     const float4* xr = reinterpret_cast<const float4*>(x + static_cast<long long>(b) * x_ld);
-    const float4* g4 = reinterpret_cast<const float4*>(gw);
-    const float4* be4 = reinterpret_cast<const float4*>(gb);
-    const int K4 = K >> 2;
+    const float4* g4 = rp_norm;
+    const float4* be4 = rp_norm + K4;
     uint32_t* q = reinterpret_cast<uint32_t*>(xq + static_cast<long long>(b) * K);
     float amax;
     if (K4 <= 32 * kRowprepRegK4) {
@@ -123,14 +132,14 @@ cudaError_t rowprep_i8_launch(const GemvArgs& g, int8_t* xq, float* xs, cudaStre
 
 template <int PRO>
 cudaError_t rowprep_i8_launch(const GemvArgs& g, int8_t* xq, float* xs, cudaStream_t st) {
-    if (g.K % 16 != 0) return cudaErrorNotSupported;
+    if (g.K % 16 != 0 || size_t(g.K) * 8 > size_t(227 * 1024)) return cudaErrorNotSupported;
     thread_local int attr_dev = -1;
-    const cudaError_t e = prefer_max_shared_once(k_rowprep_i8<PRO>, attr_dev);
+    const cudaError_t e = prefer_max_shared_once(k_rowprep_i8<PRO>, attr_dev, 227 * 1024);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((g.B + 3) / 4);
     cfg.blockDim = dim3(128);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = size_t(g.K) * 4 * (PRO == PRO_LN ? 2 : (PRO == PRO_RMS ? 1 : 0));
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
