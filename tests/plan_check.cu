@@ -61,11 +61,9 @@ int main() {
                 CHECK(p.ksl % kTcKC == 0 || p.ksl == s.K, "digit slice not whole stages N=%d K=%d", s.N, s.K);
                 const int nch = (p.ksl + kTcKC - 1) / kTcKC;
                 CHECK(size_t(3) * kTcMaxBT * nch * 128 <= kTcXBudget, "digit X budget N=%d K=%d", s.N, s.K);
-                for (int wd : {1}) {   // W8A32: one weight plane (the three-plane f32 form is not launched)
+                for (int wd : {1, 3}) {
                     // ring: at least two stages of wd weight planes next to the activation slice
-                    // (and, when the kernel splits the rows itself, the LayerNorm weight and bias)
-                    const size_t own = s.K <= kTcOwnPlanesMaxK ? size_t(8) * s.K : 0;
-                    const size_t avail = size_t(227 * 1024) - 2048 - size_t(3) * nch * kTcMaxBT * 128 - own;
+                    const size_t avail = size_t(227 * 1024) - 2048 - size_t(3) * nch * kTcMaxBT * 128;
                     CHECK(avail / (size_t(wd) * kTcStageBytes) >= 2, "digit ring N=%d K=%d wd=%d", s.N, s.K, wd);
                 }
                 for (int B = 1; B <= DEC_MAX_BATCH; ++B) {

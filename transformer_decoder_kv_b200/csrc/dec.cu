@@ -427,26 +427,18 @@ bool tcd_eligible(const dec_handle* h, int N, int K, int B) {
     return p.n_ks == 1 || (tc_part_bytes(p, B, 3) <= h->w->mma_part_bytes && tc_counters(p, B) <= h->w->mma_cnt_len);
 }
 
-// Whisper W8A32 projections on tcgen05 int8 tensor cores: the (normalised) activation rows
-// split into three int8 digit planes -- by the projection kernel itself for rows of up to
-// kTcOwnPlanesMaxK columns, else by k_rowprep_digits first -- times the int8 weights, with
-// exact int32 sums; y = s_n s_b (A0 + (A1 + A2 / 254) / 254) + bias.
+// Whisper projections on tcgen05 int8 tensor cores: the (normalised) activation rows split
+// into three int8 digit planes by k_rowprep_digits, times the int8 weights (W8A32, one
+// plane, three products per K step) or the f32 weights' three digit planes (six products),
+// with exact int32 sums; y = s_n s_b (A0 + (A1 + A2 / 254) / 254) + bias.
 template <int PRO, int EPI>
 dec_status proj_digits_tc(dec_handle* h, const GemvArgs& a, const LayerDev* L, int m, cudaStream_t st) {
+    cudaError_t e = rowprep_digits_launch<PRO>(a.x, a.x_ld, a.norm_w, a.norm_b, a.eps, a.K, a.B,
+                                               static_cast<long long>(h->w->xd_rows) * a.K, h->w->xd3, h->w->xsd,
+                                               nullptr, true, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "row digit split launch");
     const int kx = a.K == h->cfg.d_model ? 0 : 1;
     const CUtensorMap* maps[6] = {&L->m_qkv, &L->m_o, &L->m_xq, &L->m_xo, &L->m_1, &L->m_2};
-    cudaError_t e;
-    if (a.K <= kTcOwnPlanesMaxK) {
-        e = proj_tc_launch<EPI, MAP_ADJ, 3, 1, PRO>(h->num_sms, *maps[m], h->w->m_xd3[kx][0], h->w->m_xd3[kx][1],
-                                                    a.N, h->w->xd_rows, h->w->xsd, h->w->mma_part,
-                                                    h->w->mma_part_bytes, h->w->mma_cnt, h->w->mma_cnt_len, a, st);
-        if (e != cudaSuccess) return cuda_fail(h, e, "tcgen05 digit projection launch");
-        return DEC_OK;
-    }
-    e = rowprep_digits_launch<PRO>(a.x, a.x_ld, a.norm_w, a.norm_b, a.eps, a.K, a.B,
-                                   static_cast<long long>(h->w->xd_rows) * a.K, h->w->xd3, h->w->xsd, nullptr, true,
-                                   st);
-    if (e != cudaSuccess) return cuda_fail(h, e, "row digit split launch");
     e = proj_tc_launch<EPI, MAP_ADJ, 3, 1>(h->num_sms, *maps[m], h->w->m_xd3[kx][0], h->w->m_xd3[kx][1], a.N,
                                            h->w->xd_rows, h->w->xsd, h->w->mma_part, h->w->mma_part_bytes,
                                            h->w->mma_cnt, h->w->mma_cnt_len, a, st);

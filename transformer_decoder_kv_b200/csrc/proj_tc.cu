@@ -7,8 +7,8 @@
 #include "proj_tc.cuh"
 
 namespace dec {
-DEC_PROJ_TC_INSTANTIATE(EPI_QKV, MAP_ROPE, 1, 1, kTcXExternal)
-DEC_PROJ_TC_INSTANTIATE(EPI_RESID, MAP_ADJ, 1, 1, kTcXExternal)
-DEC_PROJ_TC_INSTANTIATE(EPI_SWIGLU, MAP_DUAL, 1, 1, kTcXExternal)
-DEC_PROJ_TC_INSTANTIATE(EPI_I32, MAP_ADJ, 1, 1, kTcXExternal)
+DEC_PROJ_TC_INSTANTIATE(EPI_QKV, MAP_ROPE, 1, 1)
+DEC_PROJ_TC_INSTANTIATE(EPI_RESID, MAP_ADJ, 1, 1)
+DEC_PROJ_TC_INSTANTIATE(EPI_SWIGLU, MAP_DUAL, 1, 1)
+DEC_PROJ_TC_INSTANTIATE(EPI_I32, MAP_ADJ, 1, 1)
 }  // namespace dec

@@ -44,8 +44,6 @@ constexpr int kTcStageBytes = 128 * kTcKC;      // 16 KB
 constexpr int kTcMaxStages = 12;
 constexpr int kTcMaxBT = 32;
 constexpr size_t kTcXBudget = 120 * 1024;       // activation slice bytes at most (all planes)
-constexpr int kTcXExternal = -1;                // activation planes made by a row-prep kernel
-constexpr int kTcOwnPlanesMaxK = 32 * 4 * kDigitsRegK4;   // rows the kernel splits itself, in registers
 
 struct TcArgs {
     CUtensorMap wmap;      // int8 weight planes [WD * n_rows, K]: box {128 bytes, 128 rows}
@@ -95,17 +93,11 @@ __host__ __device__ inline uint32_t tc_tmem_cols(int xd, int bt, int sets) {
     return t;
 }
 
-// XPRO: kTcXExternal when a row-prep kernel made the activation planes (loaded by TMA), or
-// the norm (PRO_NONE, PRO_LN) with which the CTA makes its batch tile's digit planes itself
-// (XD = 3, K <= kTcOwnPlanesMaxK): one warp per row, with k_rowprep_digits' arithmetic (the
-// same function), the norm's weight rows copied into shared memory before the dependency wait.
-template <int BT, int EPI, int MAP, int XD, int WD, int XPRO>
+template <int BT, int EPI, int MAP, int XD, int WD>
 __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant__ TcArgs A, int NS) {
     static_assert(BT == 16 || BT == 32, "batch tile");
     static_assert(XD == 1 || (MAP == MAP_ADJ && EPI != EPI_I32 && EPI != EPI_SWIGLU), "digit planes: plain rows");
     (void)sizeof(TcDigits<XD, WD>);
-    static_assert(XPRO == kTcXExternal || XD == 3, "in-kernel activation planes: digit path only");
-    constexpr bool OWN = XPRO != kTcXExternal;
     constexpr int NACC = XD;                              // accumulators A0 .. A(XD-1)
     constexpr int kStage = WD * kTcStageBytes;
     constexpr int XC = XD * BT * 128;                     // bytes of one chunk's stacked planes
@@ -120,7 +112,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
     unsigned char* ring = smem;
     unsigned char* sx = smem + static_cast<size_t>(NS) * kStage;
     __shared__ __align__(8) uint64_t full[kTcMaxStages], empty[kTcMaxStages];
-    __shared__ __align__(8) uint64_t tfull[2], tempty[2], bar_x, bar_done, bar_g;
+    __shared__ __align__(8) uint64_t tfull[2], tempty[2], bar_x, bar_done;
     __shared__ uint32_t s_tmem;
     __shared__ float s_xs[BT];
     __shared__ int s_pos[BT], s_slot[BT], s_len[BT];   // EPI_QKV: position, cache page, row in the page
@@ -154,7 +146,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
             mbar_init(&tempty[i], kTcEpiWarps);
         }
         mbar_init(&bar_x, 1);
-        mbar_init(&bar_g, 1);
         mbar_init(&bar_done, 1);
         mbar_fence_init();
         s_fail = 0;
@@ -179,24 +170,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
             tma_load_2d(dst + p * kTcStageBytes, &A.wmap, kstart + c * kTcKC, p * A.n_rows + jb * 128,
                         &full[it % NS]);
     };
-    // OWN: the norm's weight (and LayerNorm bias) rows, after the activation slice
-    constexpr bool NORM_W = OWN && (XPRO == PRO_LN || XPRO == PRO_RMS);
-    float* sNw = reinterpret_cast<float*>(sx + static_cast<size_t>(XD * nch) * BT * 128);
-    float* sNb = sNw + a.K;
     int n_issued = 0;
-    if (warp == 0 && lane == 0) {
-        if (NORM_W) {
-            const uint32_t nbytes = static_cast<uint32_t>(a.K) * 4;
-            mbar_arrive_expect_tx(&bar_g, XPRO == PRO_LN ? 2 * nbytes : nbytes);
-            bulk_g2s(sNw, a.norm_w, nbytes, &bar_g);
-            if (XPRO == PRO_LN) bulk_g2s(sNb, a.norm_b, nbytes, &bar_g);
-        }
+    if (warp == 0 && lane == 0)
         for (; n_issued < NS && n_issued < n_items; ++n_issued) issue(n_issued);
-    }
     pdl_launch_dependents();
     pdl_wait();
     if (tid < BT) {
-        s_xs[tid] = (!OWN && tid < nb) ? A.xs[b0 + tid] : 0.0f;
+        s_xs[tid] = tid < nb ? A.xs[b0 + tid] : 0.0f;
         if (EPI == EPI_QKV) {
             // position, and the cache page and row within it of this step's new row
             int page = 0, r = 0;
@@ -206,49 +186,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
             s_len[tid] = r;
         }
     }
-    if (OWN) {
-        // the batch tile's digit planes of this K slice, in the swizzled K-major layout the
-        // MMA reads: zero first (rows past the batch, columns past the slice), then one warp per
-        // row splits the whole row (its norm and scale need every column) and keeps the slice
-        for (int o = tid * 16; o < XD * nch * BT * 128; o += kTcThreads * 16)
-            *reinterpret_cast<uint4*>(sx + o) = make_uint4(0u, 0u, 0u, 0u);
-        if (NORM_W && tid == 0 && !mbar_wait_bounded(&bar_g, 0, a.err)) s_fail = 1;
-        __syncthreads();
-        if (NORM_W) (void)mbar_try_wait(&bar_g, 0);
-        constexpr int kPro = XPRO < 0 ? PRO_NONE : XPRO;
-        const int K4 = a.K >> 2;
-        for (int b = warp; b < nb; b += kTcThreads / 32) {
-            const float4* xr = reinterpret_cast<const float4*>(a.x + static_cast<long long>(b0 + b) * a.x_ld);
-            auto sink = [&](int k4, uint32_t p1, uint32_t p2, uint32_t p3) {
-                const int k = 4 * k4 - kstart;
-                if (k < 0 || k >= klen) return;
-                const int j = k & 127;   // byte within the 128-byte row of chunk k / 128
-                const int off = (k >> 7) * XC + b * 128 + (((j >> 4) ^ (b & 7)) << 4) + (j & 15);
-                *reinterpret_cast<uint32_t*>(sx + off) = p1;
-                *reinterpret_cast<uint32_t*>(sx + BT * 128 + off) = p2;
-                *reinterpret_cast<uint32_t*>(sx + 2 * BT * 128 + off) = p3;
-            };
-            float4 rv[kDigitsRegK4];
-#pragma unroll
-            for (int j = 0; j < kDigitsRegK4; ++j)
-                rv[j] = lane + 32 * j < K4 ? xr[lane + 32 * j] : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float sc = row_digits_passes<kPro>([&](int j) { return rv[j]; }, kDigitsRegK4, sNw, sNb, a.eps,
-                                                     a.K, lane, sink, nullptr);
-            if (lane == 0) s_xs[b] = sc;
-        }
-        // generic-proxy shared-memory writes become visible to the tensor core
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    }
     __syncthreads();
 
     if (warp == 0 && lane == 0) {
         // the activation slice of this batch tile: XD planes, one box per 128 columns
-        if (!OWN) {
-            mbar_arrive_expect_tx(&bar_x, static_cast<uint32_t>(XD * nch) * BT * 128);
-            for (int p = 0; p < XD; ++p)
-                for (int c = 0; c < nch; ++c)
-                    tma_load_2d(sx + c * XC + p * BT * 128, &A.xmap, kstart + c * kTcKC, p * A.MB + b0, &bar_x);
-        }
+        mbar_arrive_expect_tx(&bar_x, static_cast<uint32_t>(XD * nch) * BT * 128);
+        for (int p = 0; p < XD; ++p)
+            for (int c = 0; c < nch; ++c)
+                tma_load_2d(sx + c * XC + p * BT * 128, &A.xmap, kstart + c * kTcKC, p * A.MB + b0, &bar_x);
         for (int it = n_issued; it < n_items; ++it) {
             if (!mbar_wait_bounded(&empty[it % NS], static_cast<uint32_t>(it / NS - 1) & 1u, a.err)) {
                 s_fail = 1;
@@ -259,7 +204,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
         }
     } else if (warp == 1 && lane == 0) {
         // ---- MMA issuer ----
-        bool ok = OWN || mbar_wait_bounded(&bar_x, 0, a.err);
+        bool ok = mbar_wait_bounded(&bar_x, 0, a.err);
         tc_fence_after();
         int it = 0;
         for (int i = 0; ok && i < my_blocks; ++i) {
@@ -447,11 +392,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const __grid_constant
             }
         }
     }
-    if (warp == 0 && lane == 0 && s_fail) {
+    if (warp == 0 && lane == 0 && s_fail)
         for (int i2 = max(0, n_issued - NS); i2 < n_issued; ++i2)
             mbar_wait_bounded(&full[i2 % NS], static_cast<uint32_t>(i2 / NS) & 1u, nullptr);
-        if (NORM_W) mbar_wait_bounded(&bar_g, 0, nullptr);
-    }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -493,7 +436,7 @@ inline int tc_counters(const MmaPlan& p, int B) { return p.n_blocks * ((B + kTcM
 
 // One projection on tcgen05: wmap over the WD weight planes, xmap16 / xmap32 over the XD
 // activation planes (MB rows each) with boxes of 16 / 32 rows; xs the activation row scales.
-template <int EPI, int MAP, int XD, int WD, int XPRO = kTcXExternal>
+template <int EPI, int MAP, int XD, int WD>
 cudaError_t proj_tc_launch(int num_sms, const CUtensorMap& wmap, const CUtensorMap& xmap16, const CUtensorMap& xmap32,
                            int n_rows, int MB, const float* xs, void* part, size_t part_bytes, int* cnt, int cnt_len,
                            const GemvArgs& g, cudaStream_t st);
@@ -533,14 +476,12 @@ cudaError_t tc_rows_permute(int map, int8_t* dst, const int8_t* src, const int8_
 }
 #endif  // DEC_PROJ_TC_PERMUTE_DEFINE
 
-template <int BT, int EPI, int MAP, int XD, int WD, int XPRO>
+template <int BT, int EPI, int MAP, int XD, int WD>
 cudaError_t proj_tc_launch_bt(int num_sms, TcArgs A, int n_blocks, cudaStream_t st) {
-    auto kern = k_proj_tc<BT, EPI, MAP, XD, WD, XPRO>;
+    auto kern = k_proj_tc<BT, EPI, MAP, XD, WD>;
     constexpr int kStage = WD * kTcStageBytes;
     const int nch = (A.ksl + kTcKC - 1) / kTcKC;
-    // the activation slice, and with in-kernel planes the norm's weight (and bias) rows
-    const size_t xbytes = size_t(XD) * nch * BT * 128 +
-                          (XPRO == PRO_LN ? 8 : (XPRO == PRO_RMS ? 4 : 0)) * size_t(A.g.K);
+    const size_t xbytes = size_t(XD) * nch * BT * 128;
     const size_t avail = size_t(227 * 1024) - 1024 - 1024 - xbytes;
     const int ns_max = int(std::min<size_t>(kTcMaxStages, avail / kStage));
     if (ns_max < 2) return cudaErrorNotSupported;
@@ -574,12 +515,11 @@ cudaError_t proj_tc_launch_bt(int num_sms, TcArgs A, int n_blocks, cudaStream_t 
     return cudaLaunchKernelEx(&cfg, kern, A, NS);
 }
 
-template <int EPI, int MAP, int XD, int WD, int XPRO>
+template <int EPI, int MAP, int XD, int WD>
 cudaError_t proj_tc_launch(int num_sms, const CUtensorMap& wmap, const CUtensorMap& xmap16, const CUtensorMap& xmap32,
                            int n_rows, int MB, const float* xs, void* part, size_t part_bytes, int* cnt, int cnt_len,
                            const GemvArgs& g, cudaStream_t st) {
     if (g.B < 1 || g.B > MB) return cudaErrorNotSupported;
-    if (XPRO != kTcXExternal && (g.K > kTcOwnPlanesMaxK || g.K % 4 != 0)) return cudaErrorNotSupported;
     const MmaPlan p = tc_plan(n_rows, g.K, num_sms, XD);
     if (!p.ok) return cudaErrorNotSupported;
     if (p.n_ks > 1 && (tc_part_bytes(p, g.B, XD) > part_bytes || tc_counters(p, g.B) > cnt_len))
@@ -597,16 +537,16 @@ cudaError_t proj_tc_launch(int num_sms, const CUtensorMap& wmap, const CUtensorM
     A.g = g;
     if (g.B <= 16) {
         A.xmap = xmap16;
-        return proj_tc_launch_bt<16, EPI, MAP, XD, WD, XPRO>(num_sms, A, p.n_blocks, st);
+        return proj_tc_launch_bt<16, EPI, MAP, XD, WD>(num_sms, A, p.n_blocks, st);
     }
     A.xmap = xmap32;
-    return proj_tc_launch_bt<32, EPI, MAP, XD, WD, XPRO>(num_sms, A, p.n_blocks, st);
+    return proj_tc_launch_bt<32, EPI, MAP, XD, WD>(num_sms, A, p.n_blocks, st);
 }
 
-#define DEC_PROJ_TC_INSTANTIATE(EPI, MAP, XD, WD, XPRO)                                                           \
-    template cudaError_t proj_tc_launch<EPI, MAP, XD, WD, XPRO>(int, const CUtensorMap&, const CUtensorMap&,     \
-                                                                const CUtensorMap&, int, int, const float*, void*, \
-                                                                size_t, int*, int, const GemvArgs&, cudaStream_t);
+#define DEC_PROJ_TC_INSTANTIATE(EPI, MAP, XD, WD)                                                                 \
+    template cudaError_t proj_tc_launch<EPI, MAP, XD, WD>(int, const CUtensorMap&, const CUtensorMap&,           \
+                                                          const CUtensorMap&, int, int, const float*, void*, size_t, \
+                                                          int*, int, const GemvArgs&, cudaStream_t);
 
 #endif  // DEC_PROJ_TC_DEFINE
 
