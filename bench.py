@@ -40,7 +40,18 @@ CONFIGS = {
     "c5": "c5_whisper_large_v3_w8a32_b32",
 }
 L2_BYTES = 126 * 1024 * 1024
-SPLIT_MIN_BATCH = 32   # decode steps of this many rows run as two chains (the library's rule)
+SPLIT_MIN_BATCH = 32   # decode steps of this many rows run as several chains (the library's rule)
+MAX_CHAINS = 2
+
+
+def chain_rows(B: int):
+    """Chain count and rows of the first chain of a split step (the library's chain_bounds)."""
+    n = min(MAX_CHAINS, B // 8)
+    base = ((-(-B // n) + 7) // 8) * 8
+    n = -(-B // base)
+    if B - base * (n - 1) < 8:
+        n -= 1
+    return n, base
 
 
 def measured_peaks():
@@ -316,11 +327,13 @@ def dominant_kernel_roofline(wl, cfg, lens, tiles_per_split: int) -> dict:
 
     peak, peak_kind = measured_peaks()
     B, H = wl.batch, cfg.n_heads
-    # a step of 32 rows or more runs as two chains, each launching the attention over its
-    # own rows: time the first chain's launch (the library's split rule)
+    # a step of 32 rows or more runs as chains over parts of the rows, each launching the
+    # attention over its own rows: time the first chain's launch (the library's split rule)
     split = B >= SPLIT_MIN_BATCH
+    n_chains = 1
     if split:
-        B = min(B - 8, ((B // 2 + 15) // 16) * 16)
+        n_chains, first = chain_rows(B)
+        B = first
         lens = list(lens)[:B]
     if cfg.is_whisper:
         name, n_keys, ld = "k_attention (cross-attention, 1500 keys)", [cfg.enc_len] * B, cfg.enc_len
@@ -359,7 +372,7 @@ def dominant_kernel_roofline(wl, cfg, lens, tiles_per_split: int) -> dict:
     max_tiles = (ld + 63) // 64
     grid = [-(-max_tiles // tiles_per_split), H, B]
     if split:
-        name += f", one of the step's two chains ({B} of {wl.batch} streams)"
+        name += f", one of the step's {n_chains} chains ({B} of {wl.batch} streams)"
     return {"kernel": name, "grid": grid, "tiles_per_split": tiles_per_split, "bound": "hbm",
             "achieved": round(achieved, 1), "peak": peak,
             "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)", "unit": "GB/s",

@@ -36,6 +36,10 @@ constexpr int kMetaRing = 8;
 // Prompt tokens of one slot that dec_prefill runs together as one step's rows.
 constexpr int kPrefillChunk = DEC_MAX_BATCH;
 constexpr int kMaxSplits = kAttnMaxSplits;
+// Most chains a decode step runs as (see run_step). Measured on B200: two free-running
+// chains C4 5.67 -> 5.40 and C5 7.21 -> 5.96 ms/step against two chains whose attentions
+// alternated; four chains C4 5.41, C5 6.19.
+constexpr int kMaxChains = 2;
 
 thread_local std::string g_create_error;
 // Allocation-failure injection for tests (dec_debug_fail_alloc): the n-th allocation of the
@@ -76,10 +80,10 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 }  // namespace
 
-// Per-chain step scratch. A decode step of many rows runs as two chains, each over half of
-// the rows, on two streams: while one chain streams its attention K/V from HBM, the other
-// runs its latency-bound projections. Each chain has its own copies of everything a
-// launch writes besides its rows of x, so the two never share scratch.
+// Per-chain step scratch. A decode step of many rows runs as up to kMaxChains chains over
+// equal parts of the rows, on their own streams, so that the chains' latency-bound kernels
+// overlap one another and the attention of one. Each chain has its own copies of everything
+// a launch writes besides its rows of x, so chains never share scratch.
 struct Chain {
     float *q = nullptr, *ctx = nullptr, *ffn = nullptr, *xq = nullptr;
     float* part = nullptr;          // attention split partials
@@ -137,11 +141,12 @@ struct dec_handle {
     // workspace: the residual rows x are shared by both chains (each owns a row range); the
     // rest of the per-step scratch is per chain (see Chain)
     float* x = nullptr;
-    Chain chain[2];
+    Chain chain[kMaxChains];
     Chain* w = &chain[0];           // the chain whose launches are being issued
-    int n_chains = 1;               // 2: decode steps of kSplitMinBatch rows or more run as two chains
+    int n_chains = 1;               // chains allocated: up to kMaxChains when batches can be split
     cudaStream_t side = nullptr;    // the second chain's stream (eager steps)
-    cudaEvent_t ev_fork = nullptr, ev_join = nullptr, ev_attn[2] = {nullptr, nullptr};
+    cudaStream_t side_streams[kMaxChains] = {};   // chain c > 0 runs on side_streams[c] (eager steps)
+    cudaEvent_t ev_fork = nullptr, ev_join[kMaxChains] = {};
     bool tcd_ok = false;            // Whisper digit-path descriptors and planes built
     unsigned long long* keys = nullptr;
     int* head_counter = nullptr;
@@ -365,7 +370,18 @@ constexpr int kMmaMinBatch = 8;
 // Decode steps of this many rows or more run as two chains (run_step); each chain's half is
 // a multiple of 16 rows, so each stays on the tensor-core paths.
 constexpr int kSplitMinBatch = 32;
-inline int split_rows(int B) { return std::min(B - kMmaMinBatch, ((B / 2 + 15) / 16) * 16); }
+// Rows of each chain of a split step: equal multiples of 8 (every chain stays on the tensor-
+// core paths, which start at 8 rows), the last one taking the rest; r0[c] .. r0[c + 1] - 1 are
+// chain c's rows. Returns the chain count.
+inline int chain_bounds(int B, int* r0) {
+    int n = std::min(kMaxChains, B / kMmaMinBatch);
+    int base = (((B + n - 1) / n + kMmaMinBatch - 1) / kMmaMinBatch) * kMmaMinBatch;
+    n = (B + base - 1) / base;
+    if (B - base * (n - 1) < kMmaMinBatch) --n;   // a short last chain joins the one before
+    for (int c = 0; c < n; ++c) r0[c] = c * base;
+    r0[n] = B;
+    return n;
+}
 constexpr long long kMmaMinWeights = 1LL << 21;
 
 bool mma_worth(int N, int K, bool w8a32) {
@@ -612,10 +628,7 @@ dec_status phase_mark(dec_handle* h, cudaStream_t st, int layer, int kind) {
 }
 
 // One decoder layer for the rows of the current chain (h->w): X holds their residual rows.
-// wait_ev / done_ev order the layer's largest attention (self for Qwen2, cross for Whisper)
-// against the other chain's: it starts after wait_ev and records done_ev.
-dec_status layer_step(dec_handle* h, int l, int B, float* X, int max_len_plus1, cudaStream_t st,
-                      cudaEvent_t wait_ev, cudaEvent_t done_ev) {
+dec_status layer_step(dec_handle* h, int l, int B, float* X, int max_len_plus1, cudaStream_t st) {
     const dec_config& c = h->cfg;
     const int d = c.d_model, F = c.d_ff, H = c.n_heads;
     (void)H;
@@ -667,9 +680,7 @@ dec_status layer_step(dec_handle* h, int l, int B, float* X, int max_len_plus1, 
     at.counters = h->w->counters;
     at.err = h->dev_err;
     at.drop_first_copy = (l == 0) ? h->inject_drop : 0;
-    if (!wh && wait_ev) DEC_CUDA(h, cudaStreamWaitEvent(st, wait_ev, 0));
     DEC_TRY(attention(h, at, B, max_len_plus1, h->tps_self, st));
-    if (!wh && done_ev) DEC_CUDA(h, cudaEventRecord(done_ev, st));
     DEC_TRY(phase_mark(h, st, l, DEC_PHASE_SELF_ATTN));
     at.drop_first_copy = 0;
     // ---- output projection + residual ----
@@ -714,9 +725,7 @@ dec_status layer_step(dec_handle* h, int l, int B, float* X, int max_len_plus1, 
         at.kv_group = 1;
         at.kv.table = nullptr;
         at.n_fixed = c.enc_len;
-        if (wait_ev) DEC_CUDA(h, cudaStreamWaitEvent(st, wait_ev, 0));
         DEC_TRY(attention(h, at, B, c.enc_len, h->tps_cross, st));
-        if (done_ev) DEC_CUDA(h, cudaEventRecord(done_ev, st));
         DEC_TRY(phase_mark(h, st, l, DEC_PHASE_CROSS_ATTN));
         g = base_args(h, B);
         g.x = h->w->ctx;
@@ -791,8 +800,9 @@ dec_status layer_step(dec_handle* h, int l, int B, float* X, int max_len_plus1, 
 // One step for the batch described in h->dmeta (already uploaded).
 // head_row0 / head_rows: the rows whose logits the head computes (all by default; a prompt
 // chunk needs its last row only, or none). trace: copy each layer's residual (decode steps).
-// split: run the layers as two chains over the two halves of the rows (the metas of both
-// halves uploaded too), on st and h->side, alternating their large attentions.
+// split: run the layers as chains over equal parts of the rows (chain_bounds; the metas of the
+// parts uploaded too), chain 0 on st and chain c on h->side_streams[c], with no dependency
+// between chains: their kernels overlap wherever the SMs allow.
 dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int* argmax, cudaStream_t st,
                     int head_row0 = 0, int head_rows = -1, bool trace = true, bool split = false) {
     if (head_rows < 0) head_rows = B;
@@ -811,31 +821,31 @@ dec_status run_step(dec_handle* h, int B, int max_len_plus1, float* logits, int*
     DEC_TRY(phase_mark(h, st, -1, DEC_PHASE_EMBED));
     if (!split) {
         for (int l = 0; l < c.n_layers; ++l) {
-            DEC_TRY(layer_step(h, l, B, h->x, max_len_plus1, st, nullptr, nullptr));
+            DEC_TRY(layer_step(h, l, B, h->x, max_len_plus1, st));
             if (trace && h->trace)
                 DEC_CUDA(h, cudaMemcpyAsync(h->trace + static_cast<size_t>(l) * B * d, h->x, size_t(B) * d * 4,
                                             cudaMemcpyDeviceToDevice, st));
         }
     } else {
-        const int n0 = split_rows(B);
+        int r0[kMaxChains + 1];
+        const int n = chain_bounds(B, r0);
         DEC_CUDA(h, cudaEventRecord(h->ev_fork, st));
-        DEC_CUDA(h, cudaStreamWaitEvent(h->side, h->ev_fork, 0));
-        h->chain[0].meta = h->dmeta + 1;
-        h->chain[1].meta = h->dmeta + 2;
+        for (int ci = 1; ci < n; ++ci) DEC_CUDA(h, cudaStreamWaitEvent(h->side_streams[ci], h->ev_fork, 0));
+        for (int ci = 0; ci < n; ++ci) h->chain[ci].meta = h->dmeta + 1 + ci;
         dec_status r = DEC_OK;
-        for (int l = 0; l < c.n_layers && r == DEC_OK; ++l) {
-            h->w = &h->chain[0];
-            r = layer_step(h, l, n0, h->x, max_len_plus1, st, l > 0 ? h->ev_attn[1] : nullptr, h->ev_attn[0]);
-            if (r != DEC_OK) break;
-            h->w = &h->chain[1];
-            r = layer_step(h, l, B - n0, h->x + static_cast<size_t>(n0) * d, max_len_plus1, h->side, h->ev_attn[0],
-                           h->ev_attn[1]);
-        }
-        // the second chain always joins, so that a capture ends with every stream joined
+        for (int l = 0; l < c.n_layers && r == DEC_OK; ++l)
+            for (int ci = 0; ci < n && r == DEC_OK; ++ci) {
+                h->w = &h->chain[ci];
+                r = layer_step(h, l, r0[ci + 1] - r0[ci], h->x + static_cast<size_t>(r0[ci]) * d, max_len_plus1,
+                               ci == 0 ? st : h->side_streams[ci]);
+            }
+        // every chain always joins, so that a capture ends with every stream joined
         h->w = &h->chain[0];
         h->chain[0].meta = h->dmeta;
-        DEC_CUDA(h, cudaEventRecord(h->ev_join, h->side));
-        DEC_CUDA(h, cudaStreamWaitEvent(st, h->ev_join, 0));
+        for (int ci = 1; ci < n; ++ci) {
+            DEC_CUDA(h, cudaEventRecord(h->ev_join[ci], h->side_streams[ci]));
+            DEC_CUDA(h, cudaStreamWaitEvent(st, h->ev_join[ci], 0));
+        }
         DEC_TRY(r);
     }
     // ---- final norm + tied head + greedy argmax ----
@@ -913,18 +923,20 @@ void shrink_slot(dec_handle* h, int slot, int rows) {
 }
 
 // Upload the step description through the pinned ring.
-// With split, the rows of the two chains follow as metas of their own (rows renumbered from
-// 0; page-table updates stay with the whole step's meta, which k_embed applies).
+// With split, the rows of each chain follow as metas of their own (rows renumbered from 0;
+// page-table updates stay with the whole step's meta, which k_embed applies).
 dec_status upload_meta(dec_handle* h, const StepMeta& m, cudaStream_t st, bool split = false) {
     const int i = h->ring;
     h->ring = (h->ring + 1) % kMetaRing;
     DEC_CUDA(h, cudaEventSynchronize(h->hev[i]));
     std::memcpy(h->hmeta[i], &m, sizeof(StepMeta));
+    int n_parts = 0;
     if (split) {
-        const int n0 = split_rows(m.B);
-        for (int ci = 0; ci < 2; ++ci) {
+        int rb[kMaxChains + 1];
+        n_parts = chain_bounds(m.B, rb);
+        for (int ci = 0; ci < n_parts; ++ci) {
             StepMeta& o = h->hmeta[i][1 + ci];
-            const int r0 = ci == 0 ? 0 : n0, n = ci == 0 ? n0 : m.B - n0;
+            const int r0 = rb[ci], n = rb[ci + 1] - rb[ci];
             o.B = n;
             o.n_upd = 0;
             for (int b = 0; b < n; ++b) {
@@ -936,7 +948,7 @@ dec_status upload_meta(dec_handle* h, const StepMeta& m, cudaStream_t st, bool s
             }
         }
     }
-    DEC_CUDA(h, cudaMemcpyAsync(h->dmeta, h->hmeta[i], (split ? 3 : 1) * sizeof(StepMeta), cudaMemcpyHostToDevice,
+    DEC_CUDA(h, cudaMemcpyAsync(h->dmeta, h->hmeta[i], (1 + n_parts) * sizeof(StepMeta), cudaMemcpyHostToDevice,
                                 st));
     DEC_CUDA(h, cudaEventRecord(h->hev[i], st));
     return DEC_OK;
@@ -1081,7 +1093,7 @@ dec_status step_validated(dec_handle* h, StepMeta& m, int max_len, float* logits
     // two chains for large batches, unless per-layer copies, phase timing or fault injection
     // need the single launch sequence
     const bool split =
-        h->n_chains == 2 && m.B >= kSplitMinBatch && !h->trace && !h->phase_timing && !h->inject_drop;
+        h->n_chains > 1 && m.B >= kSplitMinBatch && !h->trace && !h->phase_timing && !h->inject_drop;
     DEC_TRY(upload_meta(h, m, st, split));
     const std::array<long long, 5> key = {m.B, (max_len + kAttnTile - 1) / kAttnTile,
                                           reinterpret_cast<long long>(logits), reinterpret_cast<long long>(argmax),
@@ -1122,9 +1134,11 @@ dec_status dec_destroy(dec_handle* h) {
         if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
     for (cudaEvent_t e : h->phase_ev) cudaEventDestroy(e);
     if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
-    if (h->side) cudaStreamDestroy(h->side);
-    for (cudaEvent_t e : {h->ev_fork, h->ev_join, h->ev_attn[0], h->ev_attn[1]})
-        if (e) cudaEventDestroy(e);
+    for (int ci = 1; ci < kMaxChains; ++ci) {
+        if (h->side_streams[ci]) cudaStreamDestroy(h->side_streams[ci]);
+        if (h->ev_join[ci]) cudaEventDestroy(h->ev_join[ci]);
+    }
+    if (h->ev_fork) cudaEventDestroy(h->ev_fork);
     for (void* p : h->dallocs) cudaFree(p);
     for (void* p : h->hallocs) cudaFreeHost(p);
     for (int i = 0; i < kMetaRing; ++i)
@@ -1311,7 +1325,10 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
         }
     }
     // per-chain scratch: chain 0 always, chain 1 when decode batches can be split in two
-    h->n_chains = h->max_batch >= kSplitMinBatch ? 2 : 1;
+    {
+        int rb[kMaxChains + 1];
+        h->n_chains = h->max_batch >= kSplitMinBatch ? chain_bounds(h->max_batch, rb) : 1;
+    }
     for (int ci = 0; ci < h->n_chains; ++ci) {
         Chain& ch = h->chain[ci];
         DEC_TRY(dalloc(h, &ch.q, size_t(MB) * d * 4));
@@ -1365,14 +1382,14 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
     DEC_CUDA(h, cudaMemset(h->last_tok, 0, size_t(c.max_slots) * 4));
     DEC_TRY(dalloc(h, &h->dev_err, kStatusWords * 4));
     DEC_CUDA(h, cudaMemset(h->dev_err, 0, kStatusWords * 4));
-    DEC_TRY(dalloc(h, &h->dmeta, 3 * sizeof(StepMeta)));
+    DEC_TRY(dalloc(h, &h->dmeta, (1 + kMaxChains) * sizeof(StepMeta)));
     h->chain[0].meta = h->dmeta;
-    h->chain[1].meta = h->dmeta + 2;
-    if (h->n_chains == 2) {
-        DEC_CUDA(h, cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking));
+    if (h->n_chains > 1) {
         DEC_CUDA(h, cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming));
-        DEC_CUDA(h, cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming));
-        for (int i = 0; i < 2; ++i) DEC_CUDA(h, cudaEventCreateWithFlags(&h->ev_attn[i], cudaEventDisableTiming));
+        for (int ci = 1; ci < h->n_chains; ++ci) {
+            DEC_CUDA(h, cudaStreamCreateWithFlags(&h->side_streams[ci], cudaStreamNonBlocking));
+            DEC_CUDA(h, cudaEventCreateWithFlags(&h->ev_join[ci], cudaEventDisableTiming));
+        }
     }
     DEC_TRY(dalloc(h, &h->stage_logits, size_t(h->max_batch) * c.vocab * 4));
     DEC_TRY(dalloc(h, &h->stage_argmax, size_t(h->max_batch) * 4));
@@ -1387,7 +1404,7 @@ static dec_status create_impl(dec_handle* h, const dec_config* cfg, const dec_we
     };
     for (int i = 0; i < kMetaRing; ++i) {
         void* p = nullptr;
-        DEC_TRY(halloc(&p, 3 * sizeof(StepMeta)));
+        DEC_TRY(halloc(&p, (1 + kMaxChains) * sizeof(StepMeta)));
         h->hmeta[i] = static_cast<StepMeta*>(p);
         DEC_CUDA(h, cudaEventCreateWithFlags(&h->hev[i], cudaEventDisableTiming));
     }
