@@ -40,7 +40,7 @@ CONFIGS = {
     "c5": "c5_whisper_large_v3_w8a32_b32",
 }
 L2_BYTES = 126 * 1024 * 1024
-SPLIT_MIN_BATCH = 32   # decode steps of this many rows run as several chains (the library's rule)
+SPLIT_MIN_BATCH = 16   # decode steps of this many rows run as several chains (the library's rule)
 MAX_CHAINS = 2
 
 
@@ -327,7 +327,7 @@ def dominant_kernel_roofline(wl, cfg, lens, tiles_per_split: int) -> dict:
 
     peak, peak_kind = measured_peaks()
     B, H = wl.batch, cfg.n_heads
-    # a step of 32 rows or more runs as chains over parts of the rows, each launching the
+    # a step of 16 rows or more runs as chains over parts of the rows, each launching the
     # attention over its own rows: time the first chain's launch (the library's split rule)
     split = B >= SPLIT_MIN_BATCH
     n_chains = 1

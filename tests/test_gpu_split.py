@@ -1,4 +1,4 @@
-"""Decode steps of 32 rows or more run as chains (two) over equal parts of the rows, on their
+"""Decode steps of 16 rows or more run as chains (two) over equal parts of the rows, on their
 own streams, with no dependency between them (run_step's split). Every output of a row
 depends only on that row's own inputs on every path the chains use (exact integer sums for
 W8A8, the digit-plane Whisper projections and the head; attention split boundaries fixed per

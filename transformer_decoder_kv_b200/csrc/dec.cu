@@ -367,9 +367,9 @@ dec_status gemv(dec_handle* h, const GemvArgs& a, cudaStream_t st) {
 // CUDA-core kernel's whole run, except for int8 weights with f32 activations, whose
 // CUDA-core kernel is arithmetic-bound from batch 8 on.
 constexpr int kMmaMinBatch = 8;
-// Decode steps of this many rows or more run as two chains (run_step); each chain's half is
-// a multiple of 16 rows, so each stays on the tensor-core paths.
-constexpr int kSplitMinBatch = 32;
+// Decode steps of this many rows or more run as chains (run_step, chain_bounds); each chain
+// has at least 8 rows, so each stays on the tensor-core paths.
+constexpr int kSplitMinBatch = 16;
 // Rows of each chain of a split step: equal multiples of 8 (every chain stays on the tensor-
 // core paths, which start at 8 rows), the last one taking the rest; r0[c] .. r0[c + 1] - 1 are
 // chain c's rows. Returns the chain count.
@@ -631,8 +631,6 @@ dec_status phase_mark(dec_handle* h, cudaStream_t st, int layer, int kind) {
 dec_status layer_step(dec_handle* h, int l, int B, float* X, int max_len_plus1, cudaStream_t st) {
     const dec_config& c = h->cfg;
     const int d = c.d_model, F = c.d_ff, H = c.n_heads;
-    (void)H;
-    const bool wh = c.family == DEC_FAMILY_WHISPER;
     const LayerDev& L = h->layers[l];
     float* kc = h->kc + l * h->self_layer_stride;
     float* vc = h->vc + l * h->self_layer_stride;
