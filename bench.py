@@ -46,11 +46,8 @@ MAX_CHAINS = 2
 
 def chain_rows(B: int):
     """Chain count and rows of the first chain of a split step (the library's chain_bounds)."""
-    n = min(MAX_CHAINS, B // 8)
-    base = ((-(-B // n) + 7) // 8) * 8
-    n = -(-B // base)
-    if B - base * (n - 1) < 8:
-        n -= 1
+    n = max(1, min(MAX_CHAINS, B // 8))
+    base = max(1, (B // n) // 8 * 8)
     return n, base
 
 

@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "dec.h"
+#include "chain_plan.h"
 #include "head_tc.cuh"
 #include "proj_mma.cuh"
 #include "proj_tc.cuh"
@@ -30,6 +31,20 @@ struct Shape {
 
 int main() {
     const int sms = 148;
+    // chains of a split step: cover the batch exactly, at least kMmaMinBatch rows each,
+    // at most kMaxChains, in ascending order
+    for (int B = 1; B <= DEC_MAX_BATCH; ++B) {
+        int r0[kMaxChains + 1];
+        const int n = chain_bounds(B, r0);
+        CHECK(n >= 1 && n <= kMaxChains, "chain count B=%d n=%d", B, n);
+        CHECK(r0[0] == 0 && r0[n] == B, "chains cover B=%d", B);
+        for (int c = 0; c < n; ++c) {
+            CHECK(r0[c + 1] > r0[c], "chain order B=%d", B);
+            if (B >= kSplitMinBatch) CHECK(r0[c + 1] - r0[c] >= kMmaMinBatch, "chain rows B=%d c=%d", B, c);
+        }
+        if (B >= kSplitMinBatch) CHECK(n == kMaxChains, "split B=%d n=%d", B, n);
+        std::printf("chain %d %d %d\n", B, n, r0[1]);
+    }
     // (d, F, V, family W8A8?, f32?)
     struct Model {
         int d, F, V;

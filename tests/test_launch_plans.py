@@ -31,3 +31,11 @@ def test_launch_plans_cover_k_fit_budgets_and_scratch():
         assert r.returncode == 0, r.stderr[-3000:]
         r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
         assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-3000:]
+    # the benchmark times the attention in the first chain's launch shape: its copy of the
+    # chain rule must agree with the library's
+    import bench
+    chains = [tuple(int(v) for v in ln.split()[1:]) for ln in r.stdout.splitlines() if ln.startswith("chain ")]
+    assert len(chains) > 100
+    for B, n, first in chains:
+        if B >= bench.SPLIT_MIN_BATCH:
+            assert bench.chain_rows(B) == (n, first), (B, n, first, bench.chain_rows(B))

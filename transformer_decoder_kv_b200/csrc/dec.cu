@@ -19,6 +19,7 @@
 #include "../../include/dec.h"
 #include "attention.cuh"
 #include "attn_plan.h"
+#include "chain_plan.h"
 #include "common.cuh"
 #include "gemv.cuh"
 #include "gemv_launch.cuh"
@@ -36,10 +37,6 @@ constexpr int kMetaRing = 8;
 // Prompt tokens of one slot that dec_prefill runs together as one step's rows.
 constexpr int kPrefillChunk = DEC_MAX_BATCH;
 constexpr int kMaxSplits = kAttnMaxSplits;
-// Most chains a decode step runs as (see run_step). Measured on B200: two free-running
-// chains C4 5.67 -> 5.40 and C5 7.21 -> 5.96 ms/step against two chains whose attentions
-// alternated; four chains C4 5.41, C5 6.19.
-constexpr int kMaxChains = 2;
 
 thread_local std::string g_create_error;
 // Allocation-failure injection for tests (dec_debug_fail_alloc): the n-th allocation of the
@@ -360,28 +357,12 @@ dec_status gemv(dec_handle* h, const GemvArgs& a, cudaStream_t st) {
     return DEC_OK;
 }
 
-// Batches of at least this many rows can take the tensor-core projection paths. Which
-// path runs also depends on the matrix (measured per shape on B200, PDL chains with
-// weights streamed from HBM): below about 2^21 weights with K < 2048 the tensor-core
+// Batches of at least kMmaMinBatch rows (chain_plan.h) can take the tensor-core projection
+// paths. Which path runs also depends on the matrix (measured per shape on B200, PDL chains
+// with weights streamed from HBM): below about 2^21 weights with K < 2048 the tensor-core
 // kernels' fixed cost (activation slice load, split-K exchange) is larger than the
 // CUDA-core kernel's whole run, except for int8 weights with f32 activations, whose
 // CUDA-core kernel is arithmetic-bound from batch 8 on.
-constexpr int kMmaMinBatch = 8;
-// Decode steps of this many rows or more run as chains (run_step, chain_bounds); each chain
-// has at least 8 rows, so each stays on the tensor-core paths.
-constexpr int kSplitMinBatch = 16;
-// Rows of each chain of a split step: equal multiples of 8 (every chain stays on the tensor-
-// core paths, which start at 8 rows), the last one taking the rest; r0[c] .. r0[c + 1] - 1 are
-// chain c's rows. Returns the chain count.
-inline int chain_bounds(int B, int* r0) {
-    int n = std::min(kMaxChains, B / kMmaMinBatch);
-    int base = (((B + n - 1) / n + kMmaMinBatch - 1) / kMmaMinBatch) * kMmaMinBatch;
-    n = (B + base - 1) / base;
-    if (B - base * (n - 1) < kMmaMinBatch) --n;   // a short last chain joins the one before
-    for (int c = 0; c < n; ++c) r0[c] = c * base;
-    r0[n] = B;
-    return n;
-}
 constexpr long long kMmaMinWeights = 1LL << 21;
 
 bool mma_worth(int N, int K, bool w8a32) {
