@@ -335,6 +335,8 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
     if (NORM_W) (void)mbar_try_wait(&bar_g, 0);
 
     // ---- per-row statistics from shared memory ----
+    // (the loops are unrolled so that several shared-memory loads are in flight; each lane
+    // still accumulates its elements in the same order)
     if (PRO != PRO_RAW_I8 && !producer) {
         for (int b = warp; b < BT; b += NWC) {
             float mu = 0.0f, rstd = 1.0f, inv = 0.0f, ascale = 0.0f;
@@ -345,12 +347,14 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
                 const int K4 = a.K >> 2;
                 if (PRO == PRO_LN) {
                     float sum = 0.0f;
+#pragma unroll 4
                     for (int k = lane; k < K4; k += 32) {
                         const float4 v = xr[k];
                         sum += (v.x + v.y) + (v.z + v.w);
                     }
                     mu = warp_sum(sum) / static_cast<float>(a.K);
                     float var = 0.0f;
+#pragma unroll 4
                     for (int k = lane; k < K4; k += 32) {
                         const float4 v = xr[k];
                         const float d0 = v.x - mu, d1 = v.y - mu, d2 = v.z - mu, d3 = v.w - mu;
@@ -363,6 +367,7 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
                     rstd = 1.0f / sqrtf(var + a.eps);
                 } else if (PRO == PRO_RMS) {
                     float ss = 0.0f;
+#pragma unroll 4
                     for (int k = lane; k < K4; k += 32) {
                         const float4 v = xr[k];
                         ss = fmaf(v.x, v.x, ss);
@@ -375,6 +380,7 @@ __global__ void __launch_bounds__(gemv_threads(BT), 2) k_gemv(const GemvArgs a, 
                 }
                 if (I8) {
                     float amax = 0.0f;
+#pragma unroll 4
                     for (int k = lane; k < K4; k += 32) {
                         const float4 v = xr[k];
                         float4 g = make_float4(1.f, 1.f, 1.f, 1.f), be = make_float4(0.f, 0.f, 0.f, 0.f);
